@@ -1,0 +1,268 @@
+"""SharQ's sparse-dense decomposition of one linear layer, step by step.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+Follows the xllm-io paper review of "SharQ: Bridging Activation Sparsity and
+FP4 Quantization for LLM Inference", section 3 (3.1 problem and group
+quantization, 3.2 sparse backbone, 3.3 dense residual, 3.4 dual-path GEMM,
+3.5 kernel design, 3.6 analysis), and the kasblo.com explainer (4:8 in-pairs,
+the residual w.r.t. the quantized backbone, one shared FP4 weight payload).
+
+Floating-point order.  Every float32 step is one IEEE float32 operation done
+in numpy float32 (round to nearest even); float64 is used where stated.  The
+pages fix none of these orders; the ones below are this library's reading and
+the GPU kernels follow the same order, which is what makes codes and scale
+bytes comparable bit for bit:
+
+  rmsnorm    ss = sum(x^2) in float64; inv = f32(1/sqrt(ss/K + eps)) in
+             float64 rounded once; xn = bf16(f32(f32(x*inv)*gamma)).
+  pts        s = f32(gmax / 2688) with 2688 = 6 (E2M1 max) * 448 (E4M3 max);
+             s = 1 when gmax = 0.
+  quantizer  per block: a = max|v|; sb = E4M3(f32(a / f32(6*s)));
+             S = f32(dec(sb)*s); inv = f32(1/S) or 0; code = E2M1(f32(v*inv)).
+  dequant    x~ = f32(val(code)*dec(sb)*s)   (val*dec is exact in float32).
+  residual   R = f32(xn - x~) at kept positions, R = xn elsewhere.
+"""
+import numpy as np
+
+from .formats import (bf16_round, e2m1_decode, e2m1_encode, e4m3_decode,
+                      e4m3_encode_nonneg, f32)
+
+E2M1_MAX = 6.0
+E4M3_MAX = 448.0
+GLOBAL_DIV = np.float32(E2M1_MAX * E4M3_MAX)   # 2688
+
+
+def rmsnorm(x, gamma, eps):
+    """RMSNorm fused into the preparation step (xllm-io review, section 3.5:
+    "RMSNorm/PTS + pair-topk mask + ... in one preparation kernel").
+
+    x: float32 [T, K] holding bf16 values.  gamma: float32 [K] (bf16 values) or
+    None for inputs that are not normalised (then xn = x).  Returns
+    (xn float32 [T, K] holding bf16 values, inv float32 [T] or None).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    if gamma is None:
+        return x.copy(), None
+    T, K = x.shape
+    ss = np.sum(x.astype(np.float64) ** 2, axis=1)
+    inv = (1.0 / np.sqrt(ss / K + np.float64(np.float32(eps)))).astype(np.float32)
+    t1 = (x * inv[:, None]).astype(np.float32)
+    t2 = (t1 * np.asarray(gamma, dtype=np.float32)[None, :]).astype(np.float32)
+    return bf16_round(t2), inv
+
+
+def pts_scale(xn):
+    """Per-tensor FP32 global scale computed online from the current tensor
+    (xllm-io review, sections 3.1 and 3.5, "PTS"; the kasblo.com explainer
+    notes SharQ needs no calibration data for it).
+
+    s = gmax / (6 * 448): maps the tensor amax onto the largest E2M1 value
+    times the largest E4M3 block scale.
+    """
+    gmax = np.float32(np.max(np.abs(xn))) if xn.size else np.float32(0)
+    if gmax == 0:
+        return np.float32(1.0), gmax
+    return np.float32(gmax / GLOBAL_DIV), gmax
+
+
+def pair_mask(xn):
+    """4:8 in-pairs mask (xllm-io review, section 3.2; kasblo.com explainer:
+    8 consecutive values form 4 pairs, keep 2 pairs = 4 values).
+
+    Pair score = max(|x_2p|, |x_2p+1|).  Keep the 2 highest scores; on equal
+    scores the lower pair index wins.  Pair p is kept iff fewer than 2 pairs q
+    beat it, where q beats p if s_q > s_p, or s_q == s_p and q < p.
+
+    Returns keep bool [T, K/8, 4] and meta uint8 [T, K/8] = p_lo | p_hi << 2.
+    """
+    T, K = xn.shape
+    a = np.abs(xn.reshape(T, K // 8, 4, 2))
+    s = np.max(a, axis=-1)                                     # [T, C, 4]
+    beats = np.zeros(s.shape + (4,), dtype=bool)               # [.., p, q]
+    for p in range(4):
+        for q in range(4):
+            if q == p:
+                continue
+            beats[..., p, q] = (s[..., q] > s[..., p]) | ((s[..., q] == s[..., p]) & (q < p))
+    keep = beats.sum(axis=-1) < 2
+    idx = np.argsort(~keep, axis=-1, kind="stable")[..., :2]   # kept, ascending
+    meta = (idx[..., 0] | (idx[..., 1] << 2)).astype(np.uint8)
+    return keep, meta
+
+
+def nvfp4_quant(v, s):
+    """Group-symmetric NVFP4 quantization of blocks (xllm-io review, section
+    3.1: s_G = max|x| / alpha_B, plus the second-level FP32 global scale s).
+
+    v: float32 [..., n] (one block per last axis).  s: float32 global scale.
+    Returns (codes uint8 [..., n], sb uint8 [...] E4M3 bytes, deq float32
+    [..., n] = f32(val * dec(sb) * s)).
+    """
+    v = np.asarray(v, dtype=np.float32)
+    s = np.float32(s)
+    a = np.max(np.abs(v), axis=-1)
+    denom = np.float32(np.float32(6.0) * s)
+    t = (a / denom).astype(np.float32)
+    sb = e4m3_encode_nonneg(t)
+    dec = e4m3_decode(sb).astype(np.float32)
+    S = (dec * s).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(S > 0, (np.float32(1.0) / S).astype(np.float32), np.float32(0.0))
+    y = (v * inv[..., None]).astype(np.float32)
+    codes = e2m1_encode(y)
+    vd = (e2m1_decode(codes) * dec[..., None].astype(np.float64))   # exact
+    deq = f32(vd * np.float64(s))
+    return codes, sb, deq
+
+
+def prep(x, gamma=None, eps=1e-5):
+    """The fused preparation step (xllm-io review, sections 3.2-3.5;
+    kasblo.com explainer, steps 1-3).
+
+    x: float32 [T, K] holding bf16 values, K a multiple of 32.
+    Returns a dict of logical (untiled) arrays:
+      xn [T,K], inv [T] or None, s_g, gmax,
+      keep [T,K/8,4], meta [T,K/8]           4:8 in-pairs mask
+      sp_vals [T,K/2]                         kept values, ascending K
+      sp_codes [T,K/2], sp_sf [T,K/32]        backbone NVFP4 (32 logical K/scale)
+      xsp [T,K], xsp_t [T,K]                  X_sp and dequantized X~_sp
+      r [T,K]                                 R = Xn - X~_sp (float32)
+      r_codes [T,K], r_sf [T,K/16], r_t [T,K] residual NVFP4 (16 K/scale)
+    """
+    xn, inv = rmsnorm(x, gamma, eps)
+    T, K = xn.shape
+    s_g, gmax = pts_scale(xn)
+    keep, meta = pair_mask(xn)
+    keep_el = np.repeat(keep, 2, axis=-1).reshape(T, K)               # [T,K]
+    xsp = np.where(keep_el, xn, np.float32(0)).astype(np.float32)
+    # compress: kept values of each chunk in ascending K order
+    sp_vals = xn[keep_el].reshape(T, K // 2)
+    # backbone: one scale per 32 logical K = 16 kept values
+    codes, sb, deq = nvfp4_quant(sp_vals.reshape(T, K // 32, 16), s_g)
+    sp_codes = codes.reshape(T, K // 2)
+    xsp_t = np.zeros((T, K), dtype=np.float32)
+    xsp_t[keep_el] = deq.reshape(-1)
+    # residual w.r.t. the quantized backbone (section 3.3)
+    r = np.where(keep_el, (xn - xsp_t).astype(np.float32), xn).astype(np.float32)
+    rc, rsb, rdeq = nvfp4_quant(r.reshape(T, K // 16, 16), s_g)
+    return dict(xn=xn, inv=inv, s_g=s_g, gmax=gmax, keep=keep, meta=meta,
+                sp_vals=sp_vals, sp_codes=sp_codes, sp_sf=sb, xsp=xsp,
+                xsp_t=xsp_t, r=r, r_codes=rc.reshape(T, K), r_sf=rsb,
+                r_t=rdeq.reshape(T, K))
+
+
+def pack_weight(w):
+    """Shared FP4 weight payload with two scale views (xllm-io review,
+    section 3.5: one FP4 weight body, sparse path group-32 scales, dense path
+    group-16 scales duplicated; kasblo.com explainer, step 3).
+
+    w: float32 [K, D] holding bf16 values (W in R^{K x D}, section 3.1).
+    Quantized per output column d along K with one scale per 32 K.
+    Returns dict: codes [D,K] (E2M1 codes), sf32 [D,K/32], sf16 [D,K/16]
+    (each sf32 byte twice), s_w, w_t [K,D] dequantized float64 without s_w,
+    i.e. val*dec(sb).
+    """
+    w = np.asarray(w, dtype=np.float32)
+    K, D = w.shape
+    amax = np.float32(np.max(np.abs(w))) if w.size else np.float32(0)
+    s_w = np.float32(1.0) if amax == 0 else np.float32(amax / GLOBAL_DIV)
+    wt = np.ascontiguousarray(w.T)                                     # [D,K]
+    codes, sb, _ = nvfp4_quant(wt.reshape(D, K // 32, 32), s_w)
+    codes = codes.reshape(D, K)
+    sf16 = np.repeat(sb, 2, axis=-1)
+    w_t = (e2m1_decode(codes).reshape(D, K // 32, 32)
+           * e4m3_decode(sb)[..., None]).reshape(D, K).T
+    return dict(codes=codes, sf32=sb, sf16=sf16, s_w=s_w, w_t=np.ascontiguousarray(w_t))
+
+
+def dequant_sparse(p):
+    """val(code)*dec(sb) of the backbone, scattered to [T,K], float64."""
+    T, K = p["xn"].shape
+    vals = (e2m1_decode(p["sp_codes"]).reshape(T, K // 32, 16)
+            * e4m3_decode(p["sp_sf"])[..., None]).reshape(T, K // 2)
+    keep_el = np.repeat(p["keep"], 2, axis=-1).reshape(T, K)
+    out = np.zeros((T, K), dtype=np.float64)
+    out[keep_el] = vals.reshape(-1)
+    return out
+
+
+def dequant_residual(p):
+    """val(code)*dec(sb) of the residual, [T,K], float64."""
+    T, K = p["xn"].shape
+    return (e2m1_decode(p["r_codes"]).reshape(T, K // 16, 16)
+            * e4m3_decode(p["r_sf"])[..., None]).reshape(T, K)
+
+
+def linear(p, wq):
+    """Dual-path GEMM of section 3.4 in float64 from the dequantized operands:
+
+        Y = GEMM_sp(Q_sp(X_sp), Q_w,sp(W)) + GEMM_dn(Q_dn(R), Q_w,dn(W))
+
+    Both GEMMs read the same weight codes; the sparse one through the
+    per-32 scales and the dense one through the per-16 view (equal values).
+    The global scales s_g * s_w multiply the sum (one accumulator).
+    Returns float64 [T, D].
+    """
+    a_sp = dequant_sparse(p)
+    a_dn = dequant_residual(p)
+    w32 = wq["w_t"]
+    K, D = w32.shape
+    w16 = (e2m1_decode(wq["codes"]).reshape(D, K // 16, 16)
+           * e4m3_decode(wq["sf16"])[..., None]).reshape(D, K).T
+    y = a_sp @ w32 + a_dn @ w16
+    return y * (np.float64(p["s_g"]) * np.float64(wq["s_w"]))
+
+
+def epilogue_f32(y64, s_g, s_w):
+    """Output rounding for the float32 output mode: the scaled float64
+    product rounded to float32 (the reference the float32 output is compared
+    against)."""
+    return f32(y64)
+
+
+def linear_grouped(p, wqs, offsets):
+    """Grouped form for MoE expert linears (xllm-io review, section 5.1: SharQ
+    applies to the expert linear layers of Qwen3-30B-A3B).
+
+    p: prep() of the whole expert-sorted activation tensor (one PTS scale for
+    the tensor).  wqs: pack_weight() per expert.  offsets: int [E+1], rows
+    offsets[e]:offsets[e+1] belong to expert e.  Returns float64 [rows, D].
+    """
+    T = p["xn"].shape[0]
+    D = wqs[0]["w_t"].shape[1]
+    y = np.zeros((T, D), dtype=np.float64)
+    for e, wq in enumerate(wqs):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi <= lo:
+            continue
+        sub = {k: (v[lo:hi] if isinstance(v, np.ndarray) and v.ndim >= 1
+                   and v.shape[0] == T else v) for k, v in p.items()}
+        y[lo:hi] = linear(sub, wq)
+    return y
+
+
+def prep_nvfp4(x, gamma=None, eps=1e-5):
+    """Plain NVFP4 preparation, the comparator the SharQ evaluation reports
+    as "NVFP4" (xllm-io review, Table 1; the kasblo.com explainer lists the
+    official repository's NVFP4 mode): RMSNorm, the same PTS global scale, and
+    every 16-element block of Xn quantized directly, with no mask and no
+    residual.  Returns dict xn, inv, s_g, gmax, codes [T,K], sf [T,K/16],
+    x_t [T,K] (dequantized, float32)."""
+    xn, inv = rmsnorm(x, gamma, eps)
+    T, K = xn.shape
+    s_g, gmax = pts_scale(xn)
+    c, sb, deq = nvfp4_quant(xn.reshape(T, K // 16, 16), s_g)
+    return dict(xn=xn, inv=inv, s_g=s_g, gmax=gmax, codes=c.reshape(T, K),
+                sf=sb, x_t=deq.reshape(T, K))
+
+
+def linear_nvfp4(p, wq):
+    """Dense NVFP4 GEMM of the plain-NVFP4 comparator in float64."""
+    T, K = p["xn"].shape
+    a = (e2m1_decode(p["codes"]).reshape(T, K // 16, 16)
+         * e4m3_decode(p["sf"])[..., None]).reshape(T, K)
+    D = wq["w_t"].shape[1]
+    w16 = (e2m1_decode(wq["codes"]).reshape(D, K // 16, 16)
+           * e4m3_decode(wq["sf16"])[..., None]).reshape(D, K).T
+    return (a @ w16) * (np.float64(p["s_g"]) * np.float64(wq["s_w"]))
