@@ -1,0 +1,264 @@
+// api.cu - the extern "C" boundary declared in include/sharq.h.
+//
+// Host-side only: size queries, carving caller-owned buffers into views,
+// argument / shape / architecture checks, and the kernel launches of
+// prep.cu, pack_weight.cu and gemm.cu.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sharq.h"
+#include "sharq_device.cuh"
+
+namespace sharq {
+cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp, int K,
+                        bool sharq_mode, float* inv_rms, float* s_g, unsigned int* gmax_bits, uint8_t* sp_codes,
+                        uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, cudaStream_t stream);
+cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf32, uint8_t* sf16,
+                               float* s_w, unsigned int* amax_bits, cudaStream_t stream);
+cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
+                          const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
+                          const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
+                          int D, int E, const int* group_offsets, void* Y, int out_f32, int* err,
+                          cudaStream_t stream);
+}  // namespace sharq
+
+namespace {
+
+constexpr int kMaxT = 1 << 22;
+constexpr int kMaxK = 1 << 17;
+constexpr int kMaxD = 1 << 18;
+constexpr int kMaxE = 4096;
+constexpr size_t kAlign = 256;
+constexpr size_t kWsBytes = 256;  // error word + reserved
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool shape_ok_k(int K) { return K > 0 && K <= kMaxK && K % 256 == 0; }
+bool shape_ok_d(int D) { return D > 0 && D <= kMaxD && D % 128 == 0; }
+bool shape_ok_t(int T) { return T >= 0 && T <= kMaxT; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// layout sizes, shared by the *_bytes and *_view functions
+struct ActLayout {
+  size_t r_codes, r_sf, sp_codes, meta, sp_sf, inv, scal, total;
+};
+ActLayout act_layout(int T, int K, int mode) {
+  ActLayout L{};
+  const size_t Tp = round_up((size_t)T, 128);
+  const size_t tiles = (Tp / 128) * (size_t)(K / 256);
+  size_t off = 0;
+  L.r_codes = off; off += tiles * sharq::kCodesTile;
+  L.r_sf = off;    off += tiles * sharq::kSf16Tile;
+  L.sp_codes = off;
+  if (mode == SHARQ_MODE_SHARQ) off += tiles * sharq::kSpTile;
+  L.meta = off;
+  if (mode == SHARQ_MODE_SHARQ) off += tiles * sharq::kMetaTile;
+  L.sp_sf = off;
+  if (mode == SHARQ_MODE_SHARQ) off += tiles * sharq::kSf32Tile;
+  L.inv = off;     off = round_up(off + Tp * sizeof(float), kAlign);
+  L.scal = off;    off += kAlign;  // s_g, gmax_bits
+  L.total = off;
+  return L;
+}
+
+struct WeightLayout {
+  size_t codes, sf32, sf16, s_w, scratch, total;
+};
+WeightLayout weight_layout(int K, int D, int E) {
+  WeightLayout L{};
+  const size_t tiles = (size_t)E * (D / 128) * (K / 256);
+  size_t off = 0;
+  L.codes = off; off += tiles * sharq::kCodesTile;
+  L.sf32 = off;  off += tiles * sharq::kSf32Tile;
+  L.sf16 = off;  off += tiles * sharq::kSf16Tile;
+  L.s_w = off;   off = round_up(off + (size_t)E * sizeof(float), kAlign);
+  L.scratch = off; off = round_up(off + (size_t)E * sizeof(unsigned), kAlign);
+  L.total = off;
+  return L;
+}
+
+int check_device() {
+  static int cached[64] = {};  // 0 unknown, 1 ok, -1 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
+  if (dev < 64 && cached[dev]) return cached[dev] > 0 ? SHARQ_OK : SHARQ_ERR_ARCH;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SHARQ_ERR_CUDA;
+  const bool ok = (major == 10 && minor == 0);
+  if (dev < 64) cached[dev] = ok ? 1 : -1;
+  return ok ? SHARQ_OK : SHARQ_ERR_ARCH;
+}
+
+int act_ok(const sharq_act* a) {
+  if (!a) return SHARQ_ERR_INVALID_ARG;
+  if (!shape_ok_t(a->T) || !shape_ok_k(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (a->mode != SHARQ_MODE_SHARQ && a->mode != SHARQ_MODE_NVFP4) return SHARQ_ERR_INVALID_ARG;
+  if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
+  if (!a->r_codes || !a->r_sf || !a->inv_rms || !a->s_g || !a->gmax_bits) return SHARQ_ERR_INVALID_ARG;
+  if (a->mode == SHARQ_MODE_SHARQ && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf};
+  for (const void* q : p)
+    if (q && !aligned(q, 16)) return SHARQ_ERR_INVALID_ARG;
+  return SHARQ_OK;
+}
+
+int weight_ok(const sharq_weight* w) {
+  if (!w) return SHARQ_ERR_INVALID_ARG;
+  if (!shape_ok_k(w->K) || !shape_ok_d(w->D) || w->E < 1 || w->E > kMaxE) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (!w->codes || !w->sf32 || !w->sf16 || !w->s_w) return SHARQ_ERR_INVALID_ARG;
+  if (!aligned(w->codes, 16) || !aligned(w->sf32, 16) || !aligned(w->sf16, 16)) return SHARQ_ERR_INVALID_ARG;
+  return SHARQ_OK;
+}
+
+int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* w, void* d_Y, int out_dtype,
+                  void* d_ws, size_t ws_bytes, sharq_stream_t stream, bool grouped) {
+  int st = act_ok(a);
+  if (st) return st;
+  if ((st = weight_ok(w))) return st;
+  if (a->K != w->K) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (!grouped && w->E != 1) return SHARQ_ERR_INVALID_ARG;
+  if (grouped && !d_offsets) return SHARQ_ERR_INVALID_ARG;
+  if (out_dtype != SHARQ_OUT_BF16 && out_dtype != SHARQ_OUT_F32) return SHARQ_ERR_INVALID_ARG;
+  if (a->T > 0 && (!d_Y || !aligned(d_Y, 16))) return SHARQ_ERR_INVALID_ARG;
+  if (!d_ws || ws_bytes < sharq_workspace_bytes(a->T, a->K, w->D, w->E) || !aligned(d_ws, 16))
+    return SHARQ_ERR_WORKSPACE;
+  if ((st = check_device())) return st;
+  cudaError_t e = sharq::launch_linear(
+      static_cast<const uint8_t*>(a->sp_codes), static_cast<const uint8_t*>(a->meta),
+      static_cast<const uint8_t*>(a->sp_sf), static_cast<const uint8_t*>(a->r_codes),
+      static_cast<const uint8_t*>(a->r_sf), a->s_g, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ ? 1 : 0,
+      static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
+      static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
+      out_dtype == SHARQ_OUT_F32 ? 1 : 0, static_cast<int*>(d_ws), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sharq_abi_version(void) { return SHARQ_ABI_VERSION; }
+
+const char* sharq_status_string(int status) {
+  switch (status) {
+    case SHARQ_OK: return "SHARQ_OK";
+    case SHARQ_ERR_INVALID_ARG: return "SHARQ_ERR_INVALID_ARG";
+    case SHARQ_ERR_UNSUPPORTED_SHAPE: return "SHARQ_ERR_UNSUPPORTED_SHAPE";
+    case SHARQ_ERR_ARCH: return "SHARQ_ERR_ARCH";
+    case SHARQ_ERR_CUDA: return "SHARQ_ERR_CUDA";
+    case SHARQ_ERR_TIMEOUT: return "SHARQ_ERR_TIMEOUT";
+    case SHARQ_ERR_WORKSPACE: return "SHARQ_ERR_WORKSPACE";
+    default: return "SHARQ_ERR_UNKNOWN";
+  }
+}
+
+size_t sharq_weight_bytes(int K, int D, int E) {
+  if (!shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return 0;
+  return weight_layout(K, D, E).total;
+}
+
+size_t sharq_act_bytes(int T, int K, int mode) {
+  if (!shape_ok_t(T) || !shape_ok_k(K)) return 0;
+  if (mode != SHARQ_MODE_SHARQ && mode != SHARQ_MODE_NVFP4) return 0;
+  return act_layout(T, K, mode).total;
+}
+
+size_t sharq_workspace_bytes(int T, int K, int D, int E) {
+  if (!shape_ok_t(T) || !shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return 0;
+  return kWsBytes;
+}
+
+int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {
+  if (!d_buf || !out) return SHARQ_ERR_INVALID_ARG;
+  if (!shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(d_buf, kAlign)) return SHARQ_ERR_INVALID_ARG;
+  const WeightLayout L = weight_layout(K, D, E);
+  uint8_t* b = static_cast<uint8_t*>(d_buf);
+  out->codes = b + L.codes;
+  out->sf32 = b + L.sf32;
+  out->sf16 = b + L.sf16;
+  out->s_w = reinterpret_cast<float*>(b + L.s_w);
+  out->K = K;
+  out->D = D;
+  out->E = E;
+  return SHARQ_OK;
+}
+
+int sharq_act_view(void* d_buf, int T, int K, int mode, sharq_act* out) {
+  if (!d_buf || !out) return SHARQ_ERR_INVALID_ARG;
+  if (!shape_ok_t(T) || !shape_ok_k(K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (mode != SHARQ_MODE_SHARQ && mode != SHARQ_MODE_NVFP4) return SHARQ_ERR_INVALID_ARG;
+  if (!aligned(d_buf, kAlign)) return SHARQ_ERR_INVALID_ARG;
+  const ActLayout L = act_layout(T, K, mode);
+  uint8_t* b = static_cast<uint8_t*>(d_buf);
+  const bool sq = mode == SHARQ_MODE_SHARQ;
+  out->r_codes = b + L.r_codes;
+  out->r_sf = b + L.r_sf;
+  out->sp_codes = sq ? b + L.sp_codes : nullptr;
+  out->meta = sq ? b + L.meta : nullptr;
+  out->sp_sf = sq ? b + L.sp_sf : nullptr;
+  out->inv_rms = reinterpret_cast<float*>(b + L.inv);
+  out->s_g = reinterpret_cast<float*>(b + L.scal);
+  out->gmax_bits = reinterpret_cast<unsigned int*>(b + L.scal + 16);
+  out->T = T;
+  out->Tp = (int)round_up((size_t)T, 128);
+  out->K = K;
+  out->mode = mode;
+  return SHARQ_OK;
+}
+
+int sharq_pack_weight(const void* d_W, const sharq_weight* w, sharq_stream_t stream) {
+  int st = weight_ok(w);
+  if (st) return st;
+  if (!d_W || !aligned(d_W, 2)) return SHARQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  const WeightLayout L = weight_layout(w->K, w->D, w->E);
+  unsigned int* scratch = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(w->s_w) + (L.scratch - L.s_w));
+  cudaError_t e = sharq::launch_pack_weight(d_W, w->K, w->D, w->E, static_cast<uint8_t*>(w->codes),
+                                            static_cast<uint8_t*>(w->sf32), static_cast<uint8_t*>(w->sf16), w->s_w,
+                                            scratch, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
+}
+
+int sharq_prep(const void* d_X, const void* d_gamma, float eps, const int* d_row_index, const sharq_act* a,
+               sharq_stream_t stream) {
+  int st = act_ok(a);
+  if (st) return st;
+  if (a->T > 0 && (!d_X || !aligned(d_X, 16))) return SHARQ_ERR_INVALID_ARG;
+  if (d_gamma && !aligned(d_gamma, 16)) return SHARQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return SHARQ_ERR_INVALID_ARG;
+  if ((st = check_device())) return st;
+  cudaError_t e = sharq::launch_prep(
+      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ, a->inv_rms, a->s_g,
+      a->gmax_bits, static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta),
+      static_cast<uint8_t*>(a->sp_sf), static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf),
+      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
+}
+
+int sharq_linear(const sharq_act* a, const sharq_weight* w, void* d_Y, int out_dtype, void* d_ws, size_t ws_bytes,
+                 sharq_stream_t stream) {
+  return linear_common(a, nullptr, w, d_Y, out_dtype, d_ws, ws_bytes, stream, false);
+}
+
+int sharq_linear_grouped(const sharq_act* a, const int* d_group_offsets, const sharq_weight* w, void* d_Y,
+                         int out_dtype, void* d_ws, size_t ws_bytes, sharq_stream_t stream) {
+  return linear_common(a, d_group_offsets, w, d_Y, out_dtype, d_ws, ws_bytes, stream, true);
+}
+
+int sharq_check_status(void* d_ws, sharq_stream_t stream) {
+  if (!d_ws) return SHARQ_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, d_ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return SHARQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SHARQ_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(d_ws, 0, sizeof(int), s) != cudaSuccess) return SHARQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SHARQ_ERR_CUDA;
+  }
+  return word;
+}
+
+}  // extern "C"

@@ -1,0 +1,344 @@
+// gemm.cu - sharq_linear / sharq_linear_grouped: the dual-path FP4 GEMM.
+//
+// xllm-io review of SharQ, section 3.4:
+//   Y = GEMM_sp(Q_sp(X_sp), Q_w,sp(W)) + GEMM_dn(Q_dn(R), Q_w,dn(W))
+// and section 3.5 ("residual accumulation: the dense branch accumulates
+// directly into the sparse branch's output, no second full branch is
+// materialised"; "shared FP4 weight payload ... path-specific scale views").
+//
+// B200 design (one CTA per 128 x BN output tile, warp-specialised):
+//   warp 0      producer: per 256-K stage, bulk copies (TMA engine) of the
+//               pre-tiled operands -- backbone codes, metadata, residual
+//               codes, their scales, the weight codes and both weight scale
+//               views -- into a STAGES-deep shared-memory ring, completion
+//               tracked by mbarrier transaction bytes.
+//   warp 1      TMEM allocation; one elected thread issues, per stage:
+//               tcgen05.cp of metadata and scale factors into TMEM, 2 sparse
+//               block-scaled FP4 MMAs (tcgen05.mma.sp kind::mxf4nvf4, K=128
+//               logical each, one scale per 32 logical K) and 4 dense ones
+//               (kind::mxf4nvf4 block16, K=64 each), all into ONE fp32 TMEM
+//               accumulator and all reading the SAME weight tile in shared
+//               memory; tcgen05.commit releases the stage.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per thread),
+//               y = f32(acc * f32(s_g * s_w)), bf16 or fp32 stores.
+// Every wait is bounded by the global timer; on timeout the CTA records
+// SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
+#include "sharq_device.cuh"
+
+namespace sharq {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far beyond any tile's work
+constexpr int kErrTimeout = -5;
+constexpr int kErrInvalid = -1;
+
+struct GemmArgs {
+  const uint8_t* a_sp;
+  const uint8_t* a_meta;
+  const uint8_t* a_spsf;
+  const uint8_t* a_r;
+  const uint8_t* a_rsf;
+  const float* s_g;
+  const uint8_t* w_codes;
+  const uint8_t* w_sf32;
+  const uint8_t* w_sf16;
+  const float* s_w;
+  void* Y;
+  const int* group_offsets;  // device [E+1] or nullptr
+  int* err;                  // workspace error word or nullptr
+  int T, K, D, E;
+  int out_f32;
+  int sharq_mode;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int kHalves = BN / 128;
+  static constexpr int kStages = BN == 256 ? 3 : 4;
+  // shared-memory stage layout (bytes); 1024-aligned where a swizzle needs it
+  static constexpr int kOffB = 0;
+  static constexpr int kOffAR = kOffB + BN * 128;
+  static constexpr int kOffASP = kOffAR + kCodesTile;
+  static constexpr int kOffE = kOffASP + kSpTile;
+  static constexpr int kOffSFASP = kOffE + kMetaTile;
+  static constexpr int kOffSFAR = kOffSFASP + kSf32Tile;
+  static constexpr int kOffSFB32 = kOffSFAR + kSf16Tile;
+  static constexpr int kOffSFB16 = kOffSFB32 + kHalves * kSf32Tile;
+  static constexpr int kStageBytes = kOffSFB16 + kHalves * kSf16Tile;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  // TMEM columns
+  static constexpr uint32_t kColAcc = 0;
+  static constexpr uint32_t kColE = BN;
+  static constexpr uint32_t kColSFASP = BN + 8;
+  static constexpr uint32_t kColSFAR = BN + 16;
+  static constexpr uint32_t kSfbCols = BN / 32;  // per MMA: one column per 32 rows of B
+  static constexpr uint32_t kColSFB32 = BN + 32;
+  static constexpr uint32_t kColSFB16 = kColSFB32 + 2 * kSfbCols;
+  static constexpr uint32_t kColsUsed = kColSFB16 + 4 * kSfbCols;
+  static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256 : 512;
+  // transaction bytes per stage
+  static constexpr uint32_t kTxSharq = BN * 128 + kHalves * (kSf32Tile + kSf16Tile) + kCodesTile + kSpTile +
+                                       kMetaTile + kSf32Tile + kSf16Tile;
+  static constexpr uint32_t kTxNvfp4 = BN * 128 + kHalves * kSf16Tile + kCodesTile + kSf16Tile;
+  static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kColsUsed <= 512, "TMEM overflow");
+};
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::kStages];
+  __shared__ __align__(8) uint64_t empty_bar[C::kStages];
+  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+  __shared__ int expert_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nt = blockIdx.x, mt = blockIdx.y;
+  const int KS = args.K >> 8;
+  const int NB = args.D >> 7;
+  const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_bar, 1);
+    fence_mbar_init();
+    abort_sh = 0;
+    // expert of this m-tile (grouped form): offsets are 128-row aligned
+    int e = 0;
+    if (args.group_offsets) {
+      const int row0 = mt * 128;
+      e = -1;
+      int lo = 0, hi = args.E - 1;
+      while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        if (args.group_offsets[mid] <= row0) { e = mid; lo = mid + 1; } else { hi = mid - 1; }
+      }
+      // skip empty groups that share this start
+      while (e >= 0 && e < args.E && args.group_offsets[e + 1] <= row0) ++e;
+      if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
+    }
+    expert_sh = e;
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int expert = expert_sh;
+  if (expert < 0) {
+    if (threadIdx.x == 0) record_error(args.err, kErrInvalid);
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+    return;
+  }
+  const bool sharq = args.sharq_mode != 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- producer ----
+    if (lane == 0) {
+      const size_t a_tile0 = (size_t)mt * KS;
+      const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
+      for (int ks = 0; ks < KS; ++ks) {
+        const int s = ks % C::kStages;
+        if (ks >= C::kStages) {
+          if (!mbar_wait(&empty_bar[s], ((ks / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+        }
+        uint8_t* st = smem + s * C::kStageBytes;
+        uint64_t* fb = &full_bar[s];
+        mbar_arrive_expect_tx(fb, sharq ? C::kTxSharq : C::kTxNvfp4);
+        const size_t at = a_tile0 + ks;
+#pragma unroll
+        for (int h = 0; h < C::kHalves; ++h) {
+          const size_t bt = b_tile0 + (size_t)h * KS + ks;
+          bulk_g2s(st + C::kOffB + h * kCodesTile, args.w_codes + bt * kCodesTile, kCodesTile, fb);
+          bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, fb);
+          if (sharq) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
+        }
+        bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, kCodesTile, fb);
+        bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
+        if (sharq) {
+          bulk_g2s(st + C::kOffASP, args.a_sp + at * kSpTile, kSpTile, fb);
+          bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, kMetaTile, fb);
+          bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_dn = idesc_nvf4(128, BN, false);
+      constexpr uint32_t idesc_sp = idesc_nvf4(128, BN, true);
+      for (int ks = 0; ks < KS; ++ks) {
+        const int s = ks % C::kStages;
+        if (!mbar_wait(&full_bar[s], (ks / C::kStages) & 1, deadline, &abort_sh)) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+        // scale factors (and metadata) shared memory -> TMEM
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tc_cp_32x128b_x4(tmem + C::kColSFAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h)
+            tc_cp_32x128b_x4(tmem + C::kColSFB16 + j * C::kSfbCols + 4 * h,
+                             smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
+        if (sharq) {
+          tc_cp_128x128b(tmem + C::kColE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tc_cp_32x128b_x4(tmem + C::kColSFASP + 4 * j,
+                             smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              tc_cp_32x128b_x4(tmem + C::kColSFB32 + j * C::kSfbCols + 4 * h,
+                               smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
+          // sparse backbone: 2 x (128 x BN x 128 logical K)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffASP + 32 * j, 16, 512, kSw64),
+                        smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), tmem + C::kColE + 2 * j, idesc_sp,
+                        tmem + C::kColSFASP + 4 * j, tmem + C::kColSFB32 + j * C::kSfbCols,
+                        (ks > 0 || j > 0) ? 1u : 0u);
+        }
+        // dense residual: 4 x (128 x BN x 64 K), same accumulator, same B tile
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffAR + 32 * j, 16, 1024, kSw128),
+                   smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, tmem + C::kColSFAR + 4 * j,
+                   tmem + C::kColSFB16 + j * C::kSfbCols, (sharq || ks > 0 || j > 0) ? 1u : 0u);
+        tc_commit(&empty_bar[s]);
+      }
+      tc_commit(&acc_bar);  // accumulator complete (or everything issued so far, on abort)
+    }
+  } else {
+    // ------------------------------------------------------- epilogue ----
+    const int sp = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = mt * 128 + sp * 32 + lane;
+    const bool ok = mbar_wait(&acc_bar, 0, deadline, &abort_sh);
+    tc_fence_after();
+    if (!ok) {
+      record_error(args.err, kErrTimeout);
+      abort_sh = 1;
+    } else {
+      const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
+      const int col0 = nt * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+        tmem_ld_wait();
+        if (row < args.T) {
+          if (args.out_f32) {
+            float* y = static_cast<float*>(args.Y) + (size_t)row * args.D + col0 + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(y + i) =
+                  make_float4(__fmul_rn(__uint_as_float(v[i]), scale), __fmul_rn(__uint_as_float(v[i + 1]), scale),
+                              __fmul_rn(__uint_as_float(v[i + 2]), scale),
+                              __fmul_rn(__uint_as_float(v[i + 3]), scale));
+          } else {
+            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.Y) + (size_t)row * args.D + col0 + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 pk;
+              uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[i + 2 * k]), scale),
+                                                          __fmul_rn(__uint_as_float(v[i + 2 * k + 1]), scale));
+                w[k] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(y + i) = pk;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
+  using C = Cfg<BN>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(sharq_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(a.D / BN, m_tiles);
+  sharq_gemm_kernel<BN><<<grid, kThreads, C::kSmemBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
+                          const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
+                          const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
+                          int D, int E, const int* group_offsets, void* Y, int out_f32, int* err,
+                          cudaStream_t stream) {
+  GemmArgs a;
+  a.a_sp = a_sp;
+  a.a_meta = a_meta;
+  a.a_spsf = a_spsf;
+  a.a_r = a_r;
+  a.a_rsf = a_rsf;
+  a.s_g = s_g;
+  a.w_codes = w_codes;
+  a.w_sf32 = w_sf32;
+  a.w_sf16 = w_sf16;
+  a.s_w = s_w;
+  a.Y = Y;
+  a.group_offsets = group_offsets;
+  a.err = err;
+  a.T = T;
+  a.K = K;
+  a.D = D;
+  a.E = E;
+  a.out_f32 = out_f32;
+  a.sharq_mode = sharq_mode;
+  const int m_tiles = Tp / 128;
+  if (m_tiles == 0) return cudaSuccess;
+  if (D % 256 == 0) return launch_bn<256>(a, m_tiles, stream);
+  return launch_bn<128>(a, m_tiles, stream);
+}
+
+}  // namespace sharq
