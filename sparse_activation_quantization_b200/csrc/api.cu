@@ -18,8 +18,8 @@ cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* code
 cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
-                          int D, int E, const int* group_offsets, void* Y, int out_f32, int* err,
-                          cudaStream_t stream);
+                          int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
+                          int* err, int* tile_count, float* partial, cudaStream_t stream);
 }  // namespace sharq
 
 namespace {
@@ -29,7 +29,8 @@ constexpr int kMaxK = 1 << 17;
 constexpr int kMaxD = 1 << 18;
 constexpr int kMaxE = 4096;
 constexpr size_t kAlign = 256;
-constexpr size_t kWsBytes = 256;  // error word + reserved
+constexpr size_t kWsHeader = 256;  // error word + reserved
+constexpr int kTargetCtas = 148;   // B200 SM count: one GEMM CTA per SM
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -74,6 +75,47 @@ WeightLayout weight_layout(int K, int D, int E) {
   L.s_w = off;   off = round_up(off + (size_t)E * sizeof(float), kAlign);
   L.scratch = off; off = round_up(off + (size_t)E * sizeof(unsigned), kAlign);
   L.total = off;
+  return L;
+}
+
+// GEMM launch shape for a problem: tile width BN and the number of K splits.
+// Prefill shapes have enough output tiles to fill the GPU (BN = 256, no
+// split).  Decode shapes split K so that about one CTA per SM streams a slice
+// of the weight; the fp32 partials cost 8 bytes (write + read) per output
+// element per split, so the split count is also capped to keep that traffic
+// well below the weight bytes (0.59375 B per weight element).
+struct GemmShape {
+  int bn, splits, m_tiles, n_tiles;
+};
+GemmShape gemm_shape(int T, int K, int D, int E) {
+  GemmShape g{};
+  const int Tp = (int)round_up((size_t)T, 128);
+  g.m_tiles = Tp / 128;
+  const int KS = K / 256;
+  const bool wide = (D % 256 == 0) && (long long)g.m_tiles * (D / 256) >= kTargetCtas;
+  g.bn = wide ? 256 : 128;
+  g.n_tiles = D / g.bn;
+  g.splits = 1;
+  const long long mn = (long long)g.m_tiles * g.n_tiles;
+  if (E == 1 && mn > 0 && mn < kTargetCtas / 2) {
+    int s = (int)(kTargetCtas / mn);
+    const int cap = (int)(0.15 * K / (T > 0 ? T : 1));
+    s = s < cap ? s : cap;
+    s = s < KS ? s : KS;
+    g.splits = s > 1 ? s : 1;
+  }
+  return g;
+}
+
+struct WsLayout {
+  size_t counters, partial, total;
+};
+WsLayout ws_layout(int T, int K, int D, int E) {
+  const GemmShape g = gemm_shape(T, K, D, E);
+  WsLayout L{};
+  L.counters = kWsHeader;
+  L.partial = round_up(L.counters + (size_t)g.m_tiles * g.n_tiles * sizeof(int), kAlign);
+  L.total = L.partial + (g.splits > 1 ? (size_t)g.splits * T * D * sizeof(float) : 0);
   return L;
 }
 
@@ -122,16 +164,21 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
   if (grouped && !d_offsets) return SHARQ_ERR_INVALID_ARG;
   if (out_dtype != SHARQ_OUT_BF16 && out_dtype != SHARQ_OUT_F32) return SHARQ_ERR_INVALID_ARG;
   if (a->T > 0 && (!d_Y || !aligned(d_Y, 16))) return SHARQ_ERR_INVALID_ARG;
-  if (!d_ws || ws_bytes < sharq_workspace_bytes(a->T, a->K, w->D, w->E) || !aligned(d_ws, 16))
+  if (!d_ws || ws_bytes < sharq_workspace_bytes(a->T, a->K, w->D, grouped ? w->E : 1) || !aligned(d_ws, 16))
     return SHARQ_ERR_WORKSPACE;
   if ((st = check_device())) return st;
+  const GemmShape g = gemm_shape(a->T, a->K, w->D, grouped ? w->E : 1);
+  const WsLayout WL = ws_layout(a->T, a->K, w->D, grouped ? w->E : 1);
+  uint8_t* wsb = static_cast<uint8_t*>(d_ws);
   cudaError_t e = sharq::launch_linear(
       static_cast<const uint8_t*>(a->sp_codes), static_cast<const uint8_t*>(a->meta),
       static_cast<const uint8_t*>(a->sp_sf), static_cast<const uint8_t*>(a->r_codes),
       static_cast<const uint8_t*>(a->r_sf), a->s_g, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ ? 1 : 0,
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
-      out_dtype == SHARQ_OUT_F32 ? 1 : 0, static_cast<int*>(d_ws), reinterpret_cast<cudaStream_t>(stream));
+      out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, reinterpret_cast<int*>(wsb),
+      reinterpret_cast<int*>(wsb + WL.counters), reinterpret_cast<float*>(wsb + WL.partial),
+      reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 
@@ -167,7 +214,7 @@ size_t sharq_act_bytes(int T, int K, int mode) {
 
 size_t sharq_workspace_bytes(int T, int K, int D, int E) {
   if (!shape_ok_t(T) || !shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return 0;
-  return kWsBytes;
+  return ws_layout(T, K, D, E).total;
 }
 
 int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {

@@ -21,6 +21,11 @@
 //               memory; tcgen05.commit releases the stage.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per thread),
 //               y = f32(acc * f32(s_g * s_w)), bf16 or fp32 stores.
+// Split-K (decode shapes, where output tiles alone cannot fill 148 SMs):
+// blockIdx.z picks a contiguous range of K stages; each CTA writes its fp32
+// partial tile to the workspace, and the last CTA to arrive at a tile (one
+// atomic counter per tile, reset by that CTA) sums the partials in split
+// order -- deterministic -- and writes Y.
 // Every wait is bounded by the global timer; on timeout the CTA records
 // SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
 #include "sharq_device.cuh"
@@ -48,9 +53,12 @@ struct GemmArgs {
   void* Y;
   const int* group_offsets;  // device [E+1] or nullptr
   int* err;                  // workspace error word or nullptr
+  int* tile_count;           // split-K: arrivals per output tile (self-resetting)
+  float* partial;            // split-K: fp32 partial sums [splits][T][D]
   int T, K, D, E;
   int out_f32;
   int sharq_mode;
+  int splits;
 };
 
 template <int BN>
@@ -90,6 +98,50 @@ __device__ __forceinline__ void record_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// y = f32(acc * scale), 32 consecutive columns of one row, bf16 or fp32
+__device__ __forceinline__ void store_row32(void* Y, int out_f32, size_t off, const uint32_t (&v)[32], float scale) {
+  if (out_f32) {
+    float* y = static_cast<float*>(Y) + off;
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+      *reinterpret_cast<float4*>(y + i) =
+          make_float4(__fmul_rn(__uint_as_float(v[i]), scale), __fmul_rn(__uint_as_float(v[i + 1]), scale),
+                      __fmul_rn(__uint_as_float(v[i + 2]), scale), __fmul_rn(__uint_as_float(v[i + 3]), scale));
+  } else {
+    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + off;
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      uint4 pk;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[i + 2 * k]), scale),
+                                                  __fmul_rn(__uint_as_float(v[i + 2 * k + 1]), scale));
+        w[k] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(y + i) = pk;
+    }
+  }
+}
+
+__device__ __forceinline__ void store4(void* Y, int out_f32, size_t off, float4 a, float scale) {
+  const float x = __fmul_rn(a.x, scale), y = __fmul_rn(a.y, scale), z = __fmul_rn(a.z, scale),
+              w = __fmul_rn(a.w, scale);
+  if (out_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(Y) + off) = make_float4(x, y, z, w);
+  } else {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(x, y), hi = __floats2bfloat162_rn(z, w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(Y) + off) = pk;
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
   using C = Cfg<BN>;
@@ -100,11 +152,15 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
+  __shared__ int last_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = blockIdx.x, mt = blockIdx.y;
+  const int nt = blockIdx.x, mt = blockIdx.y, split = blockIdx.z;
   const int KS = args.K >> 8;
+  const int ks0 = (int)(((long long)split * KS) / args.splits);
+  const int ks1 = (int)(((long long)(split + 1) * KS) / args.splits);
+  const int nks = ks1 - ks0;
   const int NB = args.D >> 7;
   const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
 
@@ -154,10 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     if (lane == 0) {
       const size_t a_tile0 = (size_t)mt * KS;
       const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
-      for (int ks = 0; ks < KS; ++ks) {
-        const int s = ks % C::kStages;
-        if (ks >= C::kStages) {
-          if (!mbar_wait(&empty_bar[s], ((ks / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
+      for (int i = 0; i < nks; ++i) {
+        const int ks = ks0 + i;
+        const int s = i % C::kStages;
+        if (i >= C::kStages) {
+          if (!mbar_wait(&empty_bar[s], ((i / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
             record_error(args.err, kErrTimeout);
             abort_sh = 1;
             break;
@@ -188,9 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     if (lane == 0) {
       constexpr uint32_t idesc_dn = idesc_nvf4(128, BN, false);
       constexpr uint32_t idesc_sp = idesc_nvf4(128, BN, true);
-      for (int ks = 0; ks < KS; ++ks) {
-        const int s = ks % C::kStages;
-        if (!mbar_wait(&full_bar[s], (ks / C::kStages) & 1, deadline, &abort_sh)) {
+      for (int i = 0; i < nks; ++i) {
+        const int s = i % C::kStages;
+        if (!mbar_wait(&full_bar[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
           record_error(args.err, kErrTimeout);
           abort_sh = 1;
           break;
@@ -225,14 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
             mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffASP + 32 * j, 16, 512, kSw64),
                         smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), tmem + C::kColE + 2 * j, idesc_sp,
                         tmem + C::kColSFASP + 4 * j, tmem + C::kColSFB32 + j * C::kSfbCols,
-                        (ks > 0 || j > 0) ? 1u : 0u);
+                        (i > 0 || j > 0) ? 1u : 0u);
         }
         // dense residual: 4 x (128 x BN x 64 K), same accumulator, same B tile
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           mma_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffAR + 32 * j, 16, 1024, kSw128),
                    smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, tmem + C::kColSFAR + 4 * j,
-                   tmem + C::kColSFB16 + j * C::kSfbCols, (sharq || ks > 0 || j > 0) ? 1u : 0u);
+                   tmem + C::kColSFB16 + j * C::kSfbCols, (sharq || i > 0 || j > 0) ? 1u : 0u);
         tc_commit(&empty_bar[s]);
       }
       tc_commit(&acc_bar);  // accumulator complete (or everything issued so far, on abort)
@@ -249,35 +306,54 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     } else {
       const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
       const int col0 = nt * BN;
+      if (args.splits == 1) {
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
-        tmem_ld_wait();
-        if (row < args.T) {
-          if (args.out_f32) {
-            float* y = static_cast<float*>(args.Y) + (size_t)row * args.D + col0 + c;
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+          tmem_ld_wait();
+          if (row < args.T) store_row32(args.Y, args.out_f32, (size_t)row * args.D + col0 + c, v, scale);
+        }
+      } else {
+        // 1. this split's fp32 partial tile -> workspace (valid rows only)
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+          tmem_ld_wait();
+          if (row < args.T) {
+            float* dst = args.partial + ((size_t)split * args.T + row) * args.D + col0 + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(y + i) =
-                  make_float4(__fmul_rn(__uint_as_float(v[i]), scale), __fmul_rn(__uint_as_float(v[i + 1]), scale),
-                              __fmul_rn(__uint_as_float(v[i + 2]), scale),
-                              __fmul_rn(__uint_as_float(v[i + 3]), scale));
-          } else {
-            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.Y) + (size_t)row * args.D + col0 + c;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 pk;
-              uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[i + 2 * k]), scale),
-                                                          __fmul_rn(__uint_as_float(v[i + 2 * k + 1]), scale));
-                w[k] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              *reinterpret_cast<uint4*>(y + i) = pk;
-            }
+              __stcg(reinterpret_cast<float4*>(dst + i),
+                     make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                                 __uint_as_float(v[i + 3])));
           }
+        }
+        // 2. count arrivals at this tile; the last CTA reduces
+        __threadfence();
+        named_barrier_sync(1, 128);
+        const int tile_id = mt * gridDim.x + nt;
+        if (threadIdx.x == 64) last_sh = (atomicAdd(args.tile_count + tile_id, 1) == args.splits - 1);
+        named_barrier_sync(1, 128);
+        if (last_sh) {
+          __threadfence();
+          const int rows = min(128, args.T - mt * 128);
+          const int q4 = BN / 4;
+          for (int idx = threadIdx.x - 64; idx < rows * q4; idx += 128) {
+            const int r = idx / q4, c4 = idx - r * q4;
+            const size_t off = (size_t)(mt * 128 + r) * args.D + col0 + 4 * c4;
+            float4 acc = __ldcg(reinterpret_cast<const float4*>(args.partial + off));
+            for (int sp2 = 1; sp2 < args.splits; ++sp2) {
+              const float4 p = __ldcg(reinterpret_cast<const float4*>(args.partial + (size_t)sp2 * args.T * args.D + off));
+              acc.x = __fadd_rn(acc.x, p.x);
+              acc.y = __fadd_rn(acc.y, p.y);
+              acc.z = __fadd_rn(acc.z, p.z);
+              acc.w = __fadd_rn(acc.w, p.w);
+            }
+            store4(args.Y, args.out_f32, off, acc, scale);
+          }
+          if (threadIdx.x == 64) args.tile_count[tile_id] = 0;  // ready for the next call
         }
       }
     }
@@ -293,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
 
 template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
+  static_assert(BN == 128 || BN == 256, "tile width");
   using C = Cfg<BN>;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -303,7 +380,7 @@ cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(a.D / BN, m_tiles);
+  dim3 grid(a.D / BN, m_tiles, a.splits);
   sharq_gemm_kernel<BN><<<grid, kThreads, C::kSmemBytes, stream>>>(a);
   return cudaGetLastError();
 }
@@ -313,8 +390,8 @@ cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
 cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
-                          int D, int E, const int* group_offsets, void* Y, int out_f32, int* err,
-                          cudaStream_t stream) {
+                          int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
+                          int* err, int* tile_count, float* partial, cudaStream_t stream) {
   GemmArgs a;
   a.a_sp = a_sp;
   a.a_meta = a_meta;
@@ -329,16 +406,18 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.Y = Y;
   a.group_offsets = group_offsets;
   a.err = err;
+  a.tile_count = tile_count;
+  a.partial = partial;
   a.T = T;
   a.K = K;
   a.D = D;
   a.E = E;
   a.out_f32 = out_f32;
   a.sharq_mode = sharq_mode;
+  a.splits = splits;
   const int m_tiles = Tp / 128;
   if (m_tiles == 0) return cudaSuccess;
-  if (D % 256 == 0) return launch_bn<256>(a, m_tiles, stream);
-  return launch_bn<128>(a, m_tiles, stream);
+  return bn == 256 ? launch_bn<256>(a, m_tiles, stream) : launch_bn<128>(a, m_tiles, stream);
 }
 
 }  // namespace sharq
