@@ -115,7 +115,9 @@ typedef struct {
  *            values), atom layout as weight sf32.
  *   inv_rms: Tp floats (1/rms per row; 1 when RMSNorm is off).
  *   s_g:     the per-tensor global scale gmax / (6*448) (1 if gmax == 0).
- *   gmax_bits: scratch for the device-wide amax.
+ *   gmax_bits: 16 bytes of scratch: device-wide amax, grid-barrier count,
+ *            reserved, and an error word that sharq_linear forwards to its
+ *            workspace (a prep whose grid barrier timed out).
  */
 typedef struct {
   void *sp_codes;

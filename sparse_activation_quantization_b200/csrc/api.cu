@@ -19,7 +19,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
-                          int* err, int* tile_count, float* partial, cudaStream_t stream);
+                          int* err, const int* act_err, int* tile_count, float* partial, cudaStream_t stream);
 }  // namespace sharq
 
 namespace {
@@ -177,7 +177,7 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
       out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, reinterpret_cast<int*>(wsb),
-      reinterpret_cast<int*>(wsb + WL.counters), reinterpret_cast<float*>(wsb + WL.partial),
+      reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<int*>(wsb + WL.counters), reinterpret_cast<float*>(wsb + WL.partial),
       reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }

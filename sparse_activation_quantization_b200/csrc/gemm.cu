@@ -53,6 +53,7 @@ struct GemmArgs {
   void* Y;
   const int* group_offsets;  // device [E+1] or nullptr
   int* err;                  // workspace error word or nullptr
+  const int* act_err;        // error word left by sharq_prep (propagated)
   int* tile_count;           // split-K: arrivals per output tile (self-resetting)
   float* partial;            // split-K: fp32 partial sums [splits][T][D]
   int T, K, D, E;
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
     }
     expert_sh = e;
+    if (blockIdx.x == 0 && blockIdx.z == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, C::kTmemCols);
@@ -391,7 +393,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
-                          int* err, int* tile_count, float* partial, cudaStream_t stream) {
+                          int* err, const int* act_err, int* tile_count, float* partial, cudaStream_t stream) {
   GemmArgs a;
   a.a_sp = a_sp;
   a.a_meta = a_meta;
@@ -406,6 +408,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.Y = Y;
   a.group_offsets = group_offsets;
   a.err = err;
+  a.act_err = act_err;
   a.tile_count = tile_count;
   a.partial = partial;
   a.T = T;

@@ -157,46 +157,11 @@ struct QuantPtrs {
 
 constexpr int kQuantThreads = 256;
 
+// Quantize one row segment of 32 logical K (row t, 32-block j) held in
+// registers: mask, backbone NVFP4, residual, dense NVFP4, tiled stores.
 template <bool kSharq>
-__global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
-    const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
-    const int* __restrict__ row_index, int T, int Tp, int K, const float* __restrict__ inv_rms,
-    const unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
-  const int nb32 = K >> 5;
-  const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
-  const float gmax = __uint_as_float(*gmax_bits);
-  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
-  if (gid == 0) *s_g_out = s;  // published even when there are no rows
-  if (gid >= (long long)Tp * nb32) return;
-  const int t = (int)(gid / nb32);
-  const int j = (int)(gid - (long long)t * nb32);
-  const float six_s = __fmul_rn(6.0f, s);
-
-  // --- load the 32 values of this row segment and normalise them ---
-  float x[32];
-  int src = -1;
-  if (t < T) src = row_index ? row_index[t] : t;
-  if (src >= 0) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * j);
-    uint4 raw[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) raw[i] = xr[i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) bf16x8_to_float(raw[i], x + 8 * i);
-    if (gamma) {
-      const float inv = inv_rms[t];
-      const uint4* gr = reinterpret_cast<const uint4*>(gamma + 32 * j);
-      float g[32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) bf16x8_to_float(gr[i], g + 8 * i);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] = norm_one(x[i], inv, g[i]);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = 0.0f;
-  }
-
+__device__ __forceinline__ void quant_segment(const float (&x)[32], int t, int j, int K, float s, float six_s,
+                                              const QuantPtrs& out) {
   const int KS = K >> 8;
   const int kt = j >> 3, q = j & 7;
   const int r = t & 127;
@@ -282,31 +247,222 @@ __global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
       (uint16_t)(b0.sb | (b1.sb << 8));
 }
 
+
+template <bool kSharq>
+__global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
+    const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
+    const int* __restrict__ row_index, int T, int Tp, int K, const float* __restrict__ inv_rms,
+    const unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
+  const int nb32 = K >> 5;
+  const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
+  const float gmax = __uint_as_float(*gmax_bits);
+  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
+  if (gid == 0) *s_g_out = s;  // published even when there are no rows
+  if (gid >= (long long)Tp * nb32) return;
+  const int t = (int)(gid / nb32);
+  const int j = (int)(gid - (long long)t * nb32);
+  const float six_s = __fmul_rn(6.0f, s);
+
+  // --- load the 32 values of this row segment and normalise them ---
+  float x[32];
+  int src = -1;
+  if (t < T) src = row_index ? row_index[t] : t;
+  if (src >= 0) {
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * j);
+    uint4 raw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) raw[i] = xr[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bf16x8_to_float(raw[i], x + 8 * i);
+    if (gamma) {
+      const float inv = inv_rms[t];
+      const uint4* gr = reinterpret_cast<const uint4*>(gamma + 32 * j);
+      float g[32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bf16x8_to_float(gr[i], g + 8 * i);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = norm_one(x[i], inv, g[i]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+  }
+
+  quant_segment<kSharq>(x, t, j, K, s, six_s, out);
+}
+
+
+// ---------------------------------------------------------------------------
+// Single-launch form: one cooperative grid, one thread per (row, 32-K block),
+// whole rows inside a CTA (rows_per_cta x K/32 threads).  The row's values
+// stay in registers from the load to the stores:
+//   1. load + sum of squares (float64, fixed-order tree per row) -> 1/rms,
+//      normalise in registers, CTA max |Xn|  -> atomicMax(gmax);
+//   2. grid-wide barrier (arrival counter, bounded spin on the global timer);
+//   3. quantize from registers (same code as prep_quant_kernel).
+// X is read from HBM exactly once.  Used whenever the grid fits on the GPU at
+// once (cooperative launch guarantees co-residency); larger tensors take the
+// two-launch path above.
+constexpr int kFusedMaxThreads = 640;            // K/32 <= 592 threads per row
+constexpr uint64_t kBarrierLimitNs = 2000000000ull;
+
+template <bool kSharq>
+__global__ void __launch_bounds__(kFusedMaxThreads) prep_fused_kernel(
+    const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
+    const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
+    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out) {
+  __shared__ double part[kFusedMaxThreads];
+  __shared__ float wmax[kFusedMaxThreads / 32];
+  __shared__ float gmax_sh;
+  const int nb32 = K >> 5;
+  const int rl = threadIdx.x / nb32;
+  const int j = threadIdx.x - rl * nb32;
+  const int t = blockIdx.x * rows_per_cta + rl;
+  const bool live = t < Tp;
+
+  float x[32];
+  int src = -1;
+  if (live && t < T) src = row_index ? row_index[t] : t;
+  if (src >= 0) {
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * j);
+    uint4 raw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) raw[i] = xr[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bf16x8_to_float(raw[i], x + 8 * i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = 0.0f;
+  }
+
+  if (gamma) {
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ss += (double)x[i] * (double)x[i];
+    part[threadIdx.x] = ss;
+    __syncthreads();
+    int span = 1;
+    while (span < nb32) span <<= 1;
+    for (int off = span >> 1; off > 0; off >>= 1) {
+      if (j < off && j + off < nb32) part[threadIdx.x] += part[threadIdx.x + off];
+      __syncthreads();
+    }
+    const float inv = (float)(1.0 / sqrt(part[rl * nb32] / (double)K + (double)eps));
+    if (live && t < T && j == 0) inv_rms[t] = inv;
+    const uint4* gr = reinterpret_cast<const uint4*>(gamma + 32 * j);
+    float g[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bf16x8_to_float(gr[i], g + 8 * i);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = norm_one(x[i], inv, g[i]);
+  } else if (live && t < T && j == 0) {
+    inv_rms[t] = 1.0f;
+  }
+
+  // CTA max |Xn| -> device-wide max
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) m = fmaxf(m, wmax[w]);
+    atomicMax(sync, __float_as_uint(m));
+    __threadfence();
+    atomicAdd(sync + 1, 1u);
+    // grid barrier: every CTA has published its max
+    const uint64_t deadline = globaltimer_ns() + kBarrierLimitNs;
+    unsigned seen = 0;
+    do {
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(sync + 1) : "memory");
+      if (seen >= gridDim.x) break;
+      if (globaltimer_ns() > deadline) {
+        atomicCAS(reinterpret_cast<int*>(sync + 3), 0, -5);  // SHARQ_ERR_TIMEOUT
+        break;
+      }
+    } while (true);
+    unsigned gb;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gb) : "l"(sync) : "memory");
+    gmax_sh = __uint_as_float(gb);
+  }
+  __syncthreads();
+  const float gmax = gmax_sh;
+  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
+  if (live) quant_segment<kSharq>(x, t, j, K, s, __fmul_rn(6.0f, s), out);
+}
+
+
+// rows per CTA of the single-launch form for a row length of K
+int fused_rows_per_cta(int K) {
+  const int nb32 = K >> 5;
+  if (nb32 > kFusedMaxThreads) return 0;
+  return nb32 >= 256 ? 1 : 256 / nb32;
+}
+
+// Largest grid of the single-launch form that can be resident at once.
+int fused_max_ctas(bool sharq_mode, int threads) {
+  static int cache[2][kFusedMaxThreads + 1][64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
+  int& c = cache[sharq_mode ? 1 : 0][threads][dev];
+  if (c == 0) {
+    int per_sm = 0, sms = 0;
+    cudaError_t e = sharq_mode
+        ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<true>, threads, 0)
+        : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<false>, threads, 0);
+    if (e != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    c = per_sm * sms > 0 ? per_sm * sms : -1;
+  }
+  return c > 0 ? c : 0;
+}
+
 }  // namespace
 
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
                         int K, bool sharq_mode, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
                         cudaStream_t stream) {
-  cudaError_t e = cudaMemsetAsync(gmax_bits, 0, sizeof(unsigned int), stream);
+  // gmax, barrier arrivals, (unused), error word
+  cudaError_t e = cudaMemsetAsync(gmax_bits, 0, 4 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
+  QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf};
+  const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+  const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
+
+  const int rpc = fused_rows_per_cta(K);
+  if (Tp > 0 && rpc > 0) {
+    const int threads = rpc * (K >> 5);
+    const int ctas = (Tp + rpc - 1) / rpc;
+    if (ctas <= fused_max_ctas(sharq_mode, threads)) {
+      void* args[] = {(void*)&Xb, (void*)&Gb, (void*)&eps, (void*)&row_index, (void*)&T, (void*)&Tp, (void*)&K,
+                      (void*)&rpc, (void*)&inv_rms, (void*)&gmax_bits, (void*)&s_g, (void*)&p};
+      const void* fn = sharq_mode ? reinterpret_cast<const void*>(prep_fused_kernel<true>)
+                                  : reinterpret_cast<const void*>(prep_fused_kernel<false>);
+      e = cudaLaunchCooperativeKernel(fn, dim3(ctas), dim3(threads), args, 0, stream);
+      if (e == cudaSuccess) return cudaSuccess;
+      cudaGetLastError();  // fall back to the two-launch form below
+    }
+  }
+
   if (T > 0) {
-    prep_stats_kernel<<<T, kStatsThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(gamma), eps, row_index, K,
-        inv_rms, gmax_bits);
+    prep_stats_kernel<<<T, kStatsThreads, 0, stream>>>(Xb, Gb, eps, row_index, K, inv_rms, gmax_bits);
   }
   const long long n = (long long)Tp * (K >> 5);
   // at least one block so that s_g is published (= 1) even for T == 0
   const unsigned grid = n > 0 ? (unsigned)((n + kQuantThreads - 1) / kQuantThreads) : 1u;
-  QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf};
   if (sharq_mode)
-    prep_quant_kernel<true><<<grid, kQuantThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(gamma), row_index, T, Tp, K,
-        inv_rms, gmax_bits, s_g, p);
+    prep_quant_kernel<true><<<grid, kQuantThreads, 0, stream>>>(Xb, Gb, row_index, T, Tp, K, inv_rms, gmax_bits,
+                                                                 s_g, p);
   else
-    prep_quant_kernel<false><<<grid, kQuantThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(gamma), row_index, T, Tp, K,
-        inv_rms, gmax_bits, s_g, p);
+    prep_quant_kernel<false><<<grid, kQuantThreads, 0, stream>>>(Xb, Gb, row_index, T, Tp, K, inv_rms,
+                                                                  gmax_bits, s_g, p);
   return cudaGetLastError();
 }
 

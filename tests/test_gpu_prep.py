@@ -94,6 +94,14 @@ def test_prep_bit_exact(name, T, K, kw, gam, eps):
     _check_sharq(x, gamma, eps)
 
 
+@pytest.mark.parametrize("T,K", [(400, 14336), (700, 8192)])
+def test_prep_two_launch_path_bit_exact(T, K):
+    """Tensors too large for one co-resident grid take the two-launch form
+    (stats kernel + quantize kernel); it must agree bit for bit as well."""
+    x = synthetic.activations(55 + T, T, K, base="student_t" if K > 10000 else "normal")
+    _check_sharq(x, synthetic.gamma(56, K), 1e-5)
+
+
 def test_prep_nvfp4_mode_bit_exact():
     T, K = 130, 512
     x = synthetic.activations(5, T, K)
