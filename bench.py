@@ -222,7 +222,7 @@ def run_gpu(args, world, rank, local):
             acts[t].prep(xs[t][i], gamma, EPS, stream=stream)
             sq.linear(acts[t], weights[i], out=outs[t], ws=wss[t], stream=stream)
 
-    launches_per_step = 3 * len(T_LIST)   # prep_stats, prep_quant, gemm per layer
+    launches_per_step = 2 * len(T_LIST)   # single-launch prep + gemm per layer
     # warm up eagerly, then capture one graph per rotation slot
     for i in range(N_ROT):
         step(i)
