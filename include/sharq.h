@@ -135,10 +135,8 @@ typedef struct {
 size_t sharq_weight_bytes(int K, int D, int E);
 size_t sharq_act_bytes(int T, int K, int mode);
 /* Workspace of sharq_linear (E = 1) / sharq_linear_grouped (E experts):
- * an error word, one arrival counter per output tile and, for decode shapes
- * that split K across CTAs, fp32 partial sums.  The caller zeroes it once
- * after allocation; every call leaves it zeroed again (except the error
- * word, which sharq_check_status clears). */
+ * the device-side error word (256 bytes reserved).  The caller zeroes it
+ * once after allocation; sharq_check_status clears it after reading. */
 size_t sharq_workspace_bytes(int T, int K, int D, int E);
 
 /* Carve the views of a caller-owned device buffer of at least the size
@@ -187,9 +185,7 @@ int sharq_prep(const void *d_X, const void *d_gamma, float eps, const int *d_row
  * Y = round(f32(acc * f32(s_g * s_w))) written to d_Y [T][D] row-major,
  * bf16 or float32 per out_dtype.  Mode NVFP4 runs the dense MMA only.
  * d_ws: workspace of at least sharq_workspace_bytes(T, K, D, 1) bytes, zeroed
- * once by the caller after allocation; it receives device-side error codes
- * and holds split-K partial sums.  Calls sharing a workspace must not
- * overlap in time (same stream, or ordered by events).
+ * once by the caller after allocation; it receives device-side error codes.
  */
 int sharq_linear(const sharq_act *a, const sharq_weight *w, void *d_Y, int out_dtype,
                  void *d_ws, size_t ws_bytes, sharq_stream_t stream);

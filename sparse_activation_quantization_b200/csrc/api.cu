@@ -19,7 +19,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
-                          int* err, const int* act_err, int* tile_count, float* partial, cudaStream_t stream);
+                          int* err, const int* act_err, cudaStream_t stream);
 }  // namespace sharq
 
 namespace {
@@ -79,11 +79,10 @@ WeightLayout weight_layout(int K, int D, int E) {
 }
 
 // GEMM launch shape for a problem: tile width BN and the number of K splits.
-// Prefill shapes have enough output tiles to fill the GPU (BN = 256, no
-// split).  Decode shapes split K so that about one CTA per SM streams a slice
-// of the weight; the fp32 partials cost 8 bytes (write + read) per output
-// element per split, so the split count is also capped to keep that traffic
-// well below the weight bytes (0.59375 B per weight element).
+// Prefill shapes have enough output tiles to fill the GPU (no split).  Decode
+// shapes split K over a cluster of up to 8 CTAs per output tile so that about
+// one CTA per SM streams a slice of the weight; the partial tiles are reduced
+// over distributed shared memory, so no workspace is needed for them.
 struct GemmShape {
   int bn, splits, m_tiles, n_tiles;
 };
@@ -92,31 +91,17 @@ GemmShape gemm_shape(int T, int K, int D, int E) {
   const int Tp = (int)round_up((size_t)T, 128);
   g.m_tiles = Tp / 128;
   const int KS = K / 256;
-  const bool wide = (D % 256 == 0) && (long long)g.m_tiles * (D / 256) >= kTargetCtas;
-  g.bn = wide ? 256 : 128;
+  g.bn = (D % 256 == 0) ? 256 : 128;
   g.n_tiles = D / g.bn;
   g.splits = 1;
   const long long mn = (long long)g.m_tiles * g.n_tiles;
   if (E == 1 && mn > 0 && mn < kTargetCtas / 2) {
     int s = (int)(kTargetCtas / mn);
-    const int cap = (int)(0.15 * K / (T > 0 ? T : 1));
-    s = s < cap ? s : cap;
+    s = s < 8 ? s : 8;
     s = s < KS ? s : KS;
     g.splits = s > 1 ? s : 1;
   }
   return g;
-}
-
-struct WsLayout {
-  size_t counters, partial, total;
-};
-WsLayout ws_layout(int T, int K, int D, int E) {
-  const GemmShape g = gemm_shape(T, K, D, E);
-  WsLayout L{};
-  L.counters = kWsHeader;
-  L.partial = round_up(L.counters + (size_t)g.m_tiles * g.n_tiles * sizeof(int), kAlign);
-  L.total = L.partial + (g.splits > 1 ? (size_t)g.splits * T * D * sizeof(float) : 0);
-  return L;
 }
 
 int check_device() {
@@ -168,17 +153,14 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
     return SHARQ_ERR_WORKSPACE;
   if ((st = check_device())) return st;
   const GemmShape g = gemm_shape(a->T, a->K, w->D, grouped ? w->E : 1);
-  const WsLayout WL = ws_layout(a->T, a->K, w->D, grouped ? w->E : 1);
-  uint8_t* wsb = static_cast<uint8_t*>(d_ws);
   cudaError_t e = sharq::launch_linear(
       static_cast<const uint8_t*>(a->sp_codes), static_cast<const uint8_t*>(a->meta),
       static_cast<const uint8_t*>(a->sp_sf), static_cast<const uint8_t*>(a->r_codes),
       static_cast<const uint8_t*>(a->r_sf), a->s_g, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ ? 1 : 0,
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
-      out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, reinterpret_cast<int*>(wsb),
-      reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<int*>(wsb + WL.counters), reinterpret_cast<float*>(wsb + WL.partial),
-      reinterpret_cast<cudaStream_t>(stream));
+      out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, static_cast<int*>(d_ws),
+      reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 
@@ -214,7 +196,7 @@ size_t sharq_act_bytes(int T, int K, int mode) {
 
 size_t sharq_workspace_bytes(int T, int K, int D, int E) {
   if (!shape_ok_t(T) || !shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return 0;
-  return ws_layout(T, K, D, E).total;
+  return kWsHeader;
 }
 
 int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {

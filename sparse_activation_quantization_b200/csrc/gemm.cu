@@ -22,10 +22,12 @@
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per thread),
 //               y = f32(acc * f32(s_g * s_w)), bf16 or fp32 stores.
 // Split-K (decode shapes, where output tiles alone cannot fill 148 SMs):
-// blockIdx.z picks a contiguous range of K stages; each CTA writes its fp32
-// partial tile to the workspace, and the last CTA to arrive at a tile (one
-// atomic counter per tile, reset by that CTA) sums the partials in split
-// order -- deterministic -- and writes Y.
+// the S CTAs that share an output tile form one thread-block cluster
+// (1 x 1 x S); each takes a contiguous range of K stages, parks its fp32
+// partial tile in its own (now idle) shared-memory ring, and after an
+// mbarrier exchange every CTA sums 1/S of the tile's rows by reading all S
+// partials over distributed shared memory in rank order -- deterministic,
+// no global scratch, no atomics.
 // Every wait is bounded by the global timer; on timeout the CTA records
 // SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
 #include "sharq_device.cuh"
@@ -54,8 +56,6 @@ struct GemmArgs {
   const int* group_offsets;  // device [E+1] or nullptr
   int* err;                  // workspace error word or nullptr
   const int* act_err;        // error word left by sharq_prep (propagated)
-  int* tile_count;           // split-K: arrivals per output tile (self-resetting)
-  float* partial;            // split-K: fp32 partial sums [splits][T][D]
   int T, K, D, E;
   int out_f32;
   int sharq_mode;
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
-  __shared__ int last_sh;
+  __shared__ __align__(8) uint64_t red_bar[2];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -171,6 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
+    mbar_init(&red_bar[0], args.splits);
+    mbar_init(&red_bar[1], args.splits);
     fence_mbar_init();
     abort_sh = 0;
     // expert of this m-tile (grouped form): offsets are 128-row aligned
@@ -197,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (args.splits > 1) cluster_sync_all();  // peers' barriers initialised
   const uint32_t tmem = tmem_base_sh;
   const int expert = expert_sh;
   if (expert < 0) {
@@ -317,46 +320,78 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           if (row < args.T) store_row32(args.Y, args.out_f32, (size_t)row * args.D + col0 + c, v, scale);
         }
       } else {
-        // 1. this split's fp32 partial tile -> workspace (valid rows only)
+        // this split's fp32 partial tile -> own shared memory (valid rows)
+        float* part = reinterpret_cast<float*>(smem);
+        const int rl = sp * 32 + lane;
+        const int valid = min(128, args.T - mt * 128);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
           tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
           tmem_ld_wait();
-          if (row < args.T) {
-            float* dst = args.partial + ((size_t)split * args.T + row) * args.D + col0 + c;
+          if (rl < valid) {
+            float* dst = part + rl * (BN + 4) + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-              __stcg(reinterpret_cast<float4*>(dst + i),
-                     make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
-                                 __uint_as_float(v[i + 3])));
+              *reinterpret_cast<float4*>(dst + i) =
+                  make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
+                              __uint_as_float(v[i + 3]));
           }
         }
-        // 2. count arrivals at this tile; the last CTA reduces
-        __threadfence();
-        named_barrier_sync(1, 128);
-        const int tile_id = mt * gridDim.x + nt;
-        if (threadIdx.x == 64) last_sh = (atomicAdd(args.tile_count + tile_id, 1) == args.splits - 1);
-        named_barrier_sync(1, 128);
-        if (last_sh) {
-          __threadfence();
-          const int rows = min(128, args.T - mt * 128);
-          const int q4 = BN / 4;
-          for (int idx = threadIdx.x - 64; idx < rows * q4; idx += 128) {
-            const int r = idx / q4, c4 = idx - r * q4;
-            const size_t off = (size_t)(mt * 128 + r) * args.D + col0 + 4 * c4;
-            float4 acc = __ldcg(reinterpret_cast<const float4*>(args.partial + off));
-            for (int sp2 = 1; sp2 < args.splits; ++sp2) {
-              const float4 p = __ldcg(reinterpret_cast<const float4*>(args.partial + (size_t)sp2 * args.T * args.D + off));
-              acc.x = __fadd_rn(acc.x, p.x);
-              acc.y = __fadd_rn(acc.y, p.y);
-              acc.z = __fadd_rn(acc.z, p.z);
-              acc.w = __fadd_rn(acc.w, p.w);
-            }
-            store4(args.Y, args.out_f32, off, acc, scale);
+      }
+    }
+  }
+
+  if (args.splits > 1) {
+    // ---------------------------------------- cluster split-K reduction --
+    const uint32_t S = (uint32_t)args.splits;
+    const uint32_t rank = cluster_ctarank();
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+    __syncthreads();  // this CTA's partial is complete and ordered before the arrive
+    if (threadIdx.x == 0)
+      for (uint32_t r = 0; r < S; ++r) mbar_arrive_remote(mapa_shared(smem_u32(&red_bar[0]), r));
+    bool ok = true;
+    while (!mbar_try_wait_cluster(&red_bar[0], 0)) {
+      if (globaltimer_ns() > deadline) { ok = false; break; }
+    }
+    if (!ok) {
+      if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
+    } else if (!abort_sh) {
+      const int valid = min(128, args.T - mt * 128);
+      const int rows_per = (valid + (int)S - 1) / (int)S;
+      const int r0 = (int)rank * rows_per;
+      const int r1 = min(valid, r0 + rows_per);
+      const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
+      const uint32_t part_local = smem_u32(smem);
+      uint32_t base[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) base[r] = r < (int)S ? mapa_shared(part_local, (uint32_t)r) : 0u;
+      constexpr int q4 = BN / 4;
+      for (int idx = threadIdx.x; idx < (r1 - r0) * q4; idx += kThreads) {
+        const int row = r0 + idx / q4, c4 = idx % q4;
+        const uint32_t off = (uint32_t)(row * (BN + 4) + 4 * c4) * 4u;
+        float4 acc = ld_shared_cluster_f4(base[0] + off);
+#pragma unroll
+        for (int r = 1; r < 8; ++r) {
+          if (r < (int)S) {
+            const float4 p = ld_shared_cluster_f4(base[r] + off);
+            acc.x = __fadd_rn(acc.x, p.x);
+            acc.y = __fadd_rn(acc.y, p.y);
+            acc.z = __fadd_rn(acc.z, p.z);
+            acc.w = __fadd_rn(acc.w, p.w);
           }
-          if (threadIdx.x == 64) args.tile_count[tile_id] = 0;  // ready for the next call
         }
+        store4(args.Y, args.out_f32, (size_t)(mt * 128 + row) * args.D + nt * BN + 4 * c4, acc, scale);
+      }
+    }
+    // nobody leaves while a peer may still read its shared memory
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (uint32_t r = 0; r < S; ++r) mbar_arrive_remote(mapa_shared(smem_u32(&red_bar[1]), r));
+    while (!mbar_try_wait_cluster(&red_bar[1], 0)) {
+      if (globaltimer_ns() > deadline) {
+        if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
+        break;
       }
     }
   }
@@ -373,6 +408,8 @@ template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   static_assert(BN == 128 || BN == 256, "tile width");
   using C = Cfg<BN>;
+  static_assert(128 * (BN + 4) * 4 <= C::kStages * C::kStageBytes, "split-K partial must fit the ring");
+  if (a.splits < 1 || a.splits > 8) return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -382,9 +419,19 @@ cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(a.D / BN, m_tiles, a.splits);
-  sharq_gemm_kernel<BN><<<grid, kThreads, C::kSmemBytes, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.D / BN, m_tiles, a.splits);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = a.splits;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.splits > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<BN>, a);
 }
 
 }  // namespace
@@ -393,7 +440,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
-                          int* err, const int* act_err, int* tile_count, float* partial, cudaStream_t stream) {
+                          int* err, const int* act_err, cudaStream_t stream) {
   GemmArgs a;
   a.a_sp = a_sp;
   a.a_meta = a_meta;
@@ -409,8 +456,6 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.group_offsets = group_offsets;
   a.err = err;
   a.act_err = act_err;
-  a.tile_count = tile_count;
-  a.partial = partial;
   a.T = T;
   a.K = K;
   a.D = D;
