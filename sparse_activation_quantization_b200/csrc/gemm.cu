@@ -37,6 +37,23 @@ namespace sharq {
 namespace {
 
 constexpr int kThreads = 192;
+
+// Optional phase timeline (compile with -DSHARQ_TRACE): 8 global-timer
+// stamps per CTA -- entry, set-up done, first stage issued, first stage
+// consumed, last MMA committed, accumulator ready, epilogue done, exit.
+#ifdef SHARQ_TRACE
+__device__ unsigned long long* g_trace = nullptr;
+#define TRACE_POINT(k)                                                                                   \
+  do {                                                                                                   \
+    if (g_trace)                                                                                         \
+      g_trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 8 + (k)] =      \
+          globaltimer_ns();                                                                              \
+  } while (0)
+#else
+#define TRACE_POINT(k) \
+  do {                 \
+  } while (0)
+#endif
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far beyond any tile's work
 constexpr int kErrTimeout = -5;
 constexpr int kErrInvalid = -1;
@@ -164,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   const int nks = ks1 - ks0;
   const int NB = args.D >> 7;
   const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+  if (threadIdx.x == 0) TRACE_POINT(0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -200,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   __syncthreads();
   tc_fence_after();
   if (args.splits > 1) cluster_sync_all();  // peers' barriers initialised
+  if (threadIdx.x == 0) TRACE_POINT(1);
   const uint32_t tmem = tmem_base_sh;
   const int expert = expert_sh;
   if (expert < 0) {
@@ -236,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, fb);
           if (sharq) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
         }
+        if (i == 0) TRACE_POINT(2);
         bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, kCodesTile, fb);
         bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
         if (sharq) {
@@ -258,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           break;
         }
         tc_fence_after();
+        if (i == 0) TRACE_POINT(3);
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
         // scale factors (and metadata) shared memory -> TMEM
 #pragma unroll
@@ -298,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         tc_commit(&empty_bar[s]);
       }
       tc_commit(&acc_bar);  // accumulator complete (or everything issued so far, on abort)
+      TRACE_POINT(4);
     }
   } else {
     // ------------------------------------------------------- epilogue ----
@@ -305,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     const int row = mt * 128 + sp * 32 + lane;
     const bool ok = mbar_wait(&acc_bar, 0, deadline, &abort_sh);
     tc_fence_after();
+    if (threadIdx.x == 64) TRACE_POINT(5);
     if (!ok) {
       record_error(args.err, kErrTimeout);
       abort_sh = 1;
@@ -342,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     }
   }
 
+  if (threadIdx.x == 64) TRACE_POINT(6);
   if (args.splits > 1) {
     // ---------------------------------------- cluster split-K reduction --
     const uint32_t S = (uint32_t)args.splits;
@@ -398,6 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) TRACE_POINT(7);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -435,6 +460,12 @@ cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
 }
 
 }  // namespace
+
+#ifdef SHARQ_TRACE
+extern "C" int sharq_debug_set_trace(void* p) {
+  return cudaMemcpyToSymbol(g_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -4;
+}
+#endif
 
 cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
