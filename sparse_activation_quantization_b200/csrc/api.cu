@@ -94,10 +94,15 @@ GemmShape gemm_shape(int T, int K, int D, int E) {
   g.bn = (D % 256 == 0) ? 256 : 128;
   g.n_tiles = D / g.bn;
   g.splits = 1;
-  const long long mn = (long long)g.m_tiles * g.n_tiles;
-  if (E == 1 && mn > 0 && mn < kTargetCtas / 2) {
+  if (E == 1 && (long long)g.m_tiles * g.n_tiles < kTargetCtas / 2) {
+    // split: 128-wide tiles (the partial and the received slices must fit the
+    // shared-memory ring) and clusters of at most 4, which the GPCs can host
+    // all at once with one CTA per SM
+    g.bn = 128;
+    g.n_tiles = D / 128;
+    const long long mn = (long long)g.m_tiles * g.n_tiles;
     int s = (int)(kTargetCtas / mn);
-    s = s < 8 ? s : 8;
+    s = s < 4 ? s : 4;
     s = s < KS ? s : KS;
     g.splits = s > 1 ? s : 1;
   }

@@ -23,11 +23,16 @@
 //               y = f32(acc * f32(s_g * s_w)), bf16 or fp32 stores.
 // Split-K (decode shapes, where output tiles alone cannot fill 148 SMs):
 // the S CTAs that share an output tile form one thread-block cluster
-// (1 x 1 x S); each takes a contiguous range of K stages, parks its fp32
-// partial tile in its own (now idle) shared-memory ring, and after an
-// mbarrier exchange every CTA sums 1/S of the tile's rows by reading all S
-// partials over distributed shared memory in rank order -- deterministic,
-// no global scratch, no atomics.
+// (1 x 1 x S); each takes a contiguous range of K stages and parks its fp32
+// partial tile in its own (now idle) shared-memory ring.  CTA r of the
+// cluster owns 1/S of the tile's valid rows: every CTA pushes that slice of
+// its partial into the owner's shared memory with one bulk copy over
+// distributed shared memory (completion = transaction bytes on the owner's
+// mbarrier), and the owner sums the S slices in rank order -- deterministic,
+// no global scratch, no atomics, one bounded wait.
+// Rows beyond the activation's valid rows are not copied into shared memory
+// (decode: T = 1 moves 1 row of codes, not 128); their accumulator rows hold
+// garbage that is never stored -- MMA rows are independent.
 // Every wait is bounded by the global timer; on timeout the CTA records
 // SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
 #include "sharq_device.cuh"
@@ -116,10 +121,6 @@ __device__ __forceinline__ void record_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // y = f32(acc * scale), 32 consecutive columns of one row, bf16 or fp32
 __device__ __forceinline__ void store_row32(void* Y, int out_f32, size_t off, const uint32_t (&v)[32], float scale) {
   if (out_f32) {
@@ -163,6 +164,7 @@ __device__ __forceinline__ void store4(void* Y, int out_f32, size_t off, float4 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
   using C = Cfg<BN>;
+  constexpr int kRowFloats = BN + 4;  // padded partial row: conflict-free float4 stores
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::kStages];
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
-  __shared__ __align__(8) uint64_t red_bar[2];
+  __shared__ __align__(8) uint64_t red_bar[1];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -189,8 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
-    mbar_init(&red_bar[0], args.splits);
-    mbar_init(&red_bar[1], args.splits);
+    mbar_init(&red_bar[0], 1);
     fence_mbar_init();
     abort_sh = 0;
     // expert of this m-tile (grouped form): offsets are 128-row aligned
@@ -217,7 +218,15 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (args.splits > 1) cluster_sync_all();  // peers' barriers initialised
+  if (args.splits > 1) {
+    cluster_sync_all();  // peers' barriers initialised before any remote traffic
+    if (threadIdx.x == 0) {
+      const int valid = min(128, args.T - mt * 128);
+      const int rows_per = (valid + args.splits - 1) / args.splits;
+      const int my0 = (int)cluster_ctarank() * rows_per, my_n = min(valid, my0 + rows_per) - my0;
+      if (my_n > 0) mbar_arrive_expect_tx(&red_bar[0], (uint32_t)(args.splits * my_n * (BN + 4) * 4));
+    }
+  }
   if (threadIdx.x == 0) TRACE_POINT(1);
   const uint32_t tmem = tmem_base_sh;
   const int expert = expert_sh;
@@ -233,6 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
       const size_t a_tile0 = (size_t)mt * KS;
+      // copy only the valid rows of the activation code tiles
+      const uint32_t a_rows = (uint32_t)min(128, args.T - mt * 128);
+      const uint32_t a_trim = (128u - a_rows) * (sharq ? 192u : 128u);
       const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
       for (int i = 0; i < nks; ++i) {
         const int ks = ks0 + i;
@@ -246,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         }
         uint8_t* st = smem + s * C::kStageBytes;
         uint64_t* fb = &full_bar[s];
-        mbar_arrive_expect_tx(fb, sharq ? C::kTxSharq : C::kTxNvfp4);
+        mbar_arrive_expect_tx(fb, (sharq ? C::kTxSharq : C::kTxNvfp4) - a_trim);
         const size_t at = a_tile0 + ks;
 #pragma unroll
         for (int h = 0; h < C::kHalves; ++h) {
@@ -256,10 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           if (sharq) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
         }
         if (i == 0) TRACE_POINT(2);
-        bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, kCodesTile, fb);
+        bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, a_rows * 128u, fb);
         bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
         if (sharq) {
-          bulk_g2s(st + C::kOffASP, args.a_sp + at * kSpTile, kSpTile, fb);
+          bulk_g2s(st + C::kOffASP, args.a_sp + at * kSpTile, a_rows * 64u, fb);
           bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, kMetaTile, fb);
           bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
         }
@@ -353,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
           tmem_ld_wait();
           if (rl < valid) {
-            float* dst = part + rl * (BN + 4) + c;
+            float* dst = part + rl * kRowFloats + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               *reinterpret_cast<float4*>(dst + i) =
@@ -361,63 +373,60 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
                               __uint_as_float(v[i + 3]));
           }
         }
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the bulk copy
       }
     }
   }
 
   if (threadIdx.x == 64) TRACE_POINT(6);
   if (args.splits > 1) {
-    // ---------------------------------------- cluster split-K reduction --
-    const uint32_t S = (uint32_t)args.splits;
+    // ------------------------------------ cluster split-K reduction (push) --
+    const int S = args.splits;
     const uint32_t rank = cluster_ctarank();
-    asm volatile("fence.acq_rel.cluster;" ::: "memory");
-    __syncthreads();  // this CTA's partial is complete and ordered before the arrive
-    if (threadIdx.x == 0)
-      for (uint32_t r = 0; r < S; ++r) mbar_arrive_remote(mapa_shared(smem_u32(&red_bar[0]), r));
-    bool ok = true;
-    while (!mbar_try_wait_cluster(&red_bar[0], 0)) {
-      if (globaltimer_ns() > deadline) { ok = false; break; }
-    }
-    if (!ok) {
-      if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
-    } else if (!abort_sh) {
-      const int valid = min(128, args.T - mt * 128);
-      const int rows_per = (valid + (int)S - 1) / (int)S;
-      const int r0 = (int)rank * rows_per;
-      const int r1 = min(valid, r0 + rows_per);
-      const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
-      const uint32_t part_local = smem_u32(smem);
-      uint32_t base[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) base[r] = r < (int)S ? mapa_shared(part_local, (uint32_t)r) : 0u;
-      constexpr int q4 = BN / 4;
-      for (int idx = threadIdx.x; idx < (r1 - r0) * q4; idx += kThreads) {
-        const int row = r0 + idx / q4, c4 = idx % q4;
-        const uint32_t off = (uint32_t)(row * (BN + 4) + 4 * c4) * 4u;
-        float4 acc = ld_shared_cluster_f4(base[0] + off);
-#pragma unroll
-        for (int r = 1; r < 8; ++r) {
-          if (r < (int)S) {
-            const float4 p = ld_shared_cluster_f4(base[r] + off);
-            acc.x = __fadd_rn(acc.x, p.x);
-            acc.y = __fadd_rn(acc.y, p.y);
-            acc.z = __fadd_rn(acc.z, p.z);
-            acc.w = __fadd_rn(acc.w, p.w);
-          }
-        }
-        store4(args.Y, args.out_f32, (size_t)(mt * 128 + row) * args.D + nt * BN + 4 * c4, acc, scale);
+    const int valid = min(128, args.T - mt * 128);
+    const int rows_per = (valid + S - 1) / S;
+    const uint32_t row_bytes = kRowFloats * 4u;
+    const uint32_t part_addr = smem_u32(smem);
+    const uint32_t recv_addr = part_addr + 128u * row_bytes;  // S slices of rows_per rows
+    __syncthreads();  // partial complete in this CTA
+    if (threadIdx.x == 0 && !abort_sh) {
+      for (int r = 0; r < S; ++r) {
+        const int r0 = r * rows_per, n = min(valid, r0 + rows_per) - r0;
+        if (n <= 0) continue;
+        const uint32_t dst = mapa_shared(recv_addr + rank * (uint32_t)rows_per * row_bytes, (uint32_t)r);
+        bulk_s2cluster(dst, part_addr + (uint32_t)r0 * row_bytes, (uint32_t)n * row_bytes,
+                       mapa_shared(smem_u32(&red_bar[0]), (uint32_t)r));
       }
+      bulk_commit_group();
     }
-    // nobody leaves while a peer may still read its shared memory
-    __syncthreads();
-    if (threadIdx.x == 0)
-      for (uint32_t r = 0; r < S; ++r) mbar_arrive_remote(mapa_shared(smem_u32(&red_bar[1]), r));
-    while (!mbar_try_wait_cluster(&red_bar[1], 0)) {
-      if (globaltimer_ns() > deadline) {
+    const int my0 = (int)rank * rows_per, my_n = min(valid, my0 + rows_per) - my0;
+    if (my_n > 0) {
+      bool ok = !abort_sh;
+      while (ok && !mbar_try_wait_cluster(&red_bar[0], 0)) {
+        if (globaltimer_ns() > deadline) ok = false;
+      }
+      if (!ok) {
         if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
-        break;
+      } else {
+        const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
+        const float* recv = reinterpret_cast<const float*>(smem + 128u * row_bytes);
+        constexpr int q4 = BN / 4;
+        for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
+          const int r = idx / q4, c4 = idx - r * q4;
+          const float* p = recv + r * kRowFloats + 4 * c4;
+          float4 acc = *reinterpret_cast<const float4*>(p);
+          for (int s2 = 1; s2 < S; ++s2) {
+            const float4 q = *reinterpret_cast<const float4*>(p + (size_t)s2 * rows_per * kRowFloats);
+            acc.x = __fadd_rn(acc.x, q.x);
+            acc.y = __fadd_rn(acc.y, q.y);
+            acc.z = __fadd_rn(acc.z, q.z);
+            acc.w = __fadd_rn(acc.w, q.w);
+          }
+          store4(args.Y, args.out_f32, (size_t)(mt * 128 + my0 + r) * args.D + nt * BN + 4 * c4, acc, scale);
+        }
       }
     }
+    if (threadIdx.x == 0) bulk_wait_read_all();  // our outgoing slices have been read
   }
 
   tc_fence_before();
@@ -433,8 +442,10 @@ template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   static_assert(BN == 128 || BN == 256, "tile width");
   using C = Cfg<BN>;
-  static_assert(128 * (BN + 4) * 4 <= C::kStages * C::kStageBytes, "split-K partial must fit the ring");
   if (a.splits < 1 || a.splits > 8) return cudaErrorInvalidValue;
+  // split-K parks the partial tile and the received slices in the ring
+  if (a.splits > 1 && 2 * 128 * (BN + 4) * 4 + 8 * (BN + 4) * 4 > C::kStages * C::kStageBytes)
+    return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
