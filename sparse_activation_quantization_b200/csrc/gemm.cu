@@ -84,10 +84,11 @@ struct GemmArgs {
   int splits;
 };
 
-template <int BN>
+template <int BN, bool kSplit>
 struct Cfg {
   static constexpr int kHalves = BN / 128;
-  static constexpr int kStages = BN == 256 ? 3 : 4;
+  // split-K CTAs do few stages and need room for the received partial rows
+  static constexpr int kStages = (kSplit || BN == 256) ? 3 : 4;
   // shared-memory stage layout (bytes); 1024-aligned where a swizzle needs it
   static constexpr int kOffB = 0;
   static constexpr int kOffAR = kOffB + BN * 128;
@@ -98,23 +99,31 @@ struct Cfg {
   static constexpr int kOffSFB32 = kOffSFAR + kSf16Tile;
   static constexpr int kOffSFB16 = kOffSFB32 + kHalves * kSf32Tile;
   static constexpr int kStageBytes = kOffSFB16 + kHalves * kSf16Tile;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-  // TMEM columns
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  // split-K receive buffer (outside the ring, so peers may write into it
+  // while this CTA's own mainloop still runs): S slices of ceil(rows/S) rows
+  static constexpr int kRowFloats = BN + 4;  // padded: conflict-free float4 access
+  static constexpr int kRecvRows = 136;      // >= 128 + S - 1 for S <= 8
+  static constexpr int kRecvBytes = kSplit ? kRecvRows * kRowFloats * 4 : 0;
+  static constexpr int kSmemBytes = kRingBytes + kRecvBytes + 1024;
+  // TMEM columns: the accumulator, then two buffers (alternating by stage)
+  // of metadata + scale factors, so the copies for stage i+1 never
+  // overwrite columns the MMAs of stage i still read.
   static constexpr uint32_t kColAcc = 0;
-  static constexpr uint32_t kColE = BN;
-  static constexpr uint32_t kColSFASP = BN + 8;
-  static constexpr uint32_t kColSFAR = BN + 16;
   static constexpr uint32_t kSfbCols = BN / 32;  // per MMA: one column per 32 rows of B
-  static constexpr uint32_t kColSFB32 = BN + 32;
-  static constexpr uint32_t kColSFB16 = kColSFB32 + 2 * kSfbCols;
-  static constexpr uint32_t kColsUsed = kColSFB16 + 4 * kSfbCols;
+  static constexpr uint32_t kSfE = 0, kSfASP = 8, kSfAR = 16, kSfB32 = 32, kSfB16 = 32 + 2 * kSfbCols;
+  static constexpr uint32_t kSfRegion = 32 + 6 * kSfbCols;
+  static constexpr uint32_t kColSf0 = BN;
+  static constexpr uint32_t kColsUsed = BN + 2 * kSfRegion;
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256 : 512;
-  // transaction bytes per stage
+  // transaction bytes per stage (activation code copies trimmed to valid rows)
   static constexpr uint32_t kTxSharq = BN * 128 + kHalves * (kSf32Tile + kSf16Tile) + kCodesTile + kSpTile +
                                        kMetaTile + kSf32Tile + kSf16Tile;
   static constexpr uint32_t kTxNvfp4 = BN * 128 + kHalves * kSf16Tile + kCodesTile + kSf16Tile;
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kColsUsed <= 512, "TMEM overflow");
+  static_assert(kSmemBytes <= 232448, "shared memory overflow");
+  static_assert(!kSplit || BN == 128, "split-K uses 128-wide tiles");
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -161,27 +170,37 @@ __device__ __forceinline__ void store4(void* Y, int out_f32, size_t off, float4 
   }
 }
 
-template <int BN>
+__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int BN, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
-  using C = Cfg<BN>;
-  constexpr int kRowFloats = BN + 4;  // padded partial row: conflict-free float4 stores
+  using C = Cfg<BN, kSplit>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::kStages];
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
   __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ __align__(8) uint64_t recv_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
-  __shared__ __align__(8) uint64_t red_bar[1];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nt = blockIdx.x, mt = blockIdx.y, split = blockIdx.z;
   const int KS = args.K >> 8;
-  const int ks0 = (int)(((long long)split * KS) / args.splits);
-  const int ks1 = (int)(((long long)(split + 1) * KS) / args.splits);
+  const int S = kSplit ? args.splits : 1;
+  const int ks0 = (int)(((long long)split * KS) / S);
+  const int ks1 = (int)(((long long)(split + 1) * KS) / S);
   const int nks = ks1 - ks0;
   const int NB = args.D >> 7;
+  const int valid = min(128, args.T - mt * 128);  // rows of this m-tile that exist
+  // split-K: CTA r of the cluster owns rows [r*rows_per, r*rows_per + my_n)
+  const int rows_per = (valid + S - 1) / S;
+  const int my0 = split * rows_per;
+  const int my_n = max(0, min(valid, my0 + rows_per) - my0);
   const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
   if (threadIdx.x == 0) TRACE_POINT(0);
 
@@ -191,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
-    mbar_init(&red_bar[0], 1);
+    // one arrival per received row: S senders x my_n rows
+    mbar_init(&recv_bar, kSplit && my_n > 0 ? (uint32_t)(S * my_n) : 1u);
     fence_mbar_init();
     abort_sh = 0;
     // expert of this m-tile (grouped form): offsets are 128-row aligned
@@ -204,7 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         const int mid = (lo + hi) >> 1;
         if (args.group_offsets[mid] <= row0) { e = mid; lo = mid + 1; } else { hi = mid - 1; }
       }
-      // skip empty groups that share this start
       while (e >= 0 && e < args.E && args.group_offsets[e + 1] <= row0) ++e;
       if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
     }
@@ -218,19 +237,11 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (args.splits > 1) {
-    cluster_sync_all();  // peers' barriers initialised before any remote traffic
-    if (threadIdx.x == 0) {
-      const int valid = min(128, args.T - mt * 128);
-      const int rows_per = (valid + args.splits - 1) / args.splits;
-      const int my0 = (int)cluster_ctarank() * rows_per, my_n = min(valid, my0 + rows_per) - my0;
-      if (my_n > 0) mbar_arrive_expect_tx(&red_bar[0], (uint32_t)(args.splits * my_n * (BN + 4) * 4));
-    }
-  }
+  if (kSplit) cluster_sync_all();  // peers' barriers initialised before any remote traffic
   if (threadIdx.x == 0) TRACE_POINT(1);
   const uint32_t tmem = tmem_base_sh;
   const int expert = expert_sh;
-  if (expert < 0) {
+  if (expert < 0) {  // (never in split mode: no groups there)
     if (threadIdx.x == 0) record_error(args.err, kErrInvalid);
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
@@ -242,10 +253,10 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
       const size_t a_tile0 = (size_t)mt * KS;
-      // copy only the valid rows of the activation code tiles
-      const uint32_t a_rows = (uint32_t)min(128, args.T - mt * 128);
-      const uint32_t a_trim = (128u - a_rows) * (sharq ? 192u : 128u);
       const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
+      // copy only the valid rows of the activation code tiles
+      const uint32_t a_rows = (uint32_t)valid;
+      const uint32_t a_trim = (128u - a_rows) * (sharq ? 192u : 128u);
       for (int i = 0; i < nks; ++i) {
         const int ks = ks0 + i;
         const int s = i % C::kStages;
@@ -267,7 +278,6 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, fb);
           if (sharq) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
         }
-        if (i == 0) TRACE_POINT(2);
         bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, a_rows * 128u, fb);
         bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
         if (sharq) {
@@ -275,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, kMetaTile, fb);
           bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
         }
+        if (i == 0) TRACE_POINT(2);
       }
     }
   } else if (warp == 1) {
@@ -292,42 +303,41 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         tc_fence_after();
         if (i == 0) TRACE_POINT(3);
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t sf = tmem + C::kColSf0 + (uint32_t)(i & 1) * C::kSfRegion;
         // scale factors (and metadata) shared memory -> TMEM
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          tc_cp_32x128b_x4(tmem + C::kColSFAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+          tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int h = 0; h < C::kHalves; ++h)
-            tc_cp_32x128b_x4(tmem + C::kColSFB16 + j * C::kSfbCols + 4 * h,
+            tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
                              smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
         if (sharq) {
-          tc_cp_128x128b(tmem + C::kColE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
+          tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
 #pragma unroll
           for (int j = 0; j < 2; ++j)
-            tc_cp_32x128b_x4(tmem + C::kColSFASP + 4 * j,
-                             smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
+            tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int h = 0; h < C::kHalves; ++h)
-              tc_cp_32x128b_x4(tmem + C::kColSFB32 + j * C::kSfbCols + 4 * h,
+              tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
                                smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
           // sparse backbone: 2 x (128 x BN x 128 logical K)
 #pragma unroll
           for (int j = 0; j < 2; ++j)
             mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffASP + 32 * j, 16, 512, kSw64),
-                        smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), tmem + C::kColE + 2 * j, idesc_sp,
-                        tmem + C::kColSFASP + 4 * j, tmem + C::kColSFB32 + j * C::kSfbCols,
-                        (i > 0 || j > 0) ? 1u : 0u);
+                        smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + C::kSfE + 2 * j, idesc_sp,
+                        sf + C::kSfASP + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, (i > 0 || j > 0) ? 1u : 0u);
         }
         // dense residual: 4 x (128 x BN x 64 K), same accumulator, same B tile
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           mma_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffAR + 32 * j, 16, 1024, kSw128),
-                   smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, tmem + C::kColSFAR + 4 * j,
-                   tmem + C::kColSFB16 + j * C::kSfbCols, (sharq || i > 0 || j > 0) ? 1u : 0u);
+                   smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + C::kSfAR + 4 * j,
+                   sf + C::kSfB16 + j * C::kSfbCols, (sharq || i > 0 || j > 0) ? 1u : 0u);
         tc_commit(&empty_bar[s]);
       }
       tc_commit(&acc_bar);  // accumulator complete (or everything issued so far, on abort)
@@ -336,97 +346,76 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   } else {
     // ------------------------------------------------------- epilogue ----
     const int sp = warp & 3;  // TMEM lane quarter this warp may access
-    const int row = mt * 128 + sp * 32 + lane;
+    const int rl = sp * 32 + lane;
     const bool ok = mbar_wait(&acc_bar, 0, deadline, &abort_sh);
     tc_fence_after();
     if (threadIdx.x == 64) TRACE_POINT(5);
     if (!ok) {
       record_error(args.err, kErrTimeout);
       abort_sh = 1;
-    } else {
+    } else if (!kSplit) {
       const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
-      const int col0 = nt * BN;
-      if (args.splits == 1) {
+      const int row = mt * 128 + rl;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
-          tmem_ld_wait();
-          if (row < args.T) store_row32(args.Y, args.out_f32, (size_t)row * args.D + col0 + c, v, scale);
-        }
-      } else {
-        // this split's fp32 partial tile -> own shared memory (valid rows)
-        float* part = reinterpret_cast<float*>(smem);
-        const int rl = sp * 32 + lane;
-        const int valid = min(128, args.T - mt * 128);
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
-          tmem_ld_wait();
-          if (rl < valid) {
-            float* dst = part + rl * kRowFloats + c;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + i) =
-                  make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]), __uint_as_float(v[i + 2]),
-                              __uint_as_float(v[i + 3]));
-          }
-        }
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the bulk copy
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+        tmem_ld_wait();
+        if (rl < valid) store_row32(args.Y, args.out_f32, (size_t)row * args.D + nt * BN + c, v, scale);
       }
+    } else {
+      // push this split's partial row straight from registers into the
+      // owner CTA's receive buffer (slot [my rank][row within the slice])
+      const int owner = rl / max(rows_per, 1);
+      const uint32_t dst =
+          rl < valid ? mapa_shared(smem_u32(smem + C::kRingBytes) +
+                                       (uint32_t)((split * rows_per + (rl - owner * rows_per)) * C::kRowFloats * 4),
+                                   (uint32_t)owner)
+                     : 0u;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+        tmem_ld_wait();
+        if (rl < valid) {
+#pragma unroll
+          for (int q = 0; q < 32; q += 4)
+            st_cluster_f4(dst + (uint32_t)(c + q) * 4u, __uint_as_float(v[q]), __uint_as_float(v[q + 1]),
+                          __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
+        }
+      }
+      // release: this thread's stores before its arrival at the owner
+      if (rl < valid) mbar_arrive_remote(mapa_shared(smem_u32(&recv_bar), (uint32_t)owner));
     }
   }
 
   if (threadIdx.x == 64) TRACE_POINT(6);
-  if (args.splits > 1) {
-    // ------------------------------------ cluster split-K reduction (push) --
-    const int S = args.splits;
-    const uint32_t rank = cluster_ctarank();
-    const int valid = min(128, args.T - mt * 128);
-    const int rows_per = (valid + S - 1) / S;
-    const uint32_t row_bytes = kRowFloats * 4u;
-    const uint32_t part_addr = smem_u32(smem);
-    const uint32_t recv_addr = part_addr + 128u * row_bytes;  // S slices of rows_per rows
-    __syncthreads();  // partial complete in this CTA
-    if (threadIdx.x == 0 && !abort_sh) {
-      for (int r = 0; r < S; ++r) {
-        const int r0 = r * rows_per, n = min(valid, r0 + rows_per) - r0;
-        if (n <= 0) continue;
-        const uint32_t dst = mapa_shared(recv_addr + rank * (uint32_t)rows_per * row_bytes, (uint32_t)r);
-        bulk_s2cluster(dst, part_addr + (uint32_t)r0 * row_bytes, (uint32_t)n * row_bytes,
-                       mapa_shared(smem_u32(&red_bar[0]), (uint32_t)r));
-      }
-      bulk_commit_group();
+  if (kSplit && my_n > 0) {
+    // ------------------------ owner: sum the S received slices in rank order
+    bool ok = !abort_sh;
+    while (ok && !mbar_try_wait_cluster(&recv_bar, 0)) {
+      if (globaltimer_ns() > deadline) ok = false;
     }
-    const int my0 = (int)rank * rows_per, my_n = min(valid, my0 + rows_per) - my0;
-    if (my_n > 0) {
-      bool ok = !abort_sh;
-      while (ok && !mbar_try_wait_cluster(&red_bar[0], 0)) {
-        if (globaltimer_ns() > deadline) ok = false;
-      }
-      if (!ok) {
-        if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
-      } else {
-        const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
-        const float* recv = reinterpret_cast<const float*>(smem + 128u * row_bytes);
-        constexpr int q4 = BN / 4;
-        for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
-          const int r = idx / q4, c4 = idx - r * q4;
-          const float* p = recv + r * kRowFloats + 4 * c4;
-          float4 acc = *reinterpret_cast<const float4*>(p);
-          for (int s2 = 1; s2 < S; ++s2) {
-            const float4 q = *reinterpret_cast<const float4*>(p + (size_t)s2 * rows_per * kRowFloats);
-            acc.x = __fadd_rn(acc.x, q.x);
-            acc.y = __fadd_rn(acc.y, q.y);
-            acc.z = __fadd_rn(acc.z, q.z);
-            acc.w = __fadd_rn(acc.w, q.w);
-          }
-          store4(args.Y, args.out_f32, (size_t)(mt * 128 + my0 + r) * args.D + nt * BN + 4 * c4, acc, scale);
+    if (!ok) {
+      if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
+    } else {
+      const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
+      const float* recv = reinterpret_cast<const float*>(smem + C::kRingBytes);
+      constexpr int q4 = BN / 4;
+      for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
+        const int r = idx / q4, c4 = idx - r * q4;
+        const float* p = recv + r * C::kRowFloats + 4 * c4;
+        float4 acc = *reinterpret_cast<const float4*>(p);
+        for (int s2 = 1; s2 < S; ++s2) {
+          const float4 q = *reinterpret_cast<const float4*>(p + (size_t)s2 * rows_per * C::kRowFloats);
+          acc.x = __fadd_rn(acc.x, q.x);
+          acc.y = __fadd_rn(acc.y, q.y);
+          acc.z = __fadd_rn(acc.z, q.z);
+          acc.w = __fadd_rn(acc.w, q.w);
         }
+        store4(args.Y, args.out_f32, (size_t)(mt * 128 + my0 + r) * args.D + nt * BN + 4 * c4, acc, scale);
       }
     }
-    if (threadIdx.x == 0) bulk_wait_read_all();  // our outgoing slices have been read
   }
 
   tc_fence_before();
@@ -438,25 +427,21 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   }
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
-  static_assert(BN == 128 || BN == 256, "tile width");
-  using C = Cfg<BN>;
-  if (a.splits < 1 || a.splits > 8) return cudaErrorInvalidValue;
-  // split-K parks the partial tile and the received slices in the ring
-  if (a.splits > 1 && 2 * 128 * (BN + 4) * 4 + 8 * (BN + 4) * 4 > C::kStages * C::kStageBytes)
-    return cudaErrorInvalidValue;
+template <int BN, bool kSplit>
+cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
+  using C = Cfg<BN, kSplit>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(sharq_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(sharq_gemm_kernel<BN, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.D / BN, m_tiles, a.splits);
+  cfg.gridDim = dim3(a.D / BN, m_tiles, kSplit ? a.splits : 1);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
@@ -464,10 +449,10 @@ cudaError_t launch_bn(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = a.splits;
+  attr[0].val.clusterDim.z = kSplit ? a.splits : 1;
   cfg.attrs = attr;
-  cfg.numAttrs = a.splits > 1 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<BN>, a);
+  cfg.numAttrs = kSplit ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<BN, kSplit>, a);
 }
 
 }  // namespace
@@ -507,7 +492,11 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.splits = splits;
   const int m_tiles = Tp / 128;
   if (m_tiles == 0) return cudaSuccess;
-  return bn == 256 ? launch_bn<256>(a, m_tiles, stream) : launch_bn<128>(a, m_tiles, stream);
+  if (splits > 1) {
+    if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
+    return launch_cfg<128, true>(a, m_tiles, stream);
+  }
+  return bn == 256 ? launch_cfg<256, false>(a, m_tiles, stream) : launch_cfg<128, false>(a, m_tiles, stream);
 }
 
 }  // namespace sharq
