@@ -5,19 +5,21 @@
 // residual construction in one preparation step) and sections 3.2-3.3 for
 // what is computed; kasblo.com explainer, steps 1-3 of the recipe.
 //
-// Two launches, because the per-tensor scale (PTS) is a device-wide max that
-// every quantization step needs before it can emit a code:
-//   prep_stats_kernel  one CTA per row: sum of squares (float64) -> 1/rms,
-//                      then max |Xn| of the row -> atomicMax into gmax.
-//   prep_quant_kernel  one thread per (row, 32 logical K): reload the row
-//                      segment (L2-resident for tensors below ~100 MB), redo
-//                      Xn, pick the 2 of 4 pairs in each run of 8, quantize
-//                      the 16 kept values (one E4M3 scale per 32 logical K),
-//                      form R = Xn - dequant(backbone) in registers, quantize
-//                      R in two 16-element blocks, store every output in the
-//                      MMA-ready tiled layout of include/sharq.h.
-// Loads are 128-bit and coalesced (consecutive threads take consecutive
-// 64-byte row segments); the residual never leaves registers.
+// The per-tensor scale (PTS) is a device-wide max that every quantization
+// step needs before it can emit a code.  Two forms:
+//   single launch (prep_fused_kernel): a cooperative grid holds the whole
+//     tensor in registers -- load, RMSNorm, device-wide max through a bounded
+//     grid barrier, then quantize; X is read once.  Used whenever the grid
+//     fits on the GPU at once.
+//   two launches (larger tensors): prep_stats_kernel (one CTA per row:
+//     float64 sum of squares -> 1/rms, row max |Xn| -> atomicMax), then
+//     prep_quant_kernel (re-reads X, L2-resident up to ~100 MB).
+// Work unit: one thread per run of 8 consecutive K (one 16-byte load, one
+// 4:8 in-pairs chunk); rows longer than 8192 give each thread 2 or 4 runs.
+// The 32-K backbone block and the 16-K residual block span 4 and 2 such
+// threads (adjacent lanes), reduced with warp shuffles.  The residual never
+// leaves registers; every output is stored in the MMA-ready tiled layout of
+// include/sharq.h.
 #include "sharq_device.cuh"
 
 namespace sharq {
@@ -126,27 +128,6 @@ __device__ __forceinline__ float pick4(const float* a, int sel) {
   return r;
 }
 
-// 16 values -> 8 bytes of E2M1 codes (value 2i in the low nibble of byte i)
-__device__ __forceinline__ uint2 quant16(const float* v, float inv, uint32_t* codes) {
-  uint32_t b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    b[i] = cvt_e2m1x2(__fmul_rn(v[2 * i], inv), __fmul_rn(v[2 * i + 1], inv));
-    codes[2 * i] = b[i] & 0xFu;
-    codes[2 * i + 1] = b[i] >> 4;
-  }
-  uint2 out;
-  out.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-  return out;
-}
-
-__device__ __forceinline__ float amax_n(const float* v, int n) {
-  float a = 0.0f;
-  for (int i = 0; i < n; ++i) a = fmaxf(a, fabsf(v[i]));
-  return a;
-}
-
 struct QuantPtrs {
   uint8_t* sp_codes;
   uint8_t* meta;
@@ -155,221 +136,239 @@ struct QuantPtrs {
   uint8_t* r_sf;
 };
 
-constexpr int kQuantThreads = 256;
+// max over the `width` adjacent lanes of an aligned lane group
+__device__ __forceinline__ float group_max(float v, int width) {
+  for (int o = 1; o < width; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 
-// Quantize one row segment of 32 logical K (row t, 32-block j) held in
-// registers: mask, backbone NVFP4, residual, dense NVFP4, tiled stores.
-template <bool kSharq>
-__device__ __forceinline__ void quant_segment(const float (&x)[32], int t, int j, int K, float s, float six_s,
-                                              const QuantPtrs& out) {
+// Quantize NC consecutive runs of 8 logical K of row t, held in registers
+// (x[8*c + e] = run c, element e), starting at run index c0 of the row.
+// All 32 lanes of the warp must call it (warp shuffles).
+template <int NC, bool kSharq>
+__device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int c0, int K, float s, float six_s,
+                                           const QuantPtrs& out) {
   const int KS = K >> 8;
-  const int kt = j >> 3, q = j & 7;
   const int r = t & 127;
-  const size_t tile = (size_t)(t >> 7) * KS + kt;
+  float res[8 * NC];
+#pragma unroll
+  for (int i = 0; i < 8 * NC; ++i) res[i] = x[i];
 
-  float res[32];
   if (kSharq) {
-    // --- 4:8 in-pairs mask: keep the 2 of 4 pairs with the largest max|x| ---
-    float v[16];
-    int lo[4], hi[4];
-    uint32_t meta16 = 0;
+    // --- 4:8 in-pairs mask per run: keep the 2 of 4 pairs with the largest max|x|
+    float v[4 * NC];
+    int lo[NC], hi[NC];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float sc[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) sc[p] = fmaxf(fabsf(x[8 * c + 2 * p]), fabsf(x[8 * c + 2 * p + 1]));
-      bool keep[4];
+    for (int c = 0; c < NC; ++c) {
+      float sc[4], ev[4], od[4];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
+        ev[p] = x[8 * c + 2 * p];
+        od[p] = x[8 * c + 2 * p + 1];
+        sc[p] = fmaxf(fabsf(ev[p]), fabsf(od[p]));
+      }
+      int a = -1, b = -1;
+#pragma unroll
+      for (int p = 3; p >= 0; --p) {
         int beaten = 0;
 #pragma unroll
         for (int o = 0; o < 4; ++o)
           if (o != p) beaten += (sc[o] > sc[p]) || (sc[o] == sc[p] && o < p);
-        keep[p] = beaten < 2;
+        if (beaten < 2) { b = a; a = p; }
       }
-      int a = -1, b = -1;
-#pragma unroll
-      for (int p = 3; p >= 0; --p)
-        if (keep[p]) { b = a; a = p; }
       lo[c] = a;
       hi[c] = b;
-      meta16 |= (uint32_t)(a | (b << 2)) << (4 * c);
-      float ev[4], od[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) { ev[p] = x[8 * c + 2 * p]; od[p] = x[8 * c + 2 * p + 1]; }
       v[4 * c + 0] = pick4(ev, a);
       v[4 * c + 1] = pick4(od, a);
       v[4 * c + 2] = pick4(ev, b);
       v[4 * c + 3] = pick4(od, b);
     }
-    // --- backbone NVFP4: one scale for these 32 logical K (16 kept values) ---
-    const BlockScale bs = block_scale(amax_n(v, 16), six_s, s);
-    uint32_t code[16];
-    const uint2 spc = quant16(v, bs.inv, code);
-    // --- residual R = Xn - dequant(backbone), exact float32 per element ---
+    // --- backbone NVFP4: one scale per 32 logical K (4 runs = 16 kept values)
+    float am = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) res[i] = x[i];
+    for (int i = 0; i < 4 * NC; ++i) am = fmaxf(am, fabsf(v[i]));
+    if (NC < 4) am = group_max(am, 4 / NC);
+    const BlockScale bs = block_scale(am, six_s, s);
+    uint32_t code[4 * NC];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int i = 0; i < 2 * NC; ++i) {
+      const uint32_t by = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
+      code[2 * i] = by & 0xFu;
+      code[2 * i + 1] = by >> 4;
+    }
+    // --- residual R = Xn - dequant(backbone) at kept positions (exact fp32)
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const bool is_lo = (p == lo[c]), is_hi = (p == hi[c]);
         if (is_lo || is_hi) {
-          const int slot = is_lo ? 0 : 2;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            uint32_t cd = code[4 * c + e];
-            cd = slot ? code[4 * c + 2 + e] : cd;
+            const uint32_t cd = is_lo ? code[4 * c + e] : code[4 * c + 2 + e];
             const float xt = __fmul_rn(__fmul_rn(e2m1_value(cd), bs.dec), s);
             res[8 * c + 2 * p + e] = __fsub_rn(x[8 * c + 2 * p + e], xt);
           }
         }
       }
     }
-    // --- stores: sparse codes, metadata, sparse scale ---
-    *reinterpret_cast<uint2*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, q >> 1) + (q & 1) * 8) = spc;
-    *reinterpret_cast<uint16_t*>(out.meta + tile * kMetaTile + r * 16 + q * 2) = (uint16_t)meta16;
-    out.sp_sf[tile * kSf32Tile + sf_off(r, q >> 2, q & 3)] = (uint8_t)bs.sb;
-  } else {
+    // --- stores: per run 2 bytes of kept codes, one metadata nibble
 #pragma unroll
-    for (int i = 0; i < 32; ++i) res[i] = x[i];
+    for (int c = 0; c < NC; ++c) {
+      const int g = c0 + c;            // run index in the row
+      const int kt = g >> 5, w = g & 31;  // K tile, run within the 256-K tile
+      const size_t tile = (size_t)(t >> 7) * KS + kt;
+      const uint32_t b0 = code[4 * c] | (code[4 * c + 1] << 4), b1 = code[4 * c + 2] | (code[4 * c + 3] << 4);
+      *reinterpret_cast<uint16_t*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
+          (uint16_t)(b0 | (b1 << 8));
+      uint32_t nib = (uint32_t)(lo[c] | (hi[c] << 2));
+      if (NC == 1) {
+        const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
+        if ((w & 1) == 0) out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
+      } else if ((c & 1) == 0) {
+        const uint32_t other = (uint32_t)(lo[c + 1 < NC ? c + 1 : c] | (hi[c + 1 < NC ? c + 1 : c] << 2));
+        out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
+      }
+      if ((w & 3) == 0) out.sp_sf[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
+    }
   }
 
-  // --- dense NVFP4 of R (or of Xn in NVFP4 mode): two 16-element blocks ---
-  const BlockScale b0 = block_scale(amax_n(res, 16), six_s, s);
-  const BlockScale b1 = block_scale(amax_n(res + 16, 16), six_s, s);
-  uint32_t dummy[16];
-  const uint2 c0 = quant16(res, b0.inv, dummy);
-  const uint2 c1 = quant16(res + 16, b1.inv, dummy);
-  *reinterpret_cast<uint4*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, q)) =
-      make_uint4(c0.x, c0.y, c1.x, c1.y);
-  *reinterpret_cast<uint16_t*>(out.r_sf + tile * kSf16Tile + sf_off(r, q >> 1, 2 * (q & 1))) =
-      (uint16_t)(b0.sb | (b1.sb << 8));
+  // --- dense NVFP4 of R (or of Xn in NVFP4 mode): 16-element blocks
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    float am = 0.0f;
+    if (NC == 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(res[i]));
+      am = group_max(am, 2);
+    } else {
+      const int c2 = c & ~1;  // this run and its partner form one block
+#pragma unroll
+      for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(res[8 * c2 + i]));
+    }
+    const BlockScale bs = block_scale(am, six_s, s);
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      word |= cvt_e2m1x2(__fmul_rn(res[8 * c + 2 * i], bs.inv), __fmul_rn(res[8 * c + 2 * i + 1], bs.inv)) << (8 * i);
+    const int g = c0 + c;
+    const int kt = g >> 5, w = g & 31;
+    const size_t tile = (size_t)(t >> 7) * KS + kt;
+    *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) = word;
+    if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+  }
 }
 
+// load NC runs of 8 (one 16-byte load each) and normalise them
+template <int NC>
+__device__ __forceinline__ void load_runs(float (&x)[8 * NC], const __nv_bfloat16* X, int src, int K, int c0) {
+  if (src >= 0) {
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K) + c0;
+    uint4 raw[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) raw[c] = xr[c];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) bf16x8_to_float(raw[c], x + 8 * c);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8 * NC; ++i) x[i] = 0.0f;
+  }
+}
 
+template <int NC>
+__device__ __forceinline__ void normalise_runs(float (&x)[8 * NC], const __nv_bfloat16* gamma, int c0, float inv) {
+  const uint4* gr = reinterpret_cast<const uint4*>(gamma) + c0;
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    float g[8];
+    bf16x8_to_float(gr[c], g);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[8 * c + e] = norm_one(x[8 * c + e], inv, g[e]);
+  }
+}
+
+constexpr int kQuantThreads = 256;
+
+// Two-launch form, second launch: one thread per run of 8, flat over rows.
 template <bool kSharq>
 __global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
     const int* __restrict__ row_index, int T, int Tp, int K, const float* __restrict__ inv_rms,
     const unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
-  const int nb32 = K >> 5;
+  const int runs = K >> 3;
   const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
   const float gmax = __uint_as_float(*gmax_bits);
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (gid == 0) *s_g_out = s;  // published even when there are no rows
-  if (gid >= (long long)Tp * nb32) return;
-  const int t = (int)(gid / nb32);
-  const int j = (int)(gid - (long long)t * nb32);
-  const float six_s = __fmul_rn(6.0f, s);
-
-  // --- load the 32 values of this row segment and normalise them ---
-  float x[32];
+  // whole warps exit together: rows span whole warps (K/8 is a multiple of 32)
+  if (gid >= (long long)Tp * runs) return;
+  const int t = (int)(gid / runs);
+  const int c0 = (int)(gid - (long long)t * runs);
   int src = -1;
   if (t < T) src = row_index ? row_index[t] : t;
-  if (src >= 0) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * j);
-    uint4 raw[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) raw[i] = xr[i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) bf16x8_to_float(raw[i], x + 8 * i);
-    if (gamma) {
-      const float inv = inv_rms[t];
-      const uint4* gr = reinterpret_cast<const uint4*>(gamma + 32 * j);
-      float g[32];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) bf16x8_to_float(gr[i], g + 8 * i);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] = norm_one(x[i], inv, g[i]);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = 0.0f;
-  }
-
-  quant_segment<kSharq>(x, t, j, K, s, six_s, out);
+  float x[8];
+  load_runs<1>(x, X, src, K, c0);
+  if (gamma && src >= 0) normalise_runs<1>(x, gamma, c0, inv_rms[t]);
+  quant_runs<1, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
 }
 
-
 // ---------------------------------------------------------------------------
-// Single-launch form: one cooperative grid, one thread per (row, 32-K block),
-// whole rows inside a CTA (rows_per_cta x K/32 threads).  The row's values
-// stay in registers from the load to the stores:
-//   1. load + sum of squares (float64, fixed-order tree per row) -> 1/rms,
-//      normalise in registers, CTA max |Xn|  -> atomicMax(gmax);
-//   2. grid-wide barrier (arrival counter, bounded spin on the global timer);
-//   3. quantize from registers (same code as prep_quant_kernel).
-// X is read from HBM exactly once.  Used whenever the grid fits on the GPU at
-// once (cooperative launch guarantees co-residency); larger tensors take the
-// two-launch path above.
-constexpr int kFusedMaxThreads = 640;            // K/32 <= 592 threads per row
+// Single-launch form (cooperative grid; whole rows inside a CTA).
+constexpr int kFusedMaxThreads = 1024;
 constexpr uint64_t kBarrierLimitNs = 2000000000ull;
 
-template <bool kSharq>
-__global__ void __launch_bounds__(kFusedMaxThreads) prep_fused_kernel(
+template <int NC>
+constexpr int fused_max_threads() { return NC == 4 ? 640 : kFusedMaxThreads; }
+
+template <int NC, bool kSharq>
+__global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
     unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out) {
-  __shared__ double part[kFusedMaxThreads];
+  __shared__ double wsum[kFusedMaxThreads / 32];
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
-  const int nb32 = K >> 5;
-  const int rl = threadIdx.x / nb32;
-  const int j = threadIdx.x - rl * nb32;
+  const int tpr = (K >> 3) / NC;            // threads per row (multiple of 32)
+  const int rl = threadIdx.x / tpr;
+  const int c0 = (threadIdx.x - rl * tpr) * NC;
   const int t = blockIdx.x * rows_per_cta + rl;
   const bool live = t < Tp;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpr = tpr >> 5;                 // warps per row
 
-  float x[32];
+  float x[8 * NC];
   int src = -1;
   if (live && t < T) src = row_index ? row_index[t] : t;
-  if (src >= 0) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * j);
-    uint4 raw[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) raw[i] = xr[i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) bf16x8_to_float(raw[i], x + 8 * i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = 0.0f;
-  }
+  load_runs<NC>(x, X, src, K, c0);
 
   if (gamma) {
     double ss = 0.0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) ss += (double)x[i] * (double)x[i];
-    part[threadIdx.x] = ss;
+    for (int i = 0; i < 8 * NC; ++i) ss += (double)x[i] * (double)x[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) wsum[warp] = ss;
     __syncthreads();
-    int span = 1;
-    while (span < nb32) span <<= 1;
-    for (int off = span >> 1; off > 0; off >>= 1) {
-      if (j < off && j + off < nb32) part[threadIdx.x] += part[threadIdx.x + off];
-      __syncthreads();
-    }
-    const float inv = (float)(1.0 / sqrt(part[rl * nb32] / (double)K + (double)eps));
-    if (live && t < T && j == 0) inv_rms[t] = inv;
-    const uint4* gr = reinterpret_cast<const uint4*>(gamma + 32 * j);
-    float g[32];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) bf16x8_to_float(gr[i], g + 8 * i);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = norm_one(x[i], inv, g[i]);
-  } else if (live && t < T && j == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < wpr; ++w) tot += wsum[rl * wpr + w];  // fixed order
+    const float inv = (float)(1.0 / sqrt(tot / (double)K + (double)eps));
+    if (live && t < T && c0 == 0) inv_rms[t] = inv;
+    if (src >= 0) normalise_runs<NC>(x, gamma, c0, inv);
+  } else if (live && t < T && c0 == 0) {
     inv_rms[t] = 1.0f;
   }
 
   // CTA max |Xn| -> device-wide max
   float a = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+  for (int i = 0; i < 8 * NC; ++i) a = fmaxf(a, fabsf(x[i]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = a;
+  if (lane == 0) wmax[warp] = a;
   __syncthreads();
   if (threadIdx.x == 0) {
     float m = 0.0f;
-    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) m = fmaxf(m, wmax[w]);
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
     atomicMax(sync, __float_as_uint(m));
     __threadfence();
     atomicAdd(sync + 1, 1u);
@@ -392,35 +391,68 @@ __global__ void __launch_bounds__(kFusedMaxThreads) prep_fused_kernel(
   const float gmax = gmax_sh;
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
-  if (live) quant_segment<kSharq>(x, t, j, K, s, __fmul_rn(6.0f, s), out);
+  // rows past Tp: whole warps (rows span whole warps), so they can skip
+  if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
 }
 
-
-// rows per CTA of the single-launch form for a row length of K
-int fused_rows_per_cta(int K) {
-  const int nb32 = K >> 5;
-  if (nb32 > kFusedMaxThreads) return 0;
-  return nb32 >= 256 ? 1 : 256 / nb32;
+// runs of 8 per thread so that a row fits one CTA (<= 1024 threads)
+int fused_runs_per_thread(int K) {
+  const int runs = K >> 3;
+  if (runs <= 1024) return 1;
+  if (runs <= 2048) return 2;
+  if (runs <= 4 * 640) return 4;
+  return 0;
 }
 
-// Largest grid of the single-launch form that can be resident at once.
-int fused_max_ctas(bool sharq_mode, int threads) {
-  static int cache[2][kFusedMaxThreads + 1][64] = {};
+template <int NC, bool kSharq>
+int fused_max_ctas_t(int threads) {
+  static int cache[kFusedMaxThreads + 1][64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
-  int& c = cache[sharq_mode ? 1 : 0][threads][dev];
+  int& c = cache[threads][dev];
   if (c == 0) {
     int per_sm = 0, sms = 0;
-    cudaError_t e = sharq_mode
-        ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<true>, threads, 0)
-        : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<false>, threads, 0);
-    if (e != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<NC, kSharq>, threads, 0) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
     c = per_sm * sms > 0 ? per_sm * sms : -1;
   }
   return c > 0 ? c : 0;
+}
+
+template <int NC, bool kSharq>
+cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
+                      int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
+                      cudaStream_t stream, bool* launched) {
+  *launched = false;
+  const int tpr = (K >> 3) / NC;
+  int rpc = 512 / tpr;
+  rpc = rpc < 1 ? 1 : rpc;
+  const int threads = rpc * tpr;
+  const int ctas = (Tp + rpc - 1) / rpc;
+  if (ctas > fused_max_ctas_t<NC, kSharq>(threads)) return cudaSuccess;
+  void* args[] = {(void*)&Xb, (void*)&Gb, (void*)&eps, (void*)&row_index, (void*)&T, (void*)&Tp, (void*)&K,
+                  (void*)&rpc, (void*)&inv_rms, (void*)&sync, (void*)&s_g, (void*)&p};
+  cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(prep_fused_kernel<NC, kSharq>),
+                                              dim3(ctas), dim3(threads), args, 0, stream);
+  if (e == cudaSuccess) *launched = true;
+  else cudaGetLastError();  // fall back to the two-launch form
+  return cudaSuccess;
+}
+
+template <bool kSharq>
+cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
+                          int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
+                          cudaStream_t stream, bool* launched) {
+  switch (fused_runs_per_thread(K)) {
+    case 1: return try_fused<1, kSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    case 2: return try_fused<2, kSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    case 4: return try_fused<4, kSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    default: *launched = false; return cudaSuccess;
+  }
 }
 
 }  // namespace
@@ -436,25 +468,20 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
 
-  const int rpc = fused_rows_per_cta(K);
-  if (Tp > 0 && rpc > 0) {
-    const int threads = rpc * (K >> 5);
-    const int ctas = (Tp + rpc - 1) / rpc;
-    if (ctas <= fused_max_ctas(sharq_mode, threads)) {
-      void* args[] = {(void*)&Xb, (void*)&Gb, (void*)&eps, (void*)&row_index, (void*)&T, (void*)&Tp, (void*)&K,
-                      (void*)&rpc, (void*)&inv_rms, (void*)&gmax_bits, (void*)&s_g, (void*)&p};
-      const void* fn = sharq_mode ? reinterpret_cast<const void*>(prep_fused_kernel<true>)
-                                  : reinterpret_cast<const void*>(prep_fused_kernel<false>);
-      e = cudaLaunchCooperativeKernel(fn, dim3(ctas), dim3(threads), args, 0, stream);
-      if (e == cudaSuccess) return cudaSuccess;
-      cudaGetLastError();  // fall back to the two-launch form below
-    }
+  if (Tp > 0) {
+    bool launched = false;
+    e = sharq_mode ? try_fused_any<true>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+                                         &launched)
+                   : try_fused_any<false>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+                                          &launched);
+    if (e != cudaSuccess) return e;
+    if (launched) return cudaSuccess;
   }
 
   if (T > 0) {
     prep_stats_kernel<<<T, kStatsThreads, 0, stream>>>(Xb, Gb, eps, row_index, K, inv_rms, gmax_bits);
   }
-  const long long n = (long long)Tp * (K >> 5);
+  const long long n = (long long)Tp * (K >> 3);
   // at least one block so that s_g is published (= 1) even for T == 0
   const unsigned grid = n > 0 ? (unsigned)((n + kQuantThreads - 1) / kQuantThreads) : 1u;
   if (sharq_mode)

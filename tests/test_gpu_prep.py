@@ -94,6 +94,15 @@ def test_prep_bit_exact(name, T, K, kw, gam, eps):
     _check_sharq(x, gamma, eps)
 
 
+@pytest.mark.parametrize("T,K", [(64, 14336), (32, 18944), (33, 3584)])
+def test_prep_long_rows_bit_exact(T, K):
+    """Rows longer than 8192 give each thread 2 or 4 runs of 8 in the
+    single-launch form (Llama MLP down_proj K = 14336, Qwen2.5-7B down_proj
+    K = 18944, Qwen2.5-7B hidden 3584)."""
+    x = synthetic.activations(77 + T, T, K, base="student_t")
+    _check_sharq(x, synthetic.gamma(78, K), 1e-6)
+
+
 @pytest.mark.parametrize("T,K", [(400, 14336), (700, 8192)])
 def test_prep_two_launch_path_bit_exact(T, K):
     """Tensors too large for one co-resident grid take the two-launch form
