@@ -147,7 +147,7 @@ __device__ __forceinline__ float group_max(float v, int width) {
 // All 32 lanes of the warp must call it (warp shuffles).
 template <int NC, bool kSharq>
 __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int c0, int K, float s, float six_s,
-                                           const QuantPtrs& out) {
+                                           const QuantPtrs& out, bool store = true) {
   const int KS = K >> 8;
   const int r = t & 127;
   float res[8 * NC];
@@ -219,17 +219,18 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
       const int kt = g >> 5, w = g & 31;  // K tile, run within the 256-K tile
       const size_t tile = (size_t)(t >> 7) * KS + kt;
       const uint32_t b0 = code[4 * c] | (code[4 * c + 1] << 4), b1 = code[4 * c + 2] | (code[4 * c + 3] << 4);
-      *reinterpret_cast<uint16_t*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
-          (uint16_t)(b0 | (b1 << 8));
+      if (store)
+        *reinterpret_cast<uint16_t*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
+            (uint16_t)(b0 | (b1 << 8));
       uint32_t nib = (uint32_t)(lo[c] | (hi[c] << 2));
       if (NC == 1) {
         const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
-        if ((w & 1) == 0) out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
-      } else if ((c & 1) == 0) {
+        if (store && (w & 1) == 0) out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
+      } else if (store && (c & 1) == 0) {
         const uint32_t other = (uint32_t)(lo[c + 1 < NC ? c + 1 : c] | (hi[c + 1 < NC ? c + 1 : c] << 2));
         out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
       }
-      if ((w & 3) == 0) out.sp_sf[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
+      if (store && (w & 3) == 0) out.sp_sf[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
     }
   }
 
@@ -254,8 +255,11 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
     const int g = c0 + c;
     const int kt = g >> 5, w = g & 31;
     const size_t tile = (size_t)(t >> 7) * KS + kt;
-    *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) = word;
-    if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+    if (store) {
+      *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
+          word;
+      if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+    }
   }
 }
 
@@ -328,9 +332,14 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   __shared__ double wsum[kFusedMaxThreads / 32];
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
-  const int tpr = (K >> 3) / NC;            // threads per row (multiple of 32)
+  // threads per row, padded to whole warps (a warp never spans two rows);
+  // the padding lanes hold zeros and store nothing
+  const int used = (K >> 3) / NC;
+  const int tpr = (used + 31) & ~31;
   const int rl = threadIdx.x / tpr;
-  const int c0 = (threadIdx.x - rl * tpr) * NC;
+  const int li = threadIdx.x - rl * tpr;
+  const bool has = li < used;
+  const int c0 = (has ? li : 0) * NC;
   const int t = blockIdx.x * rows_per_cta + rl;
   const bool live = t < Tp;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -338,7 +347,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
 
   float x[8 * NC];
   int src = -1;
-  if (live && t < T) src = row_index ? row_index[t] : t;
+  if (live && t < T && has) src = row_index ? row_index[t] : t;
   load_runs<NC>(x, X, src, K, c0);
 
   if (gamma) {
@@ -352,9 +361,9 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     double tot = 0.0;
     for (int w = 0; w < wpr; ++w) tot += wsum[rl * wpr + w];  // fixed order
     const float inv = (float)(1.0 / sqrt(tot / (double)K + (double)eps));
-    if (live && t < T && c0 == 0) inv_rms[t] = inv;
+    if (live && t < T && li == 0) inv_rms[t] = inv;
     if (src >= 0) normalise_runs<NC>(x, gamma, c0, inv);
-  } else if (live && t < T && c0 == 0) {
+  } else if (live && t < T && li == 0) {
     inv_rms[t] = 1.0f;
   }
 
@@ -392,14 +401,14 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
   // rows past Tp: whole warps (rows span whole warps), so they can skip
-  if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
+  if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
 }
 
 // runs of 8 per thread so that a row fits one CTA (<= 1024 threads)
 int fused_runs_per_thread(int K) {
   const int runs = K >> 3;
   if (runs <= 1024) return 1;
-  if (runs <= 2048) return 2;
+  if (runs <= 2048 && (runs / 2) % 2 == 0) return 2;
   if (runs <= 4 * 640) return 4;
   return 0;
 }
@@ -428,7 +437,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
                       int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
                       cudaStream_t stream, bool* launched) {
   *launched = false;
-  const int tpr = (K >> 3) / NC;
+  const int tpr = (((K >> 3) / NC) + 31) & ~31;
   int rpc = 512 / tpr;
   rpc = rpc < 1 ? 1 : rpc;
   const int threads = rpc * tpr;
