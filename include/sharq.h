@@ -116,8 +116,12 @@ typedef struct {
  *   inv_rms: Tp floats (1/rms per row; 1 when RMSNorm is off).
  *   s_g:     the per-tensor global scale gmax / (6*448) (1 if gmax == 0).
  *   gmax_bits: 16 bytes of scratch: device-wide amax, grid-barrier count,
- *            reserved, and an error word that sharq_linear forwards to its
- *            workspace (a prep whose grid barrier timed out).
+ *            departure count, and an error word that sharq_linear forwards
+ *            to its workspace (a prep whose grid barrier timed out).
+ *   The 256-byte scalar block that starts at s_g (s_g, gmax_bits[0..3])
+ *   must be zero before the first sharq_prep on a buffer (zero the whole
+ *   buffer once after allocation); sharq_prep leaves gmax_bits[0..2] zero
+ *   again, so no per-call memset is needed.
  */
 typedef struct {
   void *sp_codes;
@@ -182,6 +186,9 @@ int sharq_prep(const void *d_X, const void *d_gamma, float eps, const int *d_row
  * FP4 MMA on the residual accumulate into one TMEM accumulator per output
  * tile; neither branch output is materialised.  Both read the same weight
  * codes, through sf32 (sparse) and sf16 (dense).
+ * Launched as a programmatic dependent of the preceding kernel in the
+ * stream: set-up and the first weight tiles overlap the tail of sharq_prep,
+ * and the activation is read only after that kernel has completed.
  * Y = round(f32(acc * f32(s_g * s_w))) written to d_Y [T][D] row-major,
  * bf16 or float32 per out_dtype.  Mode NVFP4 runs the dense MMA only.
  * d_ws: workspace of at least sharq_workspace_bytes(T, K, D, 1) bytes, zeroed

@@ -204,6 +204,12 @@ class PreparedAct:
         self.T, self.K, self.mode = T, K, mode
         self.buf = _buffer(nbytes, device)
         self.view = sharq_act_view(self.buf.data_ptr(), T, K, mode)
+        self.reset()
+
+    def reset(self):
+        """Zero the scalar block (s_g and the prep's sync words), as the C ABI
+        requires before the first sharq_prep on a buffer."""
+        self.region("s_g", 256).zero_()
 
     def prep(self, X, gamma=None, eps=1e-5, row_index=None, stream=None):
         sharq_prep(X.data_ptr() if X is not None else None,

@@ -170,6 +170,10 @@ __device__ __forceinline__ void store4(void* Y, int out_f32, size_t off, float4 
   }
 }
 
+// Programmatic dependent launch: wait until the preceding grid in the stream
+// has completed and its memory is visible (returns at once if there is none).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -228,7 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
     }
     expert_sh = e;
-    if (blockIdx.x == 0 && blockIdx.z == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, C::kTmemCols);
@@ -257,27 +260,16 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       // copy only the valid rows of the activation code tiles
       const uint32_t a_rows = (uint32_t)valid;
       const uint32_t a_trim = (128u - a_rows) * (sharq ? 192u : 128u);
-      for (int i = 0; i < nks; ++i) {
-        const int ks = ks0 + i;
-        const int s = i % C::kStages;
-        if (i >= C::kStages) {
-          if (!mbar_wait(&empty_bar[s], ((i / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
-            record_error(args.err, kErrTimeout);
-            abort_sh = 1;
-            break;
-          }
-        }
-        uint8_t* st = smem + s * C::kStageBytes;
-        uint64_t* fb = &full_bar[s];
-        mbar_arrive_expect_tx(fb, (sharq ? C::kTxSharq : C::kTxNvfp4) - a_trim);
-        const size_t at = a_tile0 + ks;
+      auto issue_b = [&](uint8_t* st, uint64_t* fb, size_t b_tile, int ks) {
 #pragma unroll
         for (int h = 0; h < C::kHalves; ++h) {
-          const size_t bt = b_tile0 + (size_t)h * KS + ks;
+          const size_t bt = b_tile + (size_t)h * KS + ks;
           bulk_g2s(st + C::kOffB + h * kCodesTile, args.w_codes + bt * kCodesTile, kCodesTile, fb);
           bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, fb);
           if (sharq) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
         }
+      };
+      auto issue_a = [&](uint8_t* st, uint64_t* fb, size_t at) {
         bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, a_rows * 128u, fb);
         bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
         if (sharq) {
@@ -285,7 +277,31 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, kMetaTile, fb);
           bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
         }
-        if (i == 0) TRACE_POINT(2);
+      };
+      // The weights do not depend on the preceding kernel (sharq_prep): issue
+      // the weight copies of the first ring's worth of stages before waiting
+      // for it (programmatic dependent launch), then the activation copies.
+      const int pre = nks < C::kStages ? nks : C::kStages;
+      for (int i = 0; i < pre; ++i) {
+        uint8_t* st = smem + i * C::kStageBytes;
+        mbar_arrive_expect_tx(&full_bar[i], (sharq ? C::kTxSharq : C::kTxNvfp4) - a_trim);
+        issue_b(st, &full_bar[i], b_tile0, ks0 + i);
+      }
+      grid_dependency_wait();
+      if (blockIdx.x == 0 && blockIdx.z == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
+      for (int i = 0; i < pre; ++i) issue_a(smem + i * C::kStageBytes, &full_bar[i], a_tile0 + ks0 + i);
+      if (pre > 0) TRACE_POINT(2);
+      for (int i = pre; i < nks; ++i) {
+        const int s = i % C::kStages;
+        if (!mbar_wait(&empty_bar[s], ((i / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full_bar[s], (sharq ? C::kTxSharq : C::kTxNvfp4) - a_trim);
+        issue_b(st, &full_bar[s], b_tile0, ks0 + i);
+        issue_a(st, &full_bar[s], a_tile0 + ks0 + i);
       }
     }
   } else if (warp == 1) {
@@ -349,6 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     const int rl = sp * 32 + lane;
     const bool ok = mbar_wait(&acc_bar, 0, deadline, &abort_sh);
     tc_fence_after();
+    grid_dependency_wait();  // s_g is written by the preceding sharq_prep
     if (threadIdx.x == 64) TRACE_POINT(5);
     if (!ok) {
       record_error(args.err, kErrTimeout);
@@ -391,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
 
   if (threadIdx.x == 64) TRACE_POINT(6);
   if (kSplit && my_n > 0) {
+    grid_dependency_wait();
     // ------------------------ owner: sum the S received slices in rank order
     bool ok = !abort_sh;
     while (ok && !mbar_try_wait_cluster(&recv_bar, 0)) {
@@ -445,13 +463,15 @@ cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = kSplit ? a.splits : 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = kSplit ? a.splits : 1;
   cfg.attrs = attr;
-  cfg.numAttrs = kSplit ? 1 : 0;
+  cfg.numAttrs = kSplit ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<BN, kSplit>, a);
 }
 

@@ -119,6 +119,25 @@ __global__ void __launch_bounds__(kStatsThreads) prep_stats_kernel(
   }
 }
 
+// Allow the next kernel in the stream (the GEMM, launched as a programmatic
+// dependent) to start its set-up and weight loads now; it waits for this
+// grid's completion (griddepcontrol.wait) before reading our outputs.
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Last CTA out resets the device-wide max and the counters (sync words
+// 0..2 of the act scalar block), so the next sharq_prep on this buffer
+// starts from zero without a memset.  Called by thread 0 of every CTA after
+// the CTA has read the max.
+__device__ __forceinline__ void depart_and_reset(unsigned int* sync) {
+  __threadfence();
+  if (atomicAdd(sync + 2, 1u) == gridDim.x - 1) {
+    sync[0] = 0u;
+    sync[1] = 0u;
+    sync[2] = 0u;
+    __threadfence();
+  }
+}
+
 // pick a[sel] for sel in 0..3 without dynamic register indexing
 __device__ __forceinline__ float pick4(const float* a, int sel) {
   float r = a[0];
@@ -299,9 +318,16 @@ __global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
     const int* __restrict__ row_index, int T, int Tp, int K, const float* __restrict__ inv_rms,
     const unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
+  __shared__ float gmax_sh;
+  allow_dependents();
   const int runs = K >> 3;
   const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
-  const float gmax = __uint_as_float(*gmax_bits);
+  if (threadIdx.x == 0) {
+    gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
+    depart_and_reset(const_cast<unsigned int*>(gmax_bits));
+  }
+  __syncthreads();
+  const float gmax = gmax_sh;
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (gid == 0) *s_g_out = s;  // published even when there are no rows
   // whole warps exit together: rows span whole warps (K/8 is a multiple of 32)
@@ -332,6 +358,8 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   __shared__ double wsum[kFusedMaxThreads / 32];
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
+  allow_dependents();
+  if (blockIdx.x == 0 && threadIdx.x == 0) sync[3] = 0u;  // error word of the previous prep
   // threads per row, padded to whole warps (a warp never spans two rows);
   // the padding lanes hold zeros and store nothing
   const int used = (K >> 3) / NC;
@@ -395,6 +423,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     unsigned gb;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gb) : "l"(sync) : "memory");
     gmax_sh = __uint_as_float(gb);
+    depart_and_reset(sync);
   }
   __syncthreads();
   const float gmax = gmax_sh;
@@ -470,9 +499,9 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
                         int K, bool sharq_mode, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
                         cudaStream_t stream) {
-  // gmax, barrier arrivals, (unused), error word
-  cudaError_t e = cudaMemsetAsync(gmax_bits, 0, 4 * sizeof(unsigned int), stream);
-  if (e != cudaSuccess) return e;
+  // gmax_bits[0..3]: device-wide max, barrier arrivals, departures, error
+  // word; zero at rest (the kernels reset them), so no memset is needed
+  cudaError_t e = cudaSuccess;
   QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf};
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);

@@ -27,6 +27,7 @@ def _gpu_prep(x, gamma, eps, mode=sq.SHARQ_MODE_SHARQ, row_index=None, T=None):
     K = x.shape[1]
     act = sq.PreparedAct(T, K, mode)
     act.buf.fill_(0xAB)    # canary: every byte the layout defines must be written
+    act.reset()            # ... except the scalar block, zero before first use
     xd = H.bf16_dev(x)
     gd = H.bf16_dev(gamma) if gamma is not None else None
     ri = torch.from_numpy(row_index.astype(np.int32)).cuda() if row_index is not None else None
