@@ -26,6 +26,21 @@ namespace sharq {
 
 namespace {
 
+// Optional phase timeline (compile with -DSHARQ_TRACE): 4 global-timer
+// stamps per CTA of the single-launch kernel -- entry, max published,
+// barrier passed, exit.
+#ifdef SHARQ_TRACE
+__device__ unsigned long long* g_trace_prep = nullptr;
+#define PREP_TRACE(k)                                                                        \
+  do {                                                                                       \
+    if (g_trace_prep && threadIdx.x == 0) g_trace_prep[(size_t)blockIdx.x * 4 + (k)] = globaltimer_ns(); \
+  } while (0)
+#else
+#define PREP_TRACE(k) \
+  do {                \
+  } while (0)
+#endif
+
 __device__ __forceinline__ void bf16x8_to_float(const uint4& v, float* f) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -358,6 +373,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   __shared__ double wsum[kFusedMaxThreads / 32];
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
+  PREP_TRACE(0);
   allow_dependents();
   if (blockIdx.x == 0 && threadIdx.x == 0) sync[3] = 0u;  // error word of the previous prep
   // threads per row, padded to whole warps (a warp never spans two rows);
@@ -409,6 +425,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     atomicMax(sync, __float_as_uint(m));
     __threadfence();
     atomicAdd(sync + 1, 1u);
+    PREP_TRACE(1);
     // grid barrier: every CTA has published its max
     const uint64_t deadline = globaltimer_ns() + kBarrierLimitNs;
     unsigned seen = 0;
@@ -424,6 +441,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gb) : "l"(sync) : "memory");
     gmax_sh = __uint_as_float(gb);
     depart_and_reset(sync);
+    PREP_TRACE(2);
   }
   __syncthreads();
   const float gmax = gmax_sh;
@@ -431,6 +449,10 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
   // rows past Tp: whole warps (rows span whole warps), so they can skip
   if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
+#ifdef SHARQ_TRACE
+  __syncthreads();
+  PREP_TRACE(3);
+#endif
 }
 
 // runs of 8 per thread so that a row fits one CTA (<= 1024 threads)
@@ -494,6 +516,12 @@ cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, floa
 }
 
 }  // namespace
+
+#ifdef SHARQ_TRACE
+extern "C" int sharq_debug_set_trace_prep(void* p) {
+  return cudaMemcpyToSymbol(g_trace_prep, &p, sizeof(p)) == cudaSuccess ? 0 : -4;
+}
+#endif
 
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
                         int K, bool sharq_mode, float* inv_rms, float* s_g, unsigned int* gmax_bits,
