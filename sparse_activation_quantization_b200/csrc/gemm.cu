@@ -288,9 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         issue_b(st, &full_bar[i], b_tile0, ks0 + i);
       }
       grid_dependency_wait();
-      if (blockIdx.x == 0 && blockIdx.z == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
       for (int i = 0; i < pre; ++i) issue_a(smem + i * C::kStageBytes, &full_bar[i], a_tile0 + ks0 + i);
       if (pre > 0) TRACE_POINT(2);
+      if (blockIdx.x == 0 && blockIdx.z == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
       for (int i = pre; i < nks; ++i) {
         const int s = i % C::kStages;
         if (!mbar_wait(&empty_bar[s], ((i / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {

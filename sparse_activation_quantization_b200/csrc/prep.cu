@@ -7,7 +7,7 @@
 //
 // The per-tensor scale (PTS) is a device-wide max that every quantization
 // step needs before it can emit a code.  Two forms:
-//   single launch (prep_fused_kernel): a cooperative grid holds the whole
+//   single launch (prep_fused_kernel): a grid that fits the GPU holds the whole
 //     tensor in registers -- load, RMSNorm, device-wide max through a bounded
 //     grid barrier, then quantize; X is read once.  Used whenever the grid
 //     fits on the GPU at once.
@@ -393,6 +393,13 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   int src = -1;
   if (live && t < T && has) src = row_index ? row_index[t] : t;
   load_runs<NC>(x, X, src, K, c0);
+  // gamma in flight together with X (not after the row reduction)
+  uint4 graw[NC];
+  if (gamma && src >= 0) {
+    const uint4* gr = reinterpret_cast<const uint4*>(gamma) + c0;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) graw[c] = gr[c];
+  }
 
   if (gamma) {
     double ss = 0.0;
@@ -406,7 +413,15 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     for (int w = 0; w < wpr; ++w) tot += wsum[rl * wpr + w];  // fixed order
     const float inv = (float)(1.0 / sqrt(tot / (double)K + (double)eps));
     if (live && t < T && li == 0) inv_rms[t] = inv;
-    if (src >= 0) normalise_runs<NC>(x, gamma, c0, inv);
+    if (src >= 0) {
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        float g[8];
+        bf16x8_to_float(graw[c], g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[8 * c + e] = norm_one(x[8 * c + e], inv, g[e]);
+      }
+    }
   } else if (live && t < T && li == 0) {
     inv_rms[t] = 1.0f;
   }
@@ -494,10 +509,18 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   const int threads = rpc * tpr;
   const int ctas = (Tp + rpc - 1) / rpc;
   if (ctas > fused_max_ctas_t<NC, kSharq>(threads)) return cudaSuccess;
-  void* args[] = {(void*)&Xb, (void*)&Gb, (void*)&eps, (void*)&row_index, (void*)&T, (void*)&Tp, (void*)&K,
-                  (void*)&rpc, (void*)&inv_rms, (void*)&sync, (void*)&s_g, (void*)&p};
-  cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(prep_fused_kernel<NC, kSharq>),
-                                              dim3(ctas), dim3(threads), args, 0, stream);
+  // A plain launch: the grid fits the GPU at once (checked above), so all
+  // CTAs are resident together when the stream reaches this kernel; the
+  // GEMM that follows as a programmatic dependent can start only after every
+  // CTA of this grid has started (each triggers at entry), so it cannot
+  // crowd out a CTA that has not arrived at the grid barrier.  The barrier's
+  // spin is bounded all the same.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = stream;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kSharq>, Xb, Gb, eps, row_index, T, Tp, K, rpc,
+                                     inv_rms, sync, s_g, p);
   if (e == cudaSuccess) *launched = true;
   else cudaGetLastError();  // fall back to the two-launch form
   return cudaSuccess;
