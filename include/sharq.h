@@ -98,8 +98,9 @@ typedef struct {
 
 /*
  * Prepared activation (output of sharq_prep, operand A of sharq_linear).
- * Rows are padded to Tp = ceil(T/128)*128; padded rows hold zero codes, zero
- * scales and metadata 0x4 (pairs 0 and 1) so they contribute nothing.
+ * The tiles cover Tp = ceil(T/128)*128 rows; rows T..Tp-1 are not written by
+ * sharq_prep and never read as operands by sharq_linear (their contents are
+ * unspecified).
  * Tile index i = (t/128) * K/256 + k/256, r = t % 128, c = k % 256:
  *   r_codes: 16384-byte tiles, 128-byte lines, 128-byte swizzle (as weight
  *            codes).  SHARQ: residual codes.  NVFP4: codes of Xn.

@@ -31,8 +31,10 @@
 // mbarrier), and the owner sums the S slices in rank order -- deterministic,
 // no global scratch, no atomics, one bounded wait.
 // Rows beyond the activation's valid rows are not copied into shared memory
-// (decode: T = 1 moves 1 row of codes, not 128); their accumulator rows hold
-// garbage that is never stored -- MMA rows are independent.
+// (decode: T = 1 moves 1 row of codes, not 128) -- sharq_prep does not even
+// write them; their accumulator rows hold garbage that is never stored (MMA
+// rows are independent), and their metadata is set to a valid pattern in
+// shared memory once at start-up.
 // Every wait is bounded by the global timer; on timeout the CTA records
 // SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
 #include "sharq_device.cuh"
@@ -237,6 +239,16 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     tmem_alloc(&tmem_base_sh, C::kTmemCols);
     tmem_relinquish();
   }
+  if (args.sharq_mode && valid < 128) {
+    // Rows past the activation's end are never copied in; give their
+    // metadata a valid pattern (pairs 0 and 1) once, in every stage.
+    for (int idx = threadIdx.x; idx < C::kStages * (128 - valid); idx += kThreads) {
+      const int st = idx / (128 - valid), row = valid + idx % (128 - valid);
+      *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE + row * 16) =
+          make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+    }
+    fence_proxy_async_smem();  // visible to tcgen05.cp (async proxy)
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -259,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
       // copy only the valid rows of the activation code tiles
       const uint32_t a_rows = (uint32_t)valid;
-      const uint32_t a_trim = (128u - a_rows) * (sharq ? 192u : 128u);
+      const uint32_t a_trim = (128u - a_rows) * (sharq ? 208u : 128u);
       auto issue_b = [&](uint8_t* st, uint64_t* fb, size_t b_tile, int ks) {
 #pragma unroll
         for (int h = 0; h < C::kHalves; ++h) {
@@ -274,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
         if (sharq) {
           bulk_g2s(st + C::kOffASP, args.a_sp + at * kSpTile, a_rows * 64u, fb);
-          bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, kMetaTile, fb);
+          bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, a_rows * 16u, fb);
           bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
         }
       };

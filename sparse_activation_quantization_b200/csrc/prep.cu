@@ -141,10 +141,9 @@ __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontro
 
 // Last CTA out resets the device-wide max and the counters (sync words
 // 0..2 of the act scalar block), so the next sharq_prep on this buffer
-// starts from zero without a memset.  Called by thread 0 of every CTA after
-// the CTA has read the max.
+// starts from zero without a memset.  Called by thread 0 of every CTA at its
+// end, after the CTA has read the max (so the reset cannot race a reader).
 __device__ __forceinline__ void depart_and_reset(unsigned int* sync) {
-  __threadfence();
   if (atomicAdd(sync + 2, 1u) == gridDim.x - 1) {
     sync[0] = 0u;
     sync[1] = 0u;
@@ -337,24 +336,22 @@ __global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
   allow_dependents();
   const int runs = K >> 3;
   const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
-  if (threadIdx.x == 0) {
-    gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
-    depart_and_reset(const_cast<unsigned int*>(gmax_bits));
-  }
+  if (threadIdx.x == 0) gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
   __syncthreads();
   const float gmax = gmax_sh;
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (gid == 0) *s_g_out = s;  // published even when there are no rows
-  // whole warps exit together: rows span whole warps (K/8 is a multiple of 32)
-  if (gid >= (long long)Tp * runs) return;
-  const int t = (int)(gid / runs);
-  const int c0 = (int)(gid - (long long)t * runs);
-  int src = -1;
-  if (t < T) src = row_index ? row_index[t] : t;
-  float x[8];
-  load_runs<1>(x, X, src, K, c0);
-  if (gamma && src >= 0) normalise_runs<1>(x, gamma, c0, inv_rms[t]);
-  quant_runs<1, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
+  // whole warps go together: rows span whole warps (K/8 is a multiple of 32)
+  if (gid < (long long)T * runs) {
+    const int t = (int)(gid / runs);
+    const int c0 = (int)(gid - (long long)t * runs);
+    const int src = row_index ? row_index[t] : t;
+    float x[8];
+    load_runs<1>(x, X, src, K, c0);
+    if (gamma && src >= 0) normalise_runs<1>(x, gamma, c0, inv_rms[t]);
+    quant_runs<1, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
+  }
+  if (threadIdx.x == 0) depart_and_reset(const_cast<unsigned int*>(gmax_bits));
 }
 
 // ---------------------------------------------------------------------------
@@ -385,13 +382,13 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   const bool has = li < used;
   const int c0 = (has ? li : 0) * NC;
   const int t = blockIdx.x * rows_per_cta + rl;
-  const bool live = t < Tp;
+  const bool live = t < T;  // rows T..Tp-1 (tile padding) are not written
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpr = tpr >> 5;                 // warps per row
 
   float x[8 * NC];
   int src = -1;
-  if (live && t < T && has) src = row_index ? row_index[t] : t;
+  if (live && has) src = row_index ? row_index[t] : t;
   load_runs<NC>(x, X, src, K, c0);
   // gamma in flight together with X (not after the row reduction)
   uint4 graw[NC];
@@ -412,7 +409,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     double tot = 0.0;
     for (int w = 0; w < wpr; ++w) tot += wsum[rl * wpr + w];  // fixed order
     const float inv = (float)(1.0 / sqrt(tot / (double)K + (double)eps));
-    if (live && t < T && li == 0) inv_rms[t] = inv;
+    if (live && li == 0) inv_rms[t] = inv;
     if (src >= 0) {
 #pragma unroll
       for (int c = 0; c < NC; ++c) {
@@ -422,7 +419,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
         for (int e = 0; e < 8; ++e) x[8 * c + e] = norm_one(x[8 * c + e], inv, g[e]);
       }
     }
-  } else if (live && t < T && li == 0) {
+  } else if (live && li == 0) {
     inv_rms[t] = 1.0f;
   }
 
@@ -437,33 +434,36 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   if (threadIdx.x == 0) {
     float m = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
-    atomicMax(sync, __float_as_uint(m));
-    __threadfence();
-    atomicAdd(sync + 1, 1u);
-    PREP_TRACE(1);
-    // grid barrier: every CTA has published its max
-    const uint64_t deadline = globaltimer_ns() + kBarrierLimitNs;
-    unsigned seen = 0;
-    do {
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(sync + 1) : "memory");
-      if (seen >= gridDim.x) break;
-      if (globaltimer_ns() > deadline) {
-        atomicCAS(reinterpret_cast<int*>(sync + 3), 0, -5);  // SHARQ_ERR_TIMEOUT
-        break;
-      }
-    } while (true);
-    unsigned gb;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gb) : "l"(sync) : "memory");
-    gmax_sh = __uint_as_float(gb);
-    depart_and_reset(sync);
+    if (gridDim.x == 1) {
+      gmax_sh = m;  // one CTA holds the whole tensor: no grid barrier
+    } else {
+      atomicMax(sync, __float_as_uint(m));
+      // arrival with release semantics: our max is visible before the count
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(sync + 1) : "memory");
+      PREP_TRACE(1);
+      // grid barrier: every CTA has published its max (bounded spin)
+      const uint64_t deadline = globaltimer_ns() + kBarrierLimitNs;
+      unsigned seen = 0;
+      do {
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(sync + 1) : "memory");
+        if (seen >= gridDim.x) break;
+        if (globaltimer_ns() > deadline) {
+          atomicCAS(reinterpret_cast<int*>(sync + 3), 0, -5);  // SHARQ_ERR_TIMEOUT
+          break;
+        }
+      } while (true);
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+      gmax_sh = __uint_as_float(*(volatile unsigned int*)sync);
+    }
     PREP_TRACE(2);
   }
   __syncthreads();
   const float gmax = gmax_sh;
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
-  // rows past Tp: whole warps (rows span whole warps), so they can skip
+  // rows past T: whole warps (rows span whole warps), so they can skip
   if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
+  if (threadIdx.x == 0 && gridDim.x > 1) depart_and_reset(sync);
 #ifdef SHARQ_TRACE
   __syncthreads();
   PREP_TRACE(3);
@@ -479,6 +479,15 @@ int fused_runs_per_thread(int K) {
   return 0;
 }
 
+// Prep CTAs use almost no shared memory; ask for the maximum shared-memory
+// carveout anyway so that an SM running them keeps room for a GEMM CTA
+// (~215 KB) launched early as their programmatic dependent.
+template <class F>
+void prefer_max_shared(F* fn) {
+  cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  cudaGetLastError();
+}
+
 template <int NC, bool kSharq>
 int fused_max_ctas_t(int threads) {
   static int cache[kFusedMaxThreads + 1][64] = {};
@@ -486,6 +495,7 @@ int fused_max_ctas_t(int threads) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
   int& c = cache[threads][dev];
   if (c == 0) {
+    prefer_max_shared(prep_fused_kernel<NC, kSharq>);
     int per_sm = 0, sms = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<NC, kSharq>, threads, 0) !=
             cudaSuccess ||
@@ -507,7 +517,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   int rpc = 512 / tpr;
   rpc = rpc < 1 ? 1 : rpc;
   const int threads = rpc * tpr;
-  const int ctas = (Tp + rpc - 1) / rpc;
+  const int ctas = (T + rpc - 1) / rpc;
   if (ctas > fused_max_ctas_t<NC, kSharq>(threads)) return cudaSuccess;
   // A plain launch: the grid fits the GPU at once (checked above), so all
   // CTAs are resident together when the stream reaches this kernel; the
@@ -557,7 +567,7 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
 
-  if (Tp > 0) {
+  if (T > 0) {
     bool launched = false;
     e = sharq_mode ? try_fused_any<true>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
                                          &launched)
@@ -567,10 +577,17 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
     if (launched) return cudaSuccess;
   }
 
+  static bool carveout_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !carveout_set[dev]) {
+    prefer_max_shared(prep_quant_kernel<true>);
+    prefer_max_shared(prep_quant_kernel<false>);
+    carveout_set[dev] = true;
+  }
   if (T > 0) {
     prep_stats_kernel<<<T, kStatsThreads, 0, stream>>>(Xb, Gb, eps, row_index, K, inv_rms, gmax_bits);
   }
-  const long long n = (long long)Tp * (K >> 3);
+  const long long n = (long long)T * (K >> 3);
   // at least one block so that s_g is published (= 1) even for T == 0
   const unsigned grid = n > 0 ? (unsigned)((n + kQuantThreads - 1) / kQuantThreads) : 1u;
   if (sharq_mode)

@@ -26,20 +26,26 @@ def bf16_dev(x_f32):
 
 
 def act_from_logical(T, K, mode, r_codes, r_sf, sp_codes=None, meta=None, sp_sf=None, s_g=1.0):
-    """PreparedAct whose buffers hold hand-built logical operands."""
+    """PreparedAct whose buffers hold hand-built logical operands.  The tile
+    padding rows past T hold random bytes (invalid metadata, NaN-coded scales
+    included): sharq_linear must not depend on them."""
     act = sq.PreparedAct(T, K, mode)
     Tp = act.view.Tp
+    g = np.random.default_rng(99)
+    junk = lambda a: np.concatenate([a, g.integers(0, 256 if a.dtype == np.uint8 else 16,
+                                                   (Tp - T, *a.shape[1:])).astype(a.dtype)])
     act.buf.zero_()
-    rc = _layout.tile_codes(_layout.pad_rows(r_codes, Tp))
+    nib = lambda a: np.concatenate([a, g.integers(0, 16, (Tp - T, *a.shape[1:])).astype(np.uint8)])
+    rc = _layout.tile_codes(nib(r_codes))
     act.region("r_codes", rc.size).copy_(to_dev(rc))
-    rs = _layout.tile_sf(_layout.pad_rows(r_sf, Tp), 16)
+    rs = _layout.tile_sf(junk(r_sf), 16)
     act.region("r_sf", rs.size).copy_(to_dev(rs))
     if mode == sq.SHARQ_MODE_SHARQ:
-        sc = _layout.tile_sp_codes(_layout.pad_rows(sp_codes, Tp))
+        sc = _layout.tile_sp_codes(nib(sp_codes))
         act.region("sp_codes", sc.size).copy_(to_dev(sc))
-        mt = _layout.tile_meta(_layout.pad_rows(meta, Tp, fill=0x4))
+        mt = _layout.tile_meta(nib(meta))
         act.region("meta", mt.size).copy_(to_dev(mt))
-        ss = _layout.tile_sf(_layout.pad_rows(sp_sf, Tp), 32)
+        ss = _layout.tile_sf(junk(sp_sf), 32)
         act.region("sp_sf", ss.size).copy_(to_dev(ss))
     act.region("s_g", 4).view(torch.float32).fill_(float(s_g))
     return act

@@ -1,8 +1,8 @@
 """sharq_prep and sharq_pack_weight vs the oracle, bit for bit (GPU).
 
 Masks, metadata nibbles, E2M1 codes, E4M3 scale bytes and the FP32 global
-scales must be identical; padded rows must hold zero codes, zero scales and
-the pairs-(0,1) nibble.
+scales must be identical on every row T of the tensor (the tile padding rows
+past T are not part of the output).
 """
 import numpy as np
 import pytest
@@ -71,10 +71,6 @@ def _check_sharq(x, gamma, eps, row_index=None, T=None):
     _assert_equal("sp_sf", g["sp_sf"][:T], p["sp_sf"])
     _assert_equal("r_codes", g["r_codes"][:T], p["r_codes"])
     _assert_equal("r_sf", g["r_sf"][:T], p["r_sf"])
-    # padded rows
-    assert np.all(g["meta"][T:] == 0x4)
-    for k in ("sp_codes", "sp_sf", "r_codes", "r_sf"):
-        assert np.all(g[k][T:] == 0), k
     return act, p
 
 
