@@ -182,6 +182,32 @@ int sharq_prep(const void *d_X, const void *d_gamma, float eps, const int *d_row
                const sharq_act *a, sharq_stream_t stream);
 
 /*
+ * sharq_prep_noalloc - sharq_prep for callers that cannot allocate device
+ * memory at run time: code inside a region being captured into a CUDA graph
+ * (where cudaMalloc is not allowed), or a host framework whose memory
+ * planner owns all device memory and hands out only the tensors it planned.
+ * The paper has no counterpart; this is a deployment variant of the same
+ * computation, with results identical to sharq_prep's.
+ * Differences from sharq_prep:
+ *  - The prep's working memory (device-wide max, grid-barrier counters,
+ *    error word, per-row 1/rms) lives in a fixed array inside the library
+ *    (256 bytes + 4 bytes per row, up to 16384 rows, about 64 KB, held by
+ *    every GPU that loads the library until the process exits).  a->inv_rms
+ *    is not written and a->gmax_bits[0..2] are not used; a->gmax_bits may be
+ *    NULL.  If it is not, the error word is copied to a->gmax_bits[3], where
+ *    sharq_linear looks for it.
+ *  - a->T > 16384 returns SHARQ_ERR_UNSUPPORTED_SHAPE.
+ *  - The first call on each device looks the array's address up
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Each call clears the array's counters with a 16-byte cudaMemsetAsync
+ *    (no allocation).  All calls share the array: calls whose work overlaps
+ *    on the GPU (different streams without ordering) race on it.
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ */
+int sharq_prep_noalloc(const void *d_X, const void *d_gamma, float eps, const int *d_row_index,
+                       const sharq_act *a, sharq_stream_t stream);
+
+/*
  * sharq_linear - dual-path FP4 GEMM (xllm-io review, sections 3.4-3.5).
  * A 4:8 sparse block-scaled FP4 MMA on the backbone and a dense block-scaled
  * FP4 MMA on the residual accumulate into one TMEM accumulator per output

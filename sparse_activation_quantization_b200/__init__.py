@@ -19,7 +19,7 @@ __all__ = [
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes",
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
-    "sharq_status_string", "sharq_abi_version",
+    "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
     "PackedWeight", "PreparedAct", "Workspace", "linear", "EXPORTED_SYMBOLS",
 ]
 
@@ -31,7 +31,7 @@ SHARQ_OUT_F32 = 1
 EXPORTED_SYMBOLS = (
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes", "sharq_weight_view",
     "sharq_act_view", "sharq_pack_weight", "sharq_prep", "sharq_linear", "sharq_linear_grouped",
-    "sharq_check_status", "sharq_status_string", "sharq_abi_version",
+    "sharq_check_status", "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -76,6 +76,7 @@ def lib():
             "sharq_act_view": (i, [vp, i, i, i, A]),
             "sharq_pack_weight": (i, [vp, W, vp]),
             "sharq_prep": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
+            "sharq_prep_noalloc": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
             "sharq_linear": (i, [A, W, vp, i, vp, sz, vp]),
             "sharq_linear_grouped": (i, [A, vp, W, vp, i, vp, sz, vp]),
             "sharq_check_status": (i, [vp, vp]),
@@ -135,6 +136,11 @@ def sharq_pack_weight(d_W, w, stream):
 
 def sharq_prep(d_X, d_gamma, eps, d_row_index, a, stream):
     return _check(lib().sharq_prep(d_X, d_gamma, eps, d_row_index, ctypes.byref(a), stream), "sharq_prep")
+
+
+def sharq_prep_noalloc(d_X, d_gamma, eps, d_row_index, a, stream):
+    return _check(lib().sharq_prep_noalloc(d_X, d_gamma, eps, d_row_index, ctypes.byref(a), stream),
+                  "sharq_prep_noalloc")
 
 
 def sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream):

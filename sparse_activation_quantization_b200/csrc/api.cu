@@ -20,6 +20,11 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
                           int* err, const int* act_err, cudaStream_t stream);
+int noalloc_max_rows();
+cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
+                                int K, bool sharq_mode, float* s_g, uint8_t* sp_codes, uint8_t* meta,
+                                uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, unsigned int* err_out,
+                                cudaStream_t stream);
 }  // namespace sharq
 
 namespace {
@@ -268,6 +273,31 @@ int sharq_prep(const void* d_X, const void* d_gamma, float eps, const int* d_row
       d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ, a->inv_rms, a->s_g,
       a->gmax_bits, static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta),
       static_cast<uint8_t*>(a->sp_sf), static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf),
+      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
+}
+
+int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const int* d_row_index,
+                       const sharq_act* a, sharq_stream_t stream) {
+  if (!a) return SHARQ_ERR_INVALID_ARG;
+  if (!shape_ok_t(a->T) || !shape_ok_k(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (a->T > sharq::noalloc_max_rows()) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (a->mode != SHARQ_MODE_SHARQ && a->mode != SHARQ_MODE_NVFP4) return SHARQ_ERR_INVALID_ARG;
+  if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
+  if (!a->r_codes || !a->r_sf || !a->s_g) return SHARQ_ERR_INVALID_ARG;
+  if (a->mode == SHARQ_MODE_SHARQ && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf};
+  for (const void* q : p)
+    if (q && !aligned(q, 16)) return SHARQ_ERR_INVALID_ARG;
+  if (a->T > 0 && (!d_X || !aligned(d_X, 16))) return SHARQ_ERR_INVALID_ARG;
+  if (d_gamma && !aligned(d_gamma, 16)) return SHARQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return SHARQ_ERR_INVALID_ARG;
+  int st = check_device();
+  if (st) return st;
+  cudaError_t e = sharq::launch_prep_noalloc(
+      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ, a->s_g,
+      static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta), static_cast<uint8_t*>(a->sp_sf),
+      static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf), a->gmax_bits ? a->gmax_bits + 3 : nullptr,
       reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }

@@ -599,4 +599,56 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free form (the sharq_prep_noalloc entry point).  The prep's
+// working memory -- the device-wide max, the grid-barrier and departure
+// counters, the error word, and the per-row 1/rms -- lives in this
+// file-scope device array instead of the caller's buffer.  Every GPU that
+// loads the library keeps the array until the process exits, and all calls
+// share it: calls whose kernels overlap on the GPU race on it.
+constexpr int kNoAllocMaxRows = 16384;
+constexpr size_t kNoAllocSyncBytes = 256;
+static __device__ __align__(256) unsigned char g_prep_scratch[kNoAllocSyncBytes + 4 * kNoAllocMaxRows];
+
+int noalloc_max_rows() { return kNoAllocMaxRows; }
+
+// Device address of g_prep_scratch for the current device, looked up on the
+// first call on that device (host code cannot use the symbol itself).
+static cudaError_t noalloc_scratch(unsigned char** out) {
+  static unsigned char* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_prep_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
+                                int K, bool sharq_mode, float* s_g, uint8_t* sp_codes, uint8_t* meta,
+                                uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, unsigned int* err_out,
+                                cudaStream_t stream) {
+  if (T > kNoAllocMaxRows) return cudaErrorInvalidValue;
+  unsigned char* scr = nullptr;
+  cudaError_t e = noalloc_scratch(&scr);
+  if (e != cudaSuccess) return e;
+  unsigned int* sync = reinterpret_cast<unsigned int*>(scr);
+  float* inv = reinterpret_cast<float*>(scr + kNoAllocSyncBytes);
+  // the array keeps the last call's contents: start every call from zero
+  e = cudaMemsetAsync(sync, 0, 4 * sizeof(unsigned int), stream);
+  if (e != cudaSuccess) return e;
+  e = launch_prep(X, gamma, eps, row_index, T, Tp, K, sharq_mode, inv, s_g, sync, sp_codes, meta, sp_sf, r_codes,
+                  r_sf, stream);
+  if (e != cudaSuccess) return e;
+  // forward the error word to where sharq_linear looks for it
+  if (err_out) e = cudaMemcpyAsync(err_out, sync + 3, sizeof(unsigned int), cudaMemcpyDeviceToDevice, stream);
+  return e;
+}
+
 }  // namespace sharq
