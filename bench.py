@@ -32,6 +32,9 @@ T_LIST = (1, 16, 128)
 N_ROT = 16
 EPS = 1e-5
 WORKLOAD = "llama3.1-8b q_proj K=4096 D=4096, T in {1,16,128}, RMSNorm gamma~U(0.5,1.5)"
+WORKLOADS = {"q_proj": "llama3.1-8b q_proj K=4096 D=4096 (prep+linear per T), RMSNorm gamma~U(0.5,1.5)",
+             "mlp": "llama3.1-8b MLP prefill: gate/up 4096->14336 (shared prep, RMSNorm), down 14336->4096 "
+                    "(Student-t input)"}
 METRIC = "prep+dual-GEMM effective TFLOP/s (2TKD)"
 
 
@@ -189,6 +192,53 @@ def run_reference(args, world, rank, budget_s=120.0):
 
 # ------------------------------------------------------------- GPU path -----
 
+class Layer:
+    """One linear of a workload: (T, K, D), RMSNorm or not, input model."""
+
+    def __init__(self, name, T, K, D, norm, base="normal", shares_prep_with=None):
+        self.name, self.T, self.K, self.D, self.norm, self.base = name, T, K, D, norm, base
+        self.shares = shares_prep_with
+
+    @property
+    def flops(self):
+        return 2.0 * self.T * self.K * self.D
+
+
+def workload_layers(name, t_list):
+    if name == "q_proj":
+        return [Layer(f"q_proj_T{t}", t, K_DIM, D_DIM, True) for t in t_list]
+    if name == "mlp":   # Llama-3.1-8B MLP at prefill: gate/up share one prep, then down
+        out = []
+        for t in t_list:
+            out += [Layer(f"gate_T{t}", t, 4096, 14336, True),
+                    Layer(f"up_T{t}", t, 4096, 14336, True, shares_prep_with=f"gate_T{t}"),
+                    Layer(f"down_T{t}", t, 14336, 4096, False, base="student_t")]
+        return out
+    raise ValueError(name)
+
+
+def kernel_us(fn, n_rot, stream, launches=96):
+    """Average duration of one launch of fn(i): a graph of `launches`
+    back-to-back launches (rotating inputs), replayed, CUDA events."""
+    import torch
+    reps = max(1, launches // n_rot)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(reps):
+            for i in range(n_rot):
+                fn(i)
+    for _ in range(2):
+        g.replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(5):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) * 1e3 / (5 * reps * n_rot)
+
+
 def run_gpu(args, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -205,32 +255,49 @@ def run_gpu(args, world, rank, local):
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
-    # --- inputs resident in HBM: N_ROT weight copies, N_ROT activation sets ---
-    gamma = torch.from_numpy(synthetic.gamma(12, K_DIM)).to(torch.bfloat16).to(dev)
-    weights = []
-    for i in range(N_ROT):
-        W = torch.from_numpy(synthetic.weights(100 + i, K_DIM, D_DIM)).to(torch.bfloat16).to(dev)
-        weights.append(sq.PackedWeight(W, stream=stream))
-        del W
-    xs = {t: [torch.from_numpy(synthetic.activations(1000 * t + i, t, K_DIM)).to(torch.bfloat16).to(dev)
-              for i in range(N_ROT)] for t in T_LIST}
-    acts = {t: sq.PreparedAct(t, K_DIM, device=dev) for t in T_LIST}
-    outs = {t: torch.empty((t, D_DIM), dtype=torch.bfloat16, device=dev) for t in T_LIST}
-    wss = {t: sq.Workspace(t, K_DIM, D_DIM, device=dev) for t in T_LIST}
+    layers = workload_layers(args.workload, args.T)
+    # inputs resident in HBM; decode shapes rotate through copies so that the
+    # working set of consecutive steps exceeds the 126 MB L2
+    wbytes = sum(sq.sharq_weight_bytes(L.K, L.D) for L in layers)
+    n_rot = max(1, min(16, -(-200_000_000 // max(wbytes, 1))))
+    weights = {L.name: [] for L in layers}
+    for li, L in enumerate(layers):
+        for i in range(n_rot):
+            W = torch.from_numpy(synthetic.weights(100 + 31 * li + i, L.K, L.D)).to(torch.bfloat16).to(dev)
+            weights[L.name].append(sq.PackedWeight(W, stream=stream))
+            del W
+    gammas, xs, acts, outs, wss = {}, {}, {}, {}, {}
+    for L in layers:
+        outs[L.name] = torch.empty((L.T, L.D), dtype=torch.bfloat16, device=dev)
+        wss[L.name] = sq.Workspace(L.T, L.K, L.D, device=dev)
+        if L.shares:
+            continue
+        gammas[L.name] = (torch.from_numpy(synthetic.gamma(12, L.K)).to(torch.bfloat16).to(dev)
+                          if L.norm else None)
+        xs[L.name] = [torch.from_numpy(synthetic.activations(1000 * L.T + i, L.T, L.K, base=L.base))
+                      .to(torch.bfloat16).to(dev) for i in range(n_rot)]
+        acts[L.name] = sq.PreparedAct(L.T, L.K, device=dev)
     torch.cuda.synchronize()
 
-    def step(i):
-        for t in T_LIST:
-            acts[t].prep(xs[t][i], gamma, EPS, stream=stream)
-            sq.linear(acts[t], weights[i], out=outs[t], ws=wss[t], stream=stream)
+    def prep(L, i):
+        acts[L.name].prep(xs[L.name][i], gammas[L.name], EPS, stream=stream)
 
-    launches_per_step = 2 * len(T_LIST)   # single-launch prep + gemm per layer
-    # warm up eagerly, then capture one graph per rotation slot
-    for i in range(N_ROT):
+    def gemm(L, i):
+        src = L.shares or L.name
+        sq.linear(acts[src], weights[L.name][i], out=outs[L.name], ws=wss[L.name], stream=stream)
+
+    def step(i):
+        for L in layers:
+            if not L.shares:
+                prep(L, i)
+            gemm(L, i)
+
+    launches_per_step = sum(1 if L.shares else 2 for L in layers)   # single-launch prep + gemm
+    for i in range(n_rot):
         step(i)
     torch.cuda.synchronize()
     graphs = []
-    for i in range(N_ROT):
+    for i in range(n_rot):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step(i)
@@ -238,7 +305,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
 
     for k in range(args.warmup):
-        graphs[k % N_ROT].replay()
+        graphs[k % n_rot].replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -247,105 +314,101 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     ev0.record(stream)
     for k in range(args.steps):
-        graphs[k % N_ROT].replay()
+        graphs[k % n_rot].replay()
     ev1.record(stream)
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+        t_ = torch.tensor([ms], device=dev)
+        dist.all_reduce(t_, op=dist.ReduceOp.MAX)
+        ms = t_.item()
         dist.barrier()
-    for t in T_LIST:
-        assert wss[t].check(stream) == 0, "device-side error"
+    for L in layers:
+        assert wss[L.name].check(stream) == 0, "device-side error"
 
-    # --- per-layer µs per T, and the dominant kernel's duration -------------
-    def time_graph(fn, reps):
-        gs = []
-        for i in range(N_ROT):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                fn(i)
-            gs.append(g)
-        for i in range(3):
-            gs[i % N_ROT].replay()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        a.record(stream)
-        for r in range(reps):
-            gs[r % N_ROT].replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / reps * 1e3  # µs
-
-    per_t = {}
-    for t in T_LIST:
-        layer = time_graph(lambda i, t=t: (acts[t].prep(xs[t][i], gamma, EPS, stream=stream),
-                                           sq.linear(acts[t], weights[i], out=outs[t], ws=wss[t], stream=stream)),
-                           200)
-        gemm = time_graph(lambda i, t=t: sq.linear(acts[t], weights[i], out=outs[t], ws=wss[t], stream=stream), 200)
-        prep = time_graph(lambda i, t=t: acts[t].prep(xs[t][i], gamma, EPS, stream=stream), 200)
-        per_t[t] = {"layer_us": layer, "gemm_us": gemm, "prep_us": prep,
-                    "tflops": 2.0 * t * K_DIM * D_DIM / (layer * 1e-6) / 1e12,
-                    "gemm_gbs": gemm_alg_bytes(t, K_DIM, D_DIM) / (gemm * 1e-6) / 1e9,
-                    "prep_gbs": prep_alg_bytes(t, K_DIM) / (prep * 1e-6) / 1e9}
+    # --- per-layer and per-kernel times -------------------------------------
+    per = {}
+    for L in layers:
+        g_us = kernel_us(lambda i, L=L: gemm(L, i), n_rot, stream)
+        p_us = None if L.shares else kernel_us(lambda i, L=L: prep(L, i), n_rot, stream)
+        lay = kernel_us(lambda i, L=L: (None if L.shares else prep(L, i), gemm(L, i)), n_rot, stream)
+        per[L.name] = {"T": L.T, "K": L.K, "D": L.D, "layer_us": lay, "gemm_us": g_us, "prep_us": p_us,
+                       "layer_tflops": L.flops / (lay * 1e-6) / 1e12,
+                       "gemm_tflops": L.flops / (g_us * 1e-6) / 1e12,
+                       "gemm_gbs": gemm_alg_bytes(L.T, L.K, L.D) / (g_us * 1e-6) / 1e9,
+                       "prep_gbs": None if p_us is None else prep_alg_bytes(L.T, L.K) / (p_us * 1e-6) / 1e9}
 
     # --- end-to-end through the public API with host buffers ----------------
-    hx = {t: torch.from_numpy(synthetic.activations(7 + t, t, K_DIM)).to(torch.bfloat16).pin_memory()
-          for t in T_LIST}
-    hy = {t: torch.empty((t, D_DIM), dtype=torch.bfloat16).pin_memory() for t in T_LIST}
-    dx = {t: torch.empty((t, K_DIM), dtype=torch.bfloat16, device=dev) for t in T_LIST}
-    h2d = sum(hx[t].numel() * 2 for t in T_LIST)
-    d2h = sum(hy[t].numel() * 2 for t in T_LIST)
+    hx = {n: torch.from_numpy(synthetic.activations(7, xs[n][0].shape[0], xs[n][0].shape[1])).to(torch.bfloat16)
+          .pin_memory() for n in xs}
+    hy = {L.name: torch.empty((L.T, L.D), dtype=torch.bfloat16).pin_memory() for L in layers}
+    dx = {n: torch.empty_like(xs[n][0]) for n in xs}
+    h2d = sum(hx[n].numel() * 2 for n in hx)
+    d2h = sum(hy[n].numel() * 2 for n in hy)
 
     def e2e_step(i):
-        for t in T_LIST:
-            dx[t].copy_(hx[t], non_blocking=True)
-            acts[t].prep(dx[t], gamma, EPS, stream=stream)
-            sq.linear(acts[t], weights[i], out=outs[t], ws=wss[t], stream=stream)
-            hy[t].copy_(outs[t], non_blocking=True)
+        for L in layers:
+            if not L.shares:
+                dx[L.name].copy_(hx[L.name], non_blocking=True)
+                acts[L.name].prep(dx[L.name], gammas[L.name], EPS, stream=stream)
+            gemm(L, i)
+            hy[L.name].copy_(outs[L.name], non_blocking=True)
     for i in range(3):
-        e2e_step(i)
+        e2e_step(i % n_rot)
     torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 200))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for k in range(args.steps):
-        e2e_step(k % N_ROT)
+    for k in range(e2e_steps):
+        e2e_step(k % n_rot)
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / args.steps
+    e2e_ms = a.elapsed_time(b) / e2e_steps
     if world > 1:
         t_ = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t_, op=dist.ReduceOp.MAX)
         e2e_ms = t_.item()
 
-    peak, peak_kind = read_peaks()
-    dom = max(T_LIST, key=lambda t: per_t[t]["gemm_us"])
-    achieved = per_t[dom]["gemm_gbs"]
+    flops_step = sum(L.flops for L in layers)
+    # dominant kernel: the GEMM with the largest share of the step
+    dom = max(layers, key=lambda L: per[L.name]["gemm_us"])
+    if args.workload == "mlp":
+        from sparse_activation_quantization_b200 import peak
+        pk = peak.fp4_peaks()
+        roof = {"kernel": f"sharq_gemm_kernel ({dom.name})", "bound": "tensor",
+                "achieved": per[dom.name]["gemm_tflops"], "peak": pk["effective_pflops"] * 1e3,
+                "unit": "TFLOP/s", "frac": per[dom.name]["gemm_tflops"] / (pk["effective_pflops"] * 1e3),
+                "peak_kind": "measured tcgen05 FP4 (dense %.2f, sparse %.2f PFLOP/s; dual-GEMM effective)"
+                             % (pk["dense_pflops"], pk["sparse_pflops"]), "traffic": None}
+    else:
+        peak_gbs, peak_kind = read_peaks()
+        ach = per[dom.name]["gemm_gbs"]
+        roof = {"kernel": f"sharq_gemm_kernel ({dom.name})", "bound": "hbm", "achieved": ach, "peak": peak_gbs,
+                "unit": "GB/s", "frac": ach / peak_gbs, "peak_kind": peak_kind + " burst copy",
+                "traffic": None}
     line = None
     if rank == 0:
         ms_step = ms / args.steps
-        value = flops_per_step() * world / (ms_step * 1e-3) / 1e12
+        value = flops_step * world / (ms_step * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3 block scales, fp32 accumulate)",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "l2": f"inputs larger than L2: {N_ROT} rotating weight copies",
+            "config": {"workload": WORKLOADS[args.workload] + f", T in {tuple(args.T)}",
+                       "l2": (f"inputs larger than L2: {n_rot} rotating weight/activation copies"
+                              if n_rot > 1 else "working set larger than L2"),
                        "parallelism": "replicas" if world > 1 else "single"},
-            "per_T": {str(t): {k: round(v, 3) for k, v in per_t[t].items()} for t in T_LIST},
-            "roofline": {"kernel": f"sharq_gemm_kernel (T={dom})", "bound": "hbm", "achieved": achieved,
-                         "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "peak_kind": peak_kind + " burst copy", "traffic": None},
-            "e2e": {"value": flops_per_step() * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "layers": {n: {k: (round(v, 3) if isinstance(v, float) else v) for k, v in d.items()}
+                       for n, d in per.items()},
+            "roofline": roof,
+            "e2e": {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
     if world > 1:
-        for g in graphs:
-            del g
         graphs.clear()
         dist.barrier()
         dist.destroy_process_group()
@@ -359,14 +422,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--workload", default="q_proj", choices=["q_proj", "mlp"])
+    ap.add_argument("--T", type=int, nargs="+", default=None)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.T is None:
+        args.T = list(T_LIST) if args.workload == "q_proj" else [2048]
     world, rank, local = init_dist(args)
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.workload == "q_proj":
         cpu, _ = oracle_sample(args.cpu_seconds)   # before any CUDA work
     line = run_gpu(args, world, rank, local)
     if rank == 0 and line is not None:

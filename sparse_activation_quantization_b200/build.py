@@ -30,6 +30,7 @@ def _stale(objs):
         return True
     t = os.path.getmtime(LIB)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
+    deps.append(os.path.join(HERE, "peak", "fp4_peak.cu"))
     deps.append(os.path.join(HERE, "..", "include", "sharq.h"))
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
@@ -53,6 +54,12 @@ def build(force=False, verbose=False, extra=()):
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    # the FP4 peak microbenchmark (roofline denominators), a separate library
+    peak_src = os.path.join(HERE, "peak", "fp4_peak.cu")
+    peak_lib = os.path.join(HERE, "peak", "libsharq_peak.so")
+    subprocess.run([nvcc(), *ARCH, *FLAGS, "-shared", "-cudart", "static", peak_src, "-o", peak_lib + ".tmp"],
+                   check=True)
+    os.replace(peak_lib + ".tmp", peak_lib)
     return LIB
 
 
