@@ -56,6 +56,13 @@ def prep_alg_bytes(T, K):
     return T * K * 2 + Tp * K * 0.90625
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel per launch, from the ncu capture summarised in
+# profiles/sharq_gemm_qproj_decode.md; reset to None whenever that kernel
+# changes until it is captured again.
+NCU_TRAFFIC = {"q_proj_T128": None}
+
+
 def read_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -386,7 +393,7 @@ def run_gpu(args, world, rank, local):
         ach = per[dom.name]["gemm_gbs"]
         roof = {"kernel": f"sharq_gemm_kernel ({dom.name})", "bound": "hbm", "achieved": ach, "peak": peak_gbs,
                 "unit": "GB/s", "frac": ach / peak_gbs, "peak_kind": peak_kind + " burst copy",
-                "traffic": None}
+                "traffic": NCU_TRAFFIC.get(dom.name)}
     line = None
     if rank == 0:
         ms_step = ms / args.steps
