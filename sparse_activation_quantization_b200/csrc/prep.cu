@@ -152,15 +152,6 @@ __device__ __forceinline__ void depart_and_reset(unsigned int* sync) {
   }
 }
 
-// pick a[sel] for sel in 0..3 without dynamic register indexing
-__device__ __forceinline__ float pick4(const float* a, int sel) {
-  float r = a[0];
-  r = sel == 1 ? a[1] : r;
-  r = sel == 2 ? a[2] : r;
-  r = sel == 3 ? a[3] : r;
-  return r;
-}
-
 struct QuantPtrs {
   uint8_t* sp_codes;
   uint8_t* meta;
@@ -175,9 +166,31 @@ __device__ __forceinline__ float group_max(float v, int width) {
   return v;
 }
 
+// Keep mask of one 4:8 in-pairs run: bit p set = pair p kept.  Pair p is
+// kept iff fewer than two pairs beat it, where q beats p if its score is
+// larger, or equal with q < p; the six pairwise comparisons give every rank.
+__device__ __forceinline__ uint32_t keep_mask4(const float (&sc)[4]) {
+  const int c01 = sc[1] > sc[0], c02 = sc[2] > sc[0], c03 = sc[3] > sc[0];
+  const int c12 = sc[2] > sc[1], c13 = sc[3] > sc[1], c23 = sc[3] > sc[2];
+  const int r0 = c01 + c02 + c03;
+  const int r1 = (1 - c01) + c12 + c13;
+  const int r2 = (1 - c02) + (1 - c12) + c23;
+  const int r3 = (1 - c03) + (1 - c13) + (1 - c23);
+  return (uint32_t)(r0 < 2) | ((uint32_t)(r1 < 2) << 1) | ((uint32_t)(r2 < 2) << 2) | ((uint32_t)(r3 < 2) << 3);
+}
+
+// one byte of two E2M1 codes -> their values (exact), low nibble first
+__device__ __forceinline__ float2 e2m1x2_values(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 q;\n\tcvt.u8.u32 q, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, q;\n\t}" : "=r"(h2) : "r"(byte));
+  return __half22float2(*reinterpret_cast<__half2*>(&h2));
+}
+
 // Quantize NC consecutive runs of 8 logical K of row t, held in registers
 // (x[8*c + e] = run c, element e), starting at run index c0 of the row.
-// All 32 lanes of the warp must call it (warp shuffles).
+// NC = 4: every block is inside the thread.  NC = 1, 2: the 32-K block spans
+// 4 / NC adjacent lanes and (NC = 1) the 16-K block 2 lanes; all 32 lanes of
+// the warp must call it then (warp shuffles).
 template <int NC, bool kSharq>
 __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int c0, int K, float s, float six_s,
                                            const QuantPtrs& out, bool store = true) {
@@ -190,31 +203,20 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
   if (kSharq) {
     // --- 4:8 in-pairs mask per run: keep the 2 of 4 pairs with the largest max|x|
     float v[4 * NC];
-    int lo[NC], hi[NC];
+    uint32_t km[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-      float sc[4], ev[4], od[4];
+      float sc[4];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        ev[p] = x[8 * c + 2 * p];
-        od[p] = x[8 * c + 2 * p + 1];
-        sc[p] = fmaxf(fabsf(ev[p]), fabsf(od[p]));
-      }
-      int a = -1, b = -1;
-#pragma unroll
-      for (int p = 3; p >= 0; --p) {
-        int beaten = 0;
-#pragma unroll
-        for (int o = 0; o < 4; ++o)
-          if (o != p) beaten += (sc[o] > sc[p]) || (sc[o] == sc[p] && o < p);
-        if (beaten < 2) { b = a; a = p; }
-      }
-      lo[c] = a;
-      hi[c] = b;
-      v[4 * c + 0] = pick4(ev, a);
-      v[4 * c + 1] = pick4(od, a);
-      v[4 * c + 2] = pick4(ev, b);
-      v[4 * c + 3] = pick4(od, b);
+      for (int p = 0; p < 4; ++p) sc[p] = fmaxf(fabsf(x[8 * c + 2 * p]), fabsf(x[8 * c + 2 * p + 1]));
+      km[c] = keep_mask4(sc);
+      const bool k0 = km[c] & 1u, k1 = km[c] & 2u, k3 = km[c] & 8u;
+      // lowest kept pair (0..2) and highest kept pair (1..3)
+      const float* xc = x + 8 * c;
+      v[4 * c + 0] = k0 ? xc[0] : (k1 ? xc[2] : xc[4]);
+      v[4 * c + 1] = k0 ? xc[1] : (k1 ? xc[3] : xc[5]);
+      v[4 * c + 2] = k3 ? xc[6] : ((km[c] & 4u) ? xc[4] : xc[2]);
+      v[4 * c + 3] = k3 ? xc[7] : ((km[c] & 4u) ? xc[5] : xc[3]);
     }
     // --- backbone NVFP4: one scale per 32 logical K (4 runs = 16 kept values)
     float am = 0.0f;
@@ -222,45 +224,41 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
     for (int i = 0; i < 4 * NC; ++i) am = fmaxf(am, fabsf(v[i]));
     if (NC < 4) am = group_max(am, 4 / NC);
     const BlockScale bs = block_scale(am, six_s, s);
-    uint32_t code[4 * NC];
+    uint32_t cb[2 * NC];  // code bytes: kept values (2i, 2i+1)
 #pragma unroll
-    for (int i = 0; i < 2 * NC; ++i) {
-      const uint32_t by = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
-      code[2 * i] = by & 0xFu;
-      code[2 * i + 1] = by >> 4;
-    }
+    for (int i = 0; i < 2 * NC; ++i) cb[i] = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
     // --- residual R = Xn - dequant(backbone) at kept positions (exact fp32)
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const bool is_lo = (p == lo[c]), is_hi = (p == hi[c]);
-        if (is_lo || is_hi) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const uint32_t cd = is_lo ? code[4 * c + e] : code[4 * c + 2 + e];
-            const float xt = __fmul_rn(__fmul_rn(e2m1_value(cd), bs.dec), s);
-            res[8 * c + 2 * p + e] = __fsub_rn(x[8 * c + 2 * p + e], xt);
-          }
-        }
-      }
+      const float2 lo2 = e2m1x2_values(cb[2 * c]), hi2 = e2m1x2_values(cb[2 * c + 1]);
+      const float t0 = __fmul_rn(__fmul_rn(lo2.x, bs.dec), s), t1 = __fmul_rn(__fmul_rn(lo2.y, bs.dec), s);
+      const float t2 = __fmul_rn(__fmul_rn(hi2.x, bs.dec), s), t3 = __fmul_rn(__fmul_rn(hi2.y, bs.dec), s);
+      const uint32_t m = km[c];
+      const bool k0 = m & 1u, k1 = m & 2u, k2 = m & 4u, k3 = m & 8u;
+      // pair p holds (t0,t1) if it is the lowest kept pair, (t2,t3) if the highest
+      float* rc = res + 8 * c;
+      if (k0) { rc[0] = __fsub_rn(rc[0], t0); rc[1] = __fsub_rn(rc[1], t1); }
+      if (k1) { rc[2] = __fsub_rn(rc[2], k0 ? t2 : t0); rc[3] = __fsub_rn(rc[3], k0 ? t3 : t1); }
+      if (k2) { rc[4] = __fsub_rn(rc[4], k3 ? t0 : t2); rc[5] = __fsub_rn(rc[5], k3 ? t1 : t3); }
+      if (k3) { rc[6] = __fsub_rn(rc[6], t2); rc[7] = __fsub_rn(rc[7], t3); }
     }
     // --- stores: per run 2 bytes of kept codes, one metadata nibble
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-      const int g = c0 + c;            // run index in the row
+      const int g = c0 + c;               // run index in the row
       const int kt = g >> 5, w = g & 31;  // K tile, run within the 256-K tile
       const size_t tile = (size_t)(t >> 7) * KS + kt;
-      const uint32_t b0 = code[4 * c] | (code[4 * c + 1] << 4), b1 = code[4 * c + 2] | (code[4 * c + 3] << 4);
       if (store)
         *reinterpret_cast<uint16_t*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
-            (uint16_t)(b0 | (b1 << 8));
-      uint32_t nib = (uint32_t)(lo[c] | (hi[c] << 2));
+            (uint16_t)(cb[2 * c] | (cb[2 * c + 1] << 8));
+      const uint32_t m = km[c];
+      const uint32_t nib = (uint32_t)((__ffs(m) - 1) | ((31 - __clz(m)) << 2));
       if (NC == 1) {
         const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
         if (store && (w & 1) == 0) out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
       } else if (store && (c & 1) == 0) {
-        const uint32_t other = (uint32_t)(lo[c + 1 < NC ? c + 1 : c] | (hi[c + 1 < NC ? c + 1 : c] << 2));
+        const uint32_t m2 = km[c + 1 < NC ? c + 1 : c];
+        const uint32_t other = (uint32_t)((__ffs(m2) - 1) | ((31 - __clz(m2)) << 2));
         out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
       }
       if (store && (w & 3) == 0) out.sp_sf[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
@@ -270,28 +268,28 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
   // --- dense NVFP4 of R (or of Xn in NVFP4 mode): 16-element blocks
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
+    if (NC > 1 && (c & 1)) continue;  // the even run handles its block of two runs
+    const int nr = NC == 1 ? 1 : 2;   // runs of this block held by this thread
     float am = 0.0f;
-    if (NC == 1) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(res[i]));
-      am = group_max(am, 2);
-    } else {
-      const int c2 = c & ~1;  // this run and its partner form one block
-#pragma unroll
-      for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(res[8 * c2 + i]));
-    }
+    for (int i = 0; i < 8 * nr; ++i) am = fmaxf(am, fabsf(res[8 * c + i]));
+    if (NC == 1) am = group_max(am, 2);
     const BlockScale bs = block_scale(am, six_s, s);
-    uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      word |= cvt_e2m1x2(__fmul_rn(res[8 * c + 2 * i], bs.inv), __fmul_rn(res[8 * c + 2 * i + 1], bs.inv)) << (8 * i);
-    const int g = c0 + c;
-    const int kt = g >> 5, w = g & 31;
-    const size_t tile = (size_t)(t >> 7) * KS + kt;
-    if (store) {
-      *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
-          word;
-      if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+    for (int h = 0; h < nr; ++h) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        word |= cvt_e2m1x2(__fmul_rn(res[8 * (c + h) + 2 * i], bs.inv), __fmul_rn(res[8 * (c + h) + 2 * i + 1], bs.inv))
+                << (8 * i);
+      const int g = c0 + c + h;
+      const int kt = g >> 5, w = g & 31;
+      const size_t tile = (size_t)(t >> 7) * KS + kt;
+      if (store) {
+        *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
+            word;
+        if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+      }
     }
   }
 }
@@ -326,7 +324,8 @@ __device__ __forceinline__ void normalise_runs(float (&x)[8 * NC], const __nv_bf
 
 constexpr int kQuantThreads = 256;
 
-// Two-launch form, second launch: one thread per run of 8, flat over rows.
+// Two-launch form, second launch: one thread per 32 consecutive K (four runs
+// of 8; every quantization block inside the thread), flat over rows.
 template <bool kSharq>
 __global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
@@ -334,22 +333,21 @@ __global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
     const unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
   __shared__ float gmax_sh;
   allow_dependents();
-  const int runs = K >> 3;
+  const int segs = K >> 5;
   const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
   if (threadIdx.x == 0) gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
   __syncthreads();
   const float gmax = gmax_sh;
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (gid == 0) *s_g_out = s;  // published even when there are no rows
-  // whole warps go together: rows span whole warps (K/8 is a multiple of 32)
-  if (gid < (long long)T * runs) {
-    const int t = (int)(gid / runs);
-    const int c0 = (int)(gid - (long long)t * runs);
+  if (gid < (long long)T * segs) {
+    const int t = (int)(gid / segs);
+    const int c0 = (int)(gid - (long long)t * segs) * 4;
     const int src = row_index ? row_index[t] : t;
-    float x[8];
-    load_runs<1>(x, X, src, K, c0);
-    if (gamma && src >= 0) normalise_runs<1>(x, gamma, c0, inv_rms[t]);
-    quant_runs<1, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
+    float x[32];
+    load_runs<4>(x, X, src, K, c0);
+    if (gamma && src >= 0) normalise_runs<4>(x, gamma, c0, inv_rms[t]);
+    quant_runs<4, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
   }
   if (threadIdx.x == 0) depart_and_reset(const_cast<unsigned int*>(gmax_bits));
 }
@@ -587,7 +585,7 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   if (T > 0) {
     prep_stats_kernel<<<T, kStatsThreads, 0, stream>>>(Xb, Gb, eps, row_index, K, inv_rms, gmax_bits);
   }
-  const long long n = (long long)T * (K >> 3);
+  const long long n = (long long)T * (K >> 5);
   // at least one block so that s_g is published (= 1) even for T == 0
   const unsigned grid = n > 0 ? (unsigned)((n + kQuantThreads - 1) / kQuantThreads) : 1u;
   if (sharq_mode)
