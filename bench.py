@@ -34,7 +34,9 @@ EPS = 1e-5
 WORKLOAD = "llama3.1-8b q_proj K=4096 D=4096, T in {1,16,128}, RMSNorm gamma~U(0.5,1.5)"
 WORKLOADS = {"q_proj": "llama3.1-8b q_proj K=4096 D=4096 (prep+linear per T), RMSNorm gamma~U(0.5,1.5)",
              "mlp": "llama3.1-8b MLP prefill: gate/up 4096->14336 (shared prep, RMSNorm), down 14336->4096 "
-                    "(Student-t input)"}
+                    "(Student-t input)",
+             "qwen_layer": "qwen2.5-7b decoder-layer linears: qkv 3584->4608 (RMSNorm), o 3584->3584, "
+                           "gate+up 3584->37888 (RMSNorm), down 18944->3584 (Student-t input)"}
 METRIC = "prep+dual-GEMM effective TFLOP/s (2TKD)"
 
 
@@ -214,6 +216,14 @@ class Layer:
 def workload_layers(name, t_list):
     if name == "q_proj":
         return [Layer(f"q_proj_T{t}", t, K_DIM, D_DIM, True) for t in t_list]
+    if name == "qwen_layer":   # Qwen2.5-7B decoder-layer linears
+        out = []
+        for t in t_list:
+            out += [Layer(f"qkv_T{t}", t, 3584, 4608, True),
+                    Layer(f"o_proj_T{t}", t, 3584, 3584, False),
+                    Layer(f"gate_up_T{t}", t, 3584, 37888, True),
+                    Layer(f"down_T{t}", t, 18944, 3584, False, base="student_t")]
+        return out
     if name == "mlp":   # Llama-3.1-8B MLP at prefill: gate/up share one prep, then down
         out = []
         for t in t_list:
@@ -377,6 +387,26 @@ def run_gpu(args, world, rank, local):
         dist.all_reduce(t_, op=dist.ReduceOp.MAX)
         e2e_ms = t_.item()
 
+    # --- comparators on the same box: plain NVFP4 (dense FP4 GEMM only, same
+    # kernels in SHARQ_MODE_NVFP4) and bf16 cuBLAS (torch.matmul) ---------
+    comparators = None
+    if args.compare:
+        comparators = {}
+        for li, L in enumerate(layers):
+            act_n = sq.PreparedAct(L.T, L.K, mode=sq.SHARQ_MODE_NVFP4, device=dev)
+            src = L.shares or L.name
+            xn_ = xs[src][0]
+            nv = kernel_us(lambda i, L=L: (act_n.prep(xs[src][i], gammas[src], EPS, stream=stream),
+                                           sq.linear(act_n, weights[L.name][i], out=outs[L.name], ws=wss[L.name],
+                                                     stream=stream)), n_rot, stream)
+            Wb = [torch.from_numpy(synthetic.weights(100 + 31 * li + i, L.K, L.D)).to(torch.bfloat16).to(dev)
+                  for i in range(min(n_rot, 2))]
+            ob = torch.empty((L.T, L.D), dtype=torch.bfloat16, device=dev)
+            bf = kernel_us(lambda i, L=L: torch.matmul(xs[src][i], Wb[i % len(Wb)], out=ob), n_rot, stream)
+            comparators[L.name] = {"sharq_layer_us": round(per[L.name]["layer_us"], 3),
+                                   "nvfp4_layer_us": round(nv, 3), "bf16_cublas_us": round(bf, 3)}
+            del Wb, act_n
+
     flops_step = sum(L.flops for L in layers)
     # dominant kernel: the GEMM with the largest share of the step
     dom = max(layers, key=lambda L: per[L.name]["gemm_us"])
@@ -410,6 +440,7 @@ def run_gpu(args, world, rank, local):
             "layers": {n: {k: (round(v, 3) if isinstance(v, float) else v) for k, v in d.items()}
                        for n, d in per.items()},
             "roofline": roof,
+            "comparators": comparators,
             "e2e": {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
@@ -429,12 +460,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--workload", default="q_proj", choices=["q_proj", "mlp"])
+    ap.add_argument("--workload", default="q_proj", choices=["q_proj", "mlp", "qwen_layer"])
+    ap.add_argument("--compare", action="store_true",
+                    help="also time plain NVFP4 and bf16 cuBLAS on the same layers")
     ap.add_argument("--T", type=int, nargs="+", default=None)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.T is None:
-        args.T = list(T_LIST) if args.workload == "q_proj" else [2048]
+        args.T = {"q_proj": list(T_LIST), "mlp": [2048], "qwen_layer": [1, 64, 1024, 8192]}[args.workload]
     world, rank, local = init_dist(args)
     if args.impl == "reference":
         run_reference(args, world, rank)

@@ -116,11 +116,13 @@ def nvfp4_quant(v, s):
     return codes, sb, deq
 
 
-def prep(x, gamma=None, eps=1e-5):
+def prep(x, gamma=None, eps=1e-5, s_g=None):
     """The fused preparation step (xllm-io review, sections 3.2-3.5;
     kasblo.com explainer, steps 1-3).
 
     x: float32 [T, K] holding bf16 values, K a multiple of 32.
+    s_g: None (the per-tensor scale of x itself, section 3.5 "PTS"), or the
+    scale of a larger tensor that these rows are a subset of.
     Returns a dict of logical (untiled) arrays:
       xn [T,K], inv [T] or None, s_g, gmax,
       keep [T,K/8,4], meta [T,K/8]           4:8 in-pairs mask
@@ -132,7 +134,10 @@ def prep(x, gamma=None, eps=1e-5):
     """
     xn, inv = rmsnorm(x, gamma, eps)
     T, K = xn.shape
-    s_g, gmax = pts_scale(xn)
+    if s_g is None:
+        s_g, gmax = pts_scale(xn)
+    else:
+        s_g, gmax = np.float32(s_g), None
     keep, meta = pair_mask(xn)
     keep_el = np.repeat(keep, 2, axis=-1).reshape(T, K)               # [T,K]
     xsp = np.where(keep_el, xn, np.float32(0)).astype(np.float32)
