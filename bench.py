@@ -239,6 +239,8 @@ def kernel_us(fn, n_rot, stream, launches=96):
     back-to-back launches (rotating inputs), replayed, CUDA events."""
     import torch
     reps = max(1, launches // n_rot)
+    fn(0)                       # eager warm-up (library workspaces) before capture
+    torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for _ in range(reps):
