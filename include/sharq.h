@@ -225,6 +225,25 @@ int sharq_linear(const sharq_act *a, const sharq_weight *w, void *d_Y, int out_d
                  void *d_ws, size_t ws_bytes, sharq_stream_t stream);
 
 /*
+ * sharq_prep_linear - sharq_prep followed by sharq_linear, as one call
+ * (xllm-io review, sections 3.4-3.5).  For decode batches (T <= 32) it runs
+ * as ONE kernel: every GEMM CTA reads the T rows of X, computes the row
+ * 1/rms and the tensor max itself (identical values in every CTA), and
+ * quantizes its own K-slice straight into shared memory in the MMA layout
+ * while its weight tiles stream in, so no prepared activation goes through
+ * HBM and no separate prep kernel runs.  Codes, scales and Y are the same
+ * as sharq_prep + sharq_linear (same arithmetic and order).
+ * T > 32 runs sharq_prep into `a` (a view for T rows, SHARQ mode) and then
+ * sharq_linear; for T <= 32 `a` is not used and may be NULL.
+ * d_X: bf16 [T][K]; d_gamma: bf16 [K] or NULL; w: E == 1; d_Y: [T][D];
+ * d_ws: workspace of at least sharq_workspace_bytes(T, K, D, 1) bytes.
+ */
+#define SHARQ_FUSED_MAX_T 32
+int sharq_prep_linear(const void *d_X, const void *d_gamma, float eps, int T, const sharq_act *a,
+                      const sharq_weight *w, void *d_Y, int out_dtype, void *d_ws, size_t ws_bytes,
+                      sharq_stream_t stream);
+
+/*
  * sharq_linear_grouped - the same GEMM over E experts (xllm-io review,
  * section 5.1: SharQ on the expert linears of Qwen3-30B-A3B).
  * a: one prepared, expert-sorted activation tensor (one PTS scale), usually

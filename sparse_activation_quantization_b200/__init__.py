@@ -19,7 +19,7 @@ __all__ = [
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes",
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
-    "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
+    "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc", "sharq_prep_linear", "prep_linear",
     "PackedWeight", "PreparedAct", "Workspace", "linear", "EXPORTED_SYMBOLS",
 ]
 
@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = (
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes", "sharq_weight_view",
     "sharq_act_view", "sharq_pack_weight", "sharq_prep", "sharq_linear", "sharq_linear_grouped",
     "sharq_check_status", "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
+    "sharq_prep_linear",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +79,7 @@ def lib():
             "sharq_prep": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
             "sharq_prep_noalloc": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
             "sharq_linear": (i, [A, W, vp, i, vp, sz, vp]),
+            "sharq_prep_linear": (i, [vp, vp, ctypes.c_float, i, A, W, vp, i, vp, sz, vp]),
             "sharq_linear_grouped": (i, [A, vp, W, vp, i, vp, sz, vp]),
             "sharq_check_status": (i, [vp, vp]),
             "sharq_status_string": (ctypes.c_char_p, [i]),
@@ -146,6 +148,12 @@ def sharq_prep_noalloc(d_X, d_gamma, eps, d_row_index, a, stream):
 def sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream):
     return _check(lib().sharq_linear(ctypes.byref(a), ctypes.byref(w), d_Y, out_dtype, d_ws, ws_bytes, stream),
                   "sharq_linear")
+
+
+def sharq_prep_linear(d_X, d_gamma, eps, T, a, w, d_Y, out_dtype, d_ws, ws_bytes, stream):
+    return _check(lib().sharq_prep_linear(d_X, d_gamma, eps, T, ctypes.byref(a) if a is not None else None,
+                                          ctypes.byref(w), d_Y, out_dtype, d_ws, ws_bytes, stream),
+                  "sharq_prep_linear")
 
 
 def sharq_linear_grouped(a, d_offsets, w, d_Y, out_dtype, d_ws, ws_bytes, stream):
@@ -259,4 +267,23 @@ def linear(act, weight, out_dtype=None, out=None, ws=None, group_offsets=None, s
     else:
         sharq_linear_grouped(act.view, group_offsets.data_ptr(), weight.view, out.data_ptr(), code,
                              ws.buf.data_ptr(), ws.nbytes, s)
+    return out
+
+
+def prep_linear(X, gamma, eps, weight, act=None, out_dtype=None, out=None, ws=None, stream=None):
+    """Y = SharQ(X) W in one call (sharq_prep_linear): a single fused kernel for
+    T <= 32 rows, prep into `act` + linear above that."""
+    torch = _torch()
+    out_dtype = out_dtype or torch.bfloat16
+    code = SHARQ_OUT_F32 if out_dtype == torch.float32 else SHARQ_OUT_BF16
+    T, K = X.shape
+    if out is None:
+        out = torch.empty((T, weight.D), dtype=out_dtype, device=X.device)
+    if ws is None:
+        ws = Workspace(T, K, weight.D, 1, device=X.device)
+    if act is None and T > 32:
+        act = PreparedAct(T, K, device=X.device)
+    sharq_prep_linear(X.data_ptr(), gamma.data_ptr() if gamma is not None else None, float(eps), T,
+                      act.view if act is not None else None, weight.view, out.data_ptr(), code,
+                      ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream))
     return out

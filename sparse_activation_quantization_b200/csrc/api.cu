@@ -19,7 +19,8 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
-                          int* err, const int* act_err, cudaStream_t stream);
+                          int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
+                          const void* gamma_fused, float eps_fused);
 int noalloc_max_rows();
 cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
                                 int K, bool sharq_mode, float* s_g, uint8_t* sp_codes, uint8_t* meta,
@@ -170,7 +171,8 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
       out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, static_cast<int*>(d_ws),
-      reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<cudaStream_t>(stream));
+      reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr,
+      0.0f);
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 
@@ -299,6 +301,34 @@ int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const in
       static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta), static_cast<uint8_t*>(a->sp_sf),
       static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf), a->gmax_bits ? a->gmax_bits + 3 : nullptr,
       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
+}
+
+int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, const sharq_act* a,
+                      const sharq_weight* w, void* d_Y, int out_dtype, void* d_ws, size_t ws_bytes,
+                      sharq_stream_t stream) {
+  int st = weight_ok(w);
+  if (st) return st;
+  if (w->E != 1) return SHARQ_ERR_INVALID_ARG;
+  if (!shape_ok_t(T)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (T > SHARQ_FUSED_MAX_T) {  // larger batches: the two-call path through `a`
+    if (!a || a->T != T || a->K != w->K || a->mode != SHARQ_MODE_SHARQ) return SHARQ_ERR_INVALID_ARG;
+    if ((st = sharq_prep(d_X, d_gamma, eps, nullptr, a, stream))) return st;
+    return sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream);
+  }
+  if (out_dtype != SHARQ_OUT_BF16 && out_dtype != SHARQ_OUT_F32) return SHARQ_ERR_INVALID_ARG;
+  if (T > 0 && (!d_X || !aligned(d_X, 16) || !d_Y || !aligned(d_Y, 16))) return SHARQ_ERR_INVALID_ARG;
+  if (d_gamma && !aligned(d_gamma, 16)) return SHARQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return SHARQ_ERR_INVALID_ARG;
+  if (!d_ws || ws_bytes < sharq_workspace_bytes(T, w->K, w->D, 1) || !aligned(d_ws, 16)) return SHARQ_ERR_WORKSPACE;
+  if ((st = check_device())) return st;
+  if (T == 0) return SHARQ_OK;
+  const GemmShape g = gemm_shape(T, w->K, w->D, 1);
+  cudaError_t e = sharq::launch_linear(
+      nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, T, (int)round_up((size_t)T, 128), w->K, 1,
+      static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
+      static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, 1, nullptr, d_Y, out_dtype == SHARQ_OUT_F32 ? 1 : 0,
+      g.bn, g.splits, static_cast<int*>(d_ws), nullptr, reinterpret_cast<cudaStream_t>(stream), d_X, d_gamma, eps);
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 

@@ -37,7 +37,7 @@
 // shared memory once at start-up.
 // Every wait is bounded by the global timer; on timeout the CTA records
 // SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
-#include "sharq_device.cuh"
+#include "quant.cuh"
 
 namespace sharq {
 
@@ -84,6 +84,10 @@ struct GemmArgs {
   int out_f32;
   int sharq_mode;
   int splits;
+  // fused decode form: raw activations are prepared inside the GEMM
+  const __nv_bfloat16* X;      // [T][K] bf16
+  const __nv_bfloat16* gamma;  // [K] bf16 or nullptr
+  float eps;
 };
 
 template <int BN, bool kSplit>
@@ -122,6 +126,7 @@ struct Cfg {
   static constexpr uint32_t kTxSharq = BN * 128 + kHalves * (kSf32Tile + kSf16Tile) + kCodesTile + kSpTile +
                                        kMetaTile + kSf32Tile + kSf16Tile;
   static constexpr uint32_t kTxNvfp4 = BN * 128 + kHalves * kSf16Tile + kCodesTile + kSf16Tile;
+  static constexpr uint32_t kTxB = BN * 128 + kHalves * (kSf32Tile + kSf16Tile);  // weight side only
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kColsUsed <= 512, "TMEM overflow");
   static_assert(kSmemBytes <= 232448, "shared memory overflow");
@@ -181,7 +186,99 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, f
                : "memory");
 }
 
-template <int BN, bool kSplit>
+__device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void epi_barrier() {  // the 128 epilogue threads
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// The epilogue warps' prep phase of the fused decode form (128 threads, T <= 32
+// rows): row statistics over the full K, the tensor max, then the A half of
+// each stage of this CTA's K-slice, written in the MMA layout.
+template <class C>
+__device__ __forceinline__ void fused_prep(const GemmArgs& args, uint8_t* smem, int ks0, int nks, int T,
+                                           uint64_t deadline, volatile int* abort, uint64_t* empty_bar,
+                                           uint64_t* afull_bar, float* inv_sh, float* wmax_sh, float* sg_sh) {
+  const int ew = (threadIdx.x >> 5) - 2, lane = threadIdx.x & 31;
+  const int K = args.K, KS = K >> 8;
+  grid_dependency_wait();  // X comes from the preceding kernel
+  // 1. per row (rows ew, ew+4, ...): sum of squares -> 1/rms; max |Xn|
+  float wmax = 0.0f;
+  for (int r = ew; r < T; r += 4) {
+    const uint4* xr = reinterpret_cast<const uint4*>(args.X + (size_t)r * K) + lane;
+    float inv = 1.0f;
+    if (args.gamma) {
+      double ss = 0.0;
+#pragma unroll 4
+      for (int it = 0; it < KS; ++it) {
+        float f[8];
+        bf16x8_to_float(xr[it * 32], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += (double)f[e] * (double)f[e];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      inv = (float)(1.0 / sqrt(ss / (double)K + (double)args.eps));
+    }
+    if (lane == 0) inv_sh[r] = inv;
+    const uint4* gr = reinterpret_cast<const uint4*>(args.gamma) + lane;
+    float m = 0.0f;
+#pragma unroll 4
+    for (int it = 0; it < KS; ++it) {
+      float f[8];
+      bf16x8_to_float(xr[it * 32], f);
+      if (args.gamma) {
+        float g[8];
+        bf16x8_to_float(gr[it * 32], g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(norm_one(f[e], inv, g[e])));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+      }
+    }
+    wmax = fmaxf(wmax, m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+  if (lane == 0) wmax_sh[ew] = wmax;
+  epi_barrier();
+  const float gmax = fmaxf(fmaxf(wmax_sh[0], wmax_sh[1]), fmaxf(wmax_sh[2], wmax_sh[3]));
+  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
+  const float six_s = __fmul_rn(6.0f, s);
+  if (threadIdx.x == 64) *sg_sh = s;
+  // 2. the A half of every stage of this CTA's K-slice
+  for (int i = 0; i < nks; ++i) {
+    const int st = i % C::kStages;
+    if (i >= C::kStages && !mbar_wait(&empty_bar[st], ((i / C::kStages) & 1) ^ 1, deadline, abort)) break;
+    uint8_t* base = smem + st * C::kStageBytes;
+    const QuantPtrs q{base + C::kOffASP, base + C::kOffE, base + C::kOffSFASP, base + C::kOffAR, base + C::kOffSFAR};
+    const int k0 = (ks0 + i) * 256;
+    for (int r = ew; r < T; r += 4) {
+      float x[8];
+      load_runs<1>(x, args.X + k0, r, K, lane);   // row r, columns k0 + 8*lane ..
+      if (args.gamma) {
+        float g[8];
+        bf16x8_to_float(reinterpret_cast<const uint4*>(args.gamma + k0)[lane], g);
+        const float inv = inv_sh[r];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = norm_one(x[e], inv, g[e]);
+      }
+      quant_runs<1, true>(x, r, lane, 256, s, six_s, q);  // one 256-K tile: tile index 0
+    }
+    fence_proxy_async_smem();   // generic writes -> visible to tcgen05.cp / MMA
+    mbar_arrive_local(&afull_bar[st]);
+  }
+}
+
+// kFused: the decode form that prepares the activation itself.  Every CTA
+// reads all T (<= 32) rows of X, computes the row 1/rms and the tensor max
+// (the same values, in the same order, in every CTA), and quantizes its own
+// K-slice straight into the A half of each shared-memory stage, in the MMA
+// layout, while the producer streams the weight half.  No prepared
+// activation goes through HBM and no separate prep kernel runs.
+template <int BN, bool kSplit, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
   using C = Cfg<BN, kSplit>;
   extern __shared__ uint8_t smem_raw[];
@@ -189,9 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ __align__(8) uint64_t recv_bar;
+  __shared__ __align__(8) uint64_t afull_bar[kFused ? C::kStages : 1];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
+  __shared__ float inv_sh[kFused ? 32 : 1];
+  __shared__ float wmax_sh[4];
+  __shared__ float sg_sh;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -216,6 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
+    if (kFused)
+      for (int st = 0; st < C::kStages; ++st) mbar_init(&afull_bar[st], 128);  // the epilogue threads
     // one arrival per received row: S senders x my_n rows
     mbar_init(&recv_bar, kSplit && my_n > 0 ? (uint32_t)(S * my_n) : 1u);
     fence_mbar_init();
@@ -290,6 +393,22 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
         }
       };
+      if (kFused) {
+        // weight half only; the A half is written by the epilogue warps
+        for (int i = 0; i < nks; ++i) {
+          const int s = i % C::kStages;
+          if (i >= C::kStages) {
+            if (!mbar_wait(&empty_bar[s], ((i / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
+              record_error(args.err, kErrTimeout);
+              abort_sh = 1;
+              break;
+            }
+          }
+          mbar_arrive_expect_tx(&full_bar[s], C::kTxB);
+          issue_b(smem + s * C::kStageBytes, &full_bar[s], b_tile0, ks0 + i);
+          if (i == 0) TRACE_POINT(2);
+        }
+      } else {
       // The weights do not depend on the preceding kernel (sharq_prep): issue
       // the weight copies of the first ring's worth of stages before waiting
       // for it (programmatic dependent launch), then the activation copies.
@@ -315,6 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         issue_b(st, &full_bar[s], b_tile0, ks0 + i);
         issue_a(st, &full_bar[s], a_tile0 + ks0 + i);
       }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA ----
@@ -332,10 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         if (i == 0) TRACE_POINT(3);
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
         const uint32_t sf = tmem + C::kColSf0 + (uint32_t)(i & 1) * C::kSfRegion;
-        // scale factors (and metadata) shared memory -> TMEM
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+        // scale factors (and metadata) shared memory -> TMEM; the weight side
+        // first (in the fused form it lands before the activation is ready)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -343,16 +461,29 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
             tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
                              smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
         if (sharq) {
-          tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int h = 0; h < C::kHalves; ++h)
               tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
                                smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
+        }
+        if (kFused) {
+          if (!mbar_wait(&afull_bar[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+        if (sharq) {
+          tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
           // sparse backbone: 2 x (128 x BN x 128 logical K)
 #pragma unroll
           for (int j = 0; j < 2; ++j)
@@ -375,6 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     // ------------------------------------------------------- epilogue ----
     const int sp = warp & 3;  // TMEM lane quarter this warp may access
     const int rl = sp * 32 + lane;
+    if (kFused) fused_prep<C>(args, smem, ks0, nks, valid, deadline, &abort_sh, empty_bar, afull_bar, inv_sh,
+                              wmax_sh, &sg_sh);
     const bool ok = mbar_wait(&acc_bar, 0, deadline, &abort_sh);
     tc_fence_after();
     grid_dependency_wait();  // s_g is written by the preceding sharq_prep
@@ -383,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       record_error(args.err, kErrTimeout);
       abort_sh = 1;
     } else if (!kSplit) {
-      const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
+      const float scale = __fmul_rn(kFused ? sg_sh : *args.s_g, args.s_w[expert]);
       const int row = mt * 128 + rl;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
@@ -419,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   }
 
   if (threadIdx.x == 64) TRACE_POINT(6);
+  if (kFused) __syncthreads();  // sg_sh visible to every warp
   if (kSplit && my_n > 0) {
     grid_dependency_wait();
     // ------------------------ owner: sum the S received slices in rank order
@@ -429,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     if (!ok) {
       if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
     } else {
-      const float scale = __fmul_rn(*args.s_g, args.s_w[expert]);
+      const float scale = __fmul_rn(kFused ? sg_sh : *args.s_g, args.s_w[expert]);
       const float* recv = reinterpret_cast<const float*>(smem + C::kRingBytes);
       constexpr int q4 = BN / 4;
       for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
@@ -457,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   }
 }
 
-template <int BN, bool kSplit>
+template <int BN, bool kSplit, bool kFused>
 cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   using C = Cfg<BN, kSplit>;
   static bool attr_set[64] = {};
@@ -465,7 +599,7 @@ cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(sharq_gemm_kernel<BN, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(sharq_gemm_kernel<BN, kSplit, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
@@ -484,7 +618,7 @@ cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   attr[1].val.clusterDim.z = kSplit ? a.splits : 1;
   cfg.attrs = attr;
   cfg.numAttrs = kSplit ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<BN, kSplit>, a);
+  return cudaLaunchKernelEx(&cfg, sharq_gemm_kernel<BN, kSplit, kFused>, a);
 }
 
 }  // namespace
@@ -499,8 +633,9 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
-                          int* err, const int* act_err, cudaStream_t stream) {
-  GemmArgs a;
+                          int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
+                          const void* gamma_fused, float eps_fused) {
+  GemmArgs a = {};
   a.a_sp = a_sp;
   a.a_meta = a_meta;
   a.a_spsf = a_spsf;
@@ -522,13 +657,26 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.out_f32 = out_f32;
   a.sharq_mode = sharq_mode;
   a.splits = splits;
+  a.X = static_cast<const __nv_bfloat16*>(X_fused);
+  a.gamma = static_cast<const __nv_bfloat16*>(gamma_fused);
+  a.eps = eps_fused;
   const int m_tiles = Tp / 128;
   if (m_tiles == 0) return cudaSuccess;
+  if (X_fused) {  // fused decode form
+    if (T > 32 || m_tiles != 1 || !sharq_mode || group_offsets) return cudaErrorInvalidValue;
+    if (splits > 1) {
+      if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
+      return launch_cfg<128, true, true>(a, m_tiles, stream);
+    }
+    return bn == 256 ? launch_cfg<256, false, true>(a, m_tiles, stream)
+                     : launch_cfg<128, false, true>(a, m_tiles, stream);
+  }
   if (splits > 1) {
     if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
-    return launch_cfg<128, true>(a, m_tiles, stream);
+    return launch_cfg<128, true, false>(a, m_tiles, stream);
   }
-  return bn == 256 ? launch_cfg<256, false>(a, m_tiles, stream) : launch_cfg<128, false>(a, m_tiles, stream);
+  return bn == 256 ? launch_cfg<256, false, false>(a, m_tiles, stream)
+                   : launch_cfg<128, false, false>(a, m_tiles, stream);
 }
 
 }  // namespace sharq

@@ -20,7 +20,7 @@
 // threads (adjacent lanes), reduced with warp shuffles.  The residual never
 // leaves registers; every output is stored in the MMA-ready tiled layout of
 // include/sharq.h.
-#include "sharq_device.cuh"
+#include "quant.cuh"
 
 namespace sharq {
 
@@ -40,21 +40,6 @@ __device__ unsigned long long* g_trace_prep = nullptr;
   do {                \
   } while (0)
 #endif
-
-__device__ __forceinline__ void bf16x8_to_float(const uint4& v, float* f) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 p = __bfloat1622float2(h[i]);
-    f[2 * i] = p.x;
-    f[2 * i + 1] = p.y;
-  }
-}
-
-// Xn = bf16_rn(f32(f32(x * inv) * g))
-__device__ __forceinline__ float norm_one(float x, float inv, float g) {
-  return __bfloat162float(__float2bfloat16_rn(__fmul_rn(__fmul_rn(x, inv), g)));
-}
 
 template <int NW>
 __device__ __forceinline__ double block_sum_d(double v, double* sh) {
@@ -149,176 +134,6 @@ __device__ __forceinline__ void depart_and_reset(unsigned int* sync) {
     sync[1] = 0u;
     sync[2] = 0u;
     __threadfence();
-  }
-}
-
-struct QuantPtrs {
-  uint8_t* sp_codes;
-  uint8_t* meta;
-  uint8_t* sp_sf;
-  uint8_t* r_codes;
-  uint8_t* r_sf;
-};
-
-// max over the `width` adjacent lanes of an aligned lane group
-__device__ __forceinline__ float group_max(float v, int width) {
-  for (int o = 1; o < width; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// Keep mask of one 4:8 in-pairs run: bit p set = pair p kept.  Pair p is
-// kept iff fewer than two pairs beat it, where q beats p if its score is
-// larger, or equal with q < p; the six pairwise comparisons give every rank.
-__device__ __forceinline__ uint32_t keep_mask4(const float (&sc)[4]) {
-  const int c01 = sc[1] > sc[0], c02 = sc[2] > sc[0], c03 = sc[3] > sc[0];
-  const int c12 = sc[2] > sc[1], c13 = sc[3] > sc[1], c23 = sc[3] > sc[2];
-  const int r0 = c01 + c02 + c03;
-  const int r1 = (1 - c01) + c12 + c13;
-  const int r2 = (1 - c02) + (1 - c12) + c23;
-  const int r3 = (1 - c03) + (1 - c13) + (1 - c23);
-  return (uint32_t)(r0 < 2) | ((uint32_t)(r1 < 2) << 1) | ((uint32_t)(r2 < 2) << 2) | ((uint32_t)(r3 < 2) << 3);
-}
-
-// one byte of two E2M1 codes -> their values (exact), low nibble first
-__device__ __forceinline__ float2 e2m1x2_values(uint32_t byte) {
-  uint32_t h2;
-  asm("{\n\t.reg .b8 q;\n\tcvt.u8.u32 q, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, q;\n\t}" : "=r"(h2) : "r"(byte));
-  return __half22float2(*reinterpret_cast<__half2*>(&h2));
-}
-
-// Quantize NC consecutive runs of 8 logical K of row t, held in registers
-// (x[8*c + e] = run c, element e), starting at run index c0 of the row.
-// NC = 4: every block is inside the thread.  NC = 1, 2: the 32-K block spans
-// 4 / NC adjacent lanes and (NC = 1) the 16-K block 2 lanes; all 32 lanes of
-// the warp must call it then (warp shuffles).
-template <int NC, bool kSharq>
-__device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int c0, int K, float s, float six_s,
-                                           const QuantPtrs& out, bool store = true) {
-  const int KS = K >> 8;
-  const int r = t & 127;
-  float res[8 * NC];
-#pragma unroll
-  for (int i = 0; i < 8 * NC; ++i) res[i] = x[i];
-
-  if (kSharq) {
-    // --- 4:8 in-pairs mask per run: keep the 2 of 4 pairs with the largest max|x|
-    float v[4 * NC];
-    uint32_t km[NC];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      float sc[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) sc[p] = fmaxf(fabsf(x[8 * c + 2 * p]), fabsf(x[8 * c + 2 * p + 1]));
-      km[c] = keep_mask4(sc);
-      const bool k0 = km[c] & 1u, k1 = km[c] & 2u, k3 = km[c] & 8u;
-      // lowest kept pair (0..2) and highest kept pair (1..3)
-      const float* xc = x + 8 * c;
-      v[4 * c + 0] = k0 ? xc[0] : (k1 ? xc[2] : xc[4]);
-      v[4 * c + 1] = k0 ? xc[1] : (k1 ? xc[3] : xc[5]);
-      v[4 * c + 2] = k3 ? xc[6] : ((km[c] & 4u) ? xc[4] : xc[2]);
-      v[4 * c + 3] = k3 ? xc[7] : ((km[c] & 4u) ? xc[5] : xc[3]);
-    }
-    // --- backbone NVFP4: one scale per 32 logical K (4 runs = 16 kept values)
-    float am = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4 * NC; ++i) am = fmaxf(am, fabsf(v[i]));
-    if (NC < 4) am = group_max(am, 4 / NC);
-    const BlockScale bs = block_scale(am, six_s, s);
-    uint32_t cb[2 * NC];  // code bytes: kept values (2i, 2i+1)
-#pragma unroll
-    for (int i = 0; i < 2 * NC; ++i) cb[i] = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
-    // --- residual R = Xn - dequant(backbone) at kept positions (exact fp32)
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      const float2 lo2 = e2m1x2_values(cb[2 * c]), hi2 = e2m1x2_values(cb[2 * c + 1]);
-      const float t0 = __fmul_rn(__fmul_rn(lo2.x, bs.dec), s), t1 = __fmul_rn(__fmul_rn(lo2.y, bs.dec), s);
-      const float t2 = __fmul_rn(__fmul_rn(hi2.x, bs.dec), s), t3 = __fmul_rn(__fmul_rn(hi2.y, bs.dec), s);
-      const uint32_t m = km[c];
-      const bool k0 = m & 1u, k1 = m & 2u, k2 = m & 4u, k3 = m & 8u;
-      // pair p holds (t0,t1) if it is the lowest kept pair, (t2,t3) if the highest
-      float* rc = res + 8 * c;
-      if (k0) { rc[0] = __fsub_rn(rc[0], t0); rc[1] = __fsub_rn(rc[1], t1); }
-      if (k1) { rc[2] = __fsub_rn(rc[2], k0 ? t2 : t0); rc[3] = __fsub_rn(rc[3], k0 ? t3 : t1); }
-      if (k2) { rc[4] = __fsub_rn(rc[4], k3 ? t0 : t2); rc[5] = __fsub_rn(rc[5], k3 ? t1 : t3); }
-      if (k3) { rc[6] = __fsub_rn(rc[6], t2); rc[7] = __fsub_rn(rc[7], t3); }
-    }
-    // --- stores: per run 2 bytes of kept codes, one metadata nibble
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      const int g = c0 + c;               // run index in the row
-      const int kt = g >> 5, w = g & 31;  // K tile, run within the 256-K tile
-      const size_t tile = (size_t)(t >> 7) * KS + kt;
-      if (store)
-        *reinterpret_cast<uint16_t*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
-            (uint16_t)(cb[2 * c] | (cb[2 * c + 1] << 8));
-      const uint32_t m = km[c];
-      const uint32_t nib = (uint32_t)((__ffs(m) - 1) | ((31 - __clz(m)) << 2));
-      if (NC == 1) {
-        const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
-        if (store && (w & 1) == 0) out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
-      } else if (store && (c & 1) == 0) {
-        const uint32_t m2 = km[c + 1 < NC ? c + 1 : c];
-        const uint32_t other = (uint32_t)((__ffs(m2) - 1) | ((31 - __clz(m2)) << 2));
-        out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
-      }
-      if (store && (w & 3) == 0) out.sp_sf[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
-    }
-  }
-
-  // --- dense NVFP4 of R (or of Xn in NVFP4 mode): 16-element blocks
-#pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    if (NC > 1 && (c & 1)) continue;  // the even run handles its block of two runs
-    const int nr = NC == 1 ? 1 : 2;   // runs of this block held by this thread
-    float am = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8 * nr; ++i) am = fmaxf(am, fabsf(res[8 * c + i]));
-    if (NC == 1) am = group_max(am, 2);
-    const BlockScale bs = block_scale(am, six_s, s);
-#pragma unroll
-    for (int h = 0; h < nr; ++h) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        word |= cvt_e2m1x2(__fmul_rn(res[8 * (c + h) + 2 * i], bs.inv), __fmul_rn(res[8 * (c + h) + 2 * i + 1], bs.inv))
-                << (8 * i);
-      const int g = c0 + c + h;
-      const int kt = g >> 5, w = g & 31;
-      const size_t tile = (size_t)(t >> 7) * KS + kt;
-      if (store) {
-        *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
-            word;
-        if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
-      }
-    }
-  }
-}
-
-// load NC runs of 8 (one 16-byte load each) and normalise them
-template <int NC>
-__device__ __forceinline__ void load_runs(float (&x)[8 * NC], const __nv_bfloat16* X, int src, int K, int c0) {
-  if (src >= 0) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K) + c0;
-    uint4 raw[NC];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) raw[c] = xr[c];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) bf16x8_to_float(raw[c], x + 8 * c);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8 * NC; ++i) x[i] = 0.0f;
-  }
-}
-
-template <int NC>
-__device__ __forceinline__ void normalise_runs(float (&x)[8 * NC], const __nv_bfloat16* gamma, int c0, float inv) {
-  const uint4* gr = reinterpret_cast<const uint4*>(gamma) + c0;
-#pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    float g[8];
-    bf16x8_to_float(gr[c], g);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[8 * c + e] = norm_one(x[8 * c + e], inv, g[e]);
   }
 }
 
