@@ -305,13 +305,27 @@ def run_gpu(args, world, rank, local):
         src = L.shares or L.name
         sq.linear(acts[src], weights[L.name][i], out=outs[L.name], ws=wss[L.name], stream=stream)
 
-    def step(i):
-        for L in layers:
+    FUSED_MAX_T = 32   # include/sharq.h SHARQ_FUSED_MAX_T: one-kernel prep+GEMM
+
+    def fused(L):
+        return not L.shares and L.T <= FUSED_MAX_T and not any(M.shares == L.name for M in layers)
+
+    def layer(L, i):
+        """one whole layer through the public API: sharq_prep_linear where the
+        prepared activation is not shared, else sharq_prep + sharq_linear"""
+        if fused(L):
+            sq.prep_linear(xs[L.name][i], gammas[L.name], EPS, weights[L.name][i], out=outs[L.name],
+                           ws=wss[L.name], stream=stream)
+        else:
             if not L.shares:
                 prep(L, i)
             gemm(L, i)
 
-    launches_per_step = sum(1 if L.shares else 2 for L in layers)   # single-launch prep + gemm
+    def step(i):
+        for L in layers:
+            layer(L, i)
+
+    launches_per_step = sum(1 if (L.shares or fused(L)) else 2 for L in layers)
     for i in range(n_rot):
         step(i)
     torch.cuda.synchronize()
@@ -351,8 +365,9 @@ def run_gpu(args, world, rank, local):
     for L in layers:
         g_us = kernel_us(lambda i, L=L: gemm(L, i), n_rot, stream)
         p_us = None if L.shares else kernel_us(lambda i, L=L: prep(L, i), n_rot, stream)
-        lay = kernel_us(lambda i, L=L: (None if L.shares else prep(L, i), gemm(L, i)), n_rot, stream)
-        per[L.name] = {"T": L.T, "K": L.K, "D": L.D, "layer_us": lay, "gemm_us": g_us, "prep_us": p_us,
+        lay = kernel_us(lambda i, L=L: layer(L, i), n_rot, stream)
+        per[L.name] = {"T": L.T, "K": L.K, "D": L.D, "fused": fused(L), "layer_us": lay, "gemm_us": g_us,
+                       "prep_us": p_us,
                        "layer_tflops": L.flops / (lay * 1e-6) / 1e12,
                        "gemm_tflops": L.flops / (g_us * 1e-6) / 1e12,
                        "gemm_gbs": gemm_alg_bytes(L.T, L.K, L.D) / (g_us * 1e-6) / 1e9,
@@ -370,8 +385,13 @@ def run_gpu(args, world, rank, local):
         for L in layers:
             if not L.shares:
                 dx[L.name].copy_(hx[L.name], non_blocking=True)
-                acts[L.name].prep(dx[L.name], gammas[L.name], EPS, stream=stream)
-            gemm(L, i)
+            if fused(L):
+                sq.prep_linear(dx[L.name], gammas[L.name], EPS, weights[L.name][i], out=outs[L.name],
+                               ws=wss[L.name], stream=stream)
+            else:
+                if not L.shares:
+                    acts[L.name].prep(dx[L.name], gammas[L.name], EPS, stream=stream)
+                gemm(L, i)
             hy[L.name].copy_(outs[L.name], non_blocking=True)
     for i in range(3):
         e2e_step(i % n_rot)
