@@ -308,7 +308,8 @@ def run_gpu(args, world, rank, local):
     FUSED_MAX_T = 32   # include/sharq.h SHARQ_FUSED_MAX_T: one-kernel prep+GEMM
 
     def fused(L):
-        return not L.shares and L.T <= FUSED_MAX_T and not any(M.shares == L.name for M in layers)
+        return (args.decode_form == "fused" and not L.shares and L.T <= FUSED_MAX_T
+                and not any(M.shares == L.name for M in layers))
 
     def layer(L, i):
         """one whole layer through the public API: sharq_prep_linear where the
@@ -458,7 +459,9 @@ def run_gpu(args, world, rank, local):
             "config": {"workload": WORKLOADS[args.workload] + f", T in {tuple(args.T)}",
                        "l2": (f"inputs larger than L2: {n_rot} rotating weight/activation copies"
                               if n_rot > 1 else "working set larger than L2"),
-                       "parallelism": "replicas" if world > 1 else "single"},
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "decode_form": ("sharq_prep_linear (one kernel for T <= 32)" if args.decode_form == "fused"
+                                       else "sharq_prep + sharq_linear")},
             "layers": {n: {k: (round(v, 3) if isinstance(v, float) else v) for k, v in d.items()}
                        for n, d in per.items()},
             "roofline": roof,
@@ -486,6 +489,8 @@ def main():
     ap.add_argument("--compare", action="store_true",
                     help="also time plain NVFP4 and bf16 cuBLAS on the same layers")
     ap.add_argument("--T", type=int, nargs="+", default=None)
+    ap.add_argument("--decode-form", default="two", choices=["two", "fused"],
+                    help="T <= 32 layers: sharq_prep + sharq_linear (two) or sharq_prep_linear's single kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.T is None:

@@ -45,15 +45,17 @@ namespace {
 
 constexpr int kThreads = 192;
 
-// Optional phase timeline (compile with -DSHARQ_TRACE): 8 global-timer
+// Optional phase timeline (compile with -DSHARQ_TRACE): 16 global-timer
 // stamps per CTA -- entry, set-up done, first stage issued, first stage
-// consumed, last MMA committed, accumulator ready, epilogue done, exit.
+// consumed, last MMA committed, accumulator ready, epilogue done, exit; in the
+// fused form also: dependency resolved, 1/rms known, s_g known, first and
+// last activation stage written.
 #ifdef SHARQ_TRACE
 __device__ unsigned long long* g_trace = nullptr;
 #define TRACE_POINT(k)                                                                                   \
   do {                                                                                                   \
     if (g_trace)                                                                                         \
-      g_trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 8 + (k)] =      \
+      g_trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 16 + (k)] =     \
           globaltimer_ns();                                                                              \
   } while (0)
 #else
@@ -193,91 +195,220 @@ __device__ __forceinline__ void epi_barrier() {  // the 128 epilogue threads
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-// The epilogue warps' prep phase of the fused decode form (128 threads, T <= 32
-// rows): row statistics over the full K, the tensor max, then the A half of
-// each stage of this CTA's K-slice, written in the MMA layout.
-template <class C>
-__device__ __forceinline__ void fused_prep(const GemmArgs& args, uint8_t* smem, int ks0, int nks, int T,
-                                           uint64_t deadline, volatile int* abort, uint64_t* empty_bar,
-                                           uint64_t* afull_bar, float* inv_sh, float* wmax_sh, float* sg_sh) {
-  const int ew = (threadIdx.x >> 5) - 2, lane = threadIdx.x & 31;
-  const int K = args.K, KS = K >> 8;
-  grid_dependency_wait();  // X comes from the preceding kernel
-  // 1. per row (rows ew, ew+4, ...): sum of squares -> 1/rms; max |Xn|
-  float wmax = 0.0f;
-  for (int r = ew; r < T; r += 4) {
-    const uint4* xr = reinterpret_cast<const uint4*>(args.X + (size_t)r * K) + lane;
-    float inv = 1.0f;
-    if (args.gamma) {
-      double ss = 0.0;
-#pragma unroll 4
-      for (int it = 0; it < KS; ++it) {
-        float f[8];
-        bf16x8_to_float(xr[it * 32], f);
+__device__ __forceinline__ void st_cluster_f64(uint32_t addr, double v) {
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(addr), "d"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Sum, across the 32 lanes, eight per-lane values at once (a transposing
+// butterfly: 9 double shuffles instead of 40).  Lane l returns the total of
+// value (l >> 2) & 7.
+__device__ __forceinline__ double warp_sum8(double (&v)[8], int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  double w4[4], w2[2];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss += (double)f[e] * (double)f[e];
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      inv = (float)(1.0 / sqrt(ss / (double)K + (double)args.eps));
-    }
-    if (lane == 0) inv_sh[r] = inv;
-    const uint4* gr = reinterpret_cast<const uint4*>(args.gamma) + lane;
-    float m = 0.0f;
-#pragma unroll 4
-    for (int it = 0; it < KS; ++it) {
-      float f[8];
-      bf16x8_to_float(xr[it * 32], f);
-      if (args.gamma) {
-        float g[8];
-        bf16x8_to_float(gr[it * 32], g);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(norm_one(f[e], inv, g[e])));
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
-      }
-    }
-    wmax = fmaxf(wmax, m);
+  for (int j = 0; j < 4; ++j) {
+    const double send = b4 ? v[j] : v[j + 4];
+    const double keep = b4 ? v[j + 4] : v[j];
+    w4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
-  if (lane == 0) wmax_sh[ew] = wmax;
+  for (int j = 0; j < 2; ++j) {
+    const double send = b3 ? w4[j] : w4[j + 2];
+    const double keep = b3 ? w4[j + 2] : w4[j];
+    w2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  double w = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
+  w += __shfl_xor_sync(0xffffffffu, w, 2);
+  w += __shfl_xor_sync(0xffffffffu, w, 1);
+  return w;
+}
+
+// Shared state of the fused decode form's statistics exchange.
+template <bool kSplit>
+struct FusedStats {
+  double part[4][32];                // per epilogue warp, per row: sum of squares over this CTA's K-slice
+  double ss[kSplit ? 8 : 1][32];     // per cluster rank, per row (written by the peers)
+  float mx[kSplit ? 8 : 1];          // per cluster rank: max |Xn| over its K-slice
+  float inv[32];                     // 1/rms per row
+  float wmax[4];
+  float s;                           // the per-tensor scale s_g
+};
+
+// bounded wait on a barrier that peers of the cluster arrive on
+__device__ __forceinline__ bool cluster_bar_wait(uint64_t* bar, uint64_t deadline, volatile int* abort) {
+  while (!mbar_try_wait_cluster(bar, 0)) {
+    if (*abort || globaltimer_ns() > deadline) return false;
+  }
+  return true;
+}
+
+// The epilogue warps' prep phase of the fused decode form (128 threads,
+// T <= 32 rows, this CTA's K-slice of ks tiles [ks0, ks0 + nks)).
+//  1. sum of squares of every row over the K-slice (fp64), exchanged with the
+//     S - 1 other CTAs of the cluster, which hold the rest of K; every CTA
+//     adds the S partials in rank order -> identical 1/rms everywhere;
+//  2. max |Xn| over the K-slice, exchanged the same way -> s_g;
+//  3. the A half of every stage of the K-slice, in the MMA layout.
+// Loads are issued eight rows at a time, so each warp keeps eight 16-byte
+// loads in flight instead of walking whole rows one load after another.
+template <class C, bool kSplit>
+__device__ __forceinline__ bool fused_prep(const GemmArgs& args, uint8_t* smem, int ks0, int nks, int T, int S,
+                                           uint64_t deadline, volatile int* abort, uint64_t* empty_bar,
+                                           uint64_t* afull_bar, uint64_t* stat_bar, FusedStats<kSplit>& fs) {
+  const int ew = (threadIdx.x >> 5) - 2, lane = threadIdx.x & 31;
+  const int K = args.K;
+  const uint32_t rank = kSplit ? cluster_ctarank() : 0u;
+  const __nv_bfloat16* Xs = args.X + (size_t)ks0 * 256 + lane * 8;  // this lane's column in tile 0 of the slice
+  grid_dependency_wait();  // X comes from the preceding kernel
+  if (threadIdx.x == 64) TRACE_POINT(8);
+  // ---- 1. sums of squares -> 1/rms
+  if (args.gamma) {
+    for (int r0 = 0; r0 < T; r0 += 8) {
+      double acc[8];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) acc[g] = 0.0;
+#pragma unroll 2
+      for (int i = ew; i < nks; i += 4) {
+        uint4 raw[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          raw[g] = r0 + g < T ? *reinterpret_cast<const uint4*>(Xs + (size_t)(r0 + g) * K + i * 256)
+                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          float f[8];
+          bf16x8_to_float(raw[g], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[g] += (double)f[e] * (double)f[e];
+        }
+      }
+      const double tot = warp_sum8(acc, lane);
+      const int r = r0 + ((lane >> 2) & 7);
+      if ((lane & 3) == 0 && r < T) fs.part[ew][r] = tot;
+    }
+    epi_barrier();
+    if (ew == 0 && lane < T) {
+      const double ps = ((fs.part[0][lane] + fs.part[1][lane]) + fs.part[2][lane]) + fs.part[3][lane];
+      if (kSplit) {
+        const uint32_t dst = smem_u32(&fs.ss[rank][lane]);
+        for (int p = 0; p < S; ++p) st_cluster_f64(mapa_shared(dst, (uint32_t)p), ps);
+        // each row's sender releases its own stores: S x T arrivals per CTA
+        for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stat_bar[0]), (uint32_t)p));
+      } else {
+        fs.ss[0][lane] = ps;
+      }
+    }
+    if (kSplit) {
+      if (!cluster_bar_wait(&stat_bar[0], deadline, abort)) return false;
+    } else {
+      epi_barrier();
+    }
+    if (ew == 0 && lane < T) {
+      double tot = fs.ss[0][lane];
+      for (int p = 1; p < (kSplit ? S : 1); ++p) tot += fs.ss[p][lane];
+      fs.inv[lane] = (float)(1.0 / sqrt(tot / (double)K + (double)args.eps));
+    }
+  } else if (ew == 0 && lane < T) {
+    fs.inv[lane] = 1.0f;
+  }
   epi_barrier();
-  const float gmax = fmaxf(fmaxf(wmax_sh[0], wmax_sh[1]), fmaxf(wmax_sh[2], wmax_sh[3]));
+  if (threadIdx.x == 64) TRACE_POINT(9);
+  // ---- 2. max |Xn| over the slice -> s_g
+  float m = 0.0f;
+  const __nv_bfloat16* Gs = args.gamma ? args.gamma + (size_t)ks0 * 256 + lane * 8 : nullptr;
+  for (int r0 = 0; r0 < T; r0 += 8) {
+#pragma unroll 2
+    for (int i = ew; i < nks; i += 4) {
+      uint4 raw[8];
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        raw[g] = r0 + g < T ? *reinterpret_cast<const uint4*>(Xs + (size_t)(r0 + g) * K + i * 256)
+                            : make_uint4(0u, 0u, 0u, 0u);
+      float gm[8];
+      if (Gs) bf16x8_to_float(*reinterpret_cast<const uint4*>(Gs + i * 256), gm);
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        float f[8];
+        bf16x8_to_float(raw[g], f);
+        const float inv = fs.inv[min(r0 + g, T - 1)];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(Gs ? norm_one(f[e], inv, gm[e]) : f[e]));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) fs.wmax[ew] = m;
+  epi_barrier();
+  if (threadIdx.x == 64) {
+    const float cm = fmaxf(fmaxf(fs.wmax[0], fs.wmax[1]), fmaxf(fs.wmax[2], fs.wmax[3]));
+    if (kSplit) {
+      const uint32_t dst = smem_u32(&fs.mx[rank]);
+      for (int p = 0; p < S; ++p) st_cluster_f32(mapa_shared(dst, (uint32_t)p), cm);
+      for (int p = 0; p < S; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&stat_bar[1]), (uint32_t)p));
+    } else {
+      fs.mx[0] = cm;
+    }
+  }
+  if (kSplit) {
+    if (!cluster_bar_wait(&stat_bar[1], deadline, abort)) return false;
+  } else {
+    epi_barrier();
+  }
+  float gmax = fs.mx[0];
+  for (int p = 1; p < (kSplit ? S : 1); ++p) gmax = fmaxf(gmax, fs.mx[p]);
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   const float six_s = __fmul_rn(6.0f, s);
-  if (threadIdx.x == 64) *sg_sh = s;
-  // 2. the A half of every stage of this CTA's K-slice
+  if (threadIdx.x == 64) {
+    fs.s = s;
+    TRACE_POINT(10);
+  }
+  // ---- 3. the A half of every stage of this CTA's K-slice (rows ew, ew+4, ...)
   for (int i = 0; i < nks; ++i) {
     const int st = i % C::kStages;
-    if (i >= C::kStages && !mbar_wait(&empty_bar[st], ((i / C::kStages) & 1) ^ 1, deadline, abort)) break;
+    uint4 raw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = ew + 4 * j;
+      raw[j] = r < T ? *reinterpret_cast<const uint4*>(Xs + (size_t)r * K + i * 256) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float gm[8];
+    if (Gs) bf16x8_to_float(*reinterpret_cast<const uint4*>(Gs + i * 256), gm);
+    if (i >= C::kStages && !mbar_wait(&empty_bar[st], ((i / C::kStages) & 1) ^ 1, deadline, abort)) return false;
     uint8_t* base = smem + st * C::kStageBytes;
     const QuantPtrs q{base + C::kOffASP, base + C::kOffE, base + C::kOffSFASP, base + C::kOffAR, base + C::kOffSFAR};
-    const int k0 = (ks0 + i) * 256;
-    for (int r = ew; r < T; r += 4) {
-      float x[8];
-      load_runs<1>(x, args.X + k0, r, K, lane);   // row r, columns k0 + 8*lane ..
-      if (args.gamma) {
-        float g[8];
-        bf16x8_to_float(reinterpret_cast<const uint4*>(args.gamma + k0)[lane], g);
-        const float inv = inv_sh[r];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = norm_one(x[e], inv, g[e]);
+    for (int j = 0; j < 8; ++j) {
+      const int r = ew + 4 * j;
+      if (r < T) {
+        float x[8];
+        bf16x8_to_float(raw[j], x);
+        if (Gs) {
+          const float inv = fs.inv[r];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = norm_one(x[e], inv, gm[e]);
+        }
+        quant_runs<1, true>(x, r, lane, 256, s, six_s, q);  // one 256-K tile: tile index 0
       }
-      quant_runs<1, true>(x, r, lane, 256, s, six_s, q);  // one 256-K tile: tile index 0
     }
     fence_proxy_async_smem();   // generic writes -> visible to tcgen05.cp / MMA
     mbar_arrive_local(&afull_bar[st]);
+    if (threadIdx.x == 64 && (i == 0 || i == nks - 1)) TRACE_POINT(i == 0 ? 11 : 12);
   }
+  return true;
 }
 
-// kFused: the decode form that prepares the activation itself.  Every CTA
-// reads all T (<= 32) rows of X, computes the row 1/rms and the tensor max
-// (the same values, in the same order, in every CTA), and quantizes its own
+// kFused: the decode form that prepares the activation itself.  The S CTAs
+// of a cluster split K between them: each reduces the row sums of squares and
+// the |Xn| max over its own K-slice and the partials are exchanged over
+// distributed shared memory (combined in rank order, so every CTA of every
+// cluster derives the same 1/rms and s_g); each CTA then quantizes its own
 // K-slice straight into the A half of each shared-memory stage, in the MMA
-// layout, while the producer streams the weight half.  No prepared
-// activation goes through HBM and no separate prep kernel runs.
+// layout, while the producer streams the weight half.  No prepared activation
+// goes through HBM and no separate prep kernel runs.
 template <int BN, bool kSplit, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
   using C = Cfg<BN, kSplit>;
@@ -290,9 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
-  __shared__ float inv_sh[kFused ? 32 : 1];
-  __shared__ float wmax_sh[4];
-  __shared__ float sg_sh;
+  __shared__ __align__(8) uint64_t stat_bar[2];
+  __shared__ __align__(8) FusedStats<kSplit> fstats;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -317,8 +447,13 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
-    if (kFused)
+    if (kFused) {
       for (int st = 0; st < C::kStages; ++st) mbar_init(&afull_bar[st], 128);  // the epilogue threads
+      // statistics exchange: every CTA of the cluster arrives once per row,
+      // then once for the max
+      mbar_init(&stat_bar[0], (uint32_t)(S * max(valid, 1)));
+      mbar_init(&stat_bar[1], (uint32_t)S);
+    }
     // one arrival per received row: S senders x my_n rows
     mbar_init(&recv_bar, kSplit && my_n > 0 ? (uint32_t)(S * my_n) : 1u);
     fence_mbar_init();
@@ -506,8 +641,11 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     // ------------------------------------------------------- epilogue ----
     const int sp = warp & 3;  // TMEM lane quarter this warp may access
     const int rl = sp * 32 + lane;
-    if (kFused) fused_prep<C>(args, smem, ks0, nks, valid, deadline, &abort_sh, empty_bar, afull_bar, inv_sh,
-                              wmax_sh, &sg_sh);
+    if (kFused && !fused_prep<C, kSplit>(args, smem, ks0, nks, valid, S, deadline, &abort_sh, empty_bar, afull_bar,
+                                         stat_bar, fstats)) {
+      record_error(args.err, kErrTimeout);
+      abort_sh = 1;
+    }
     const bool ok = mbar_wait(&acc_bar, 0, deadline, &abort_sh);
     tc_fence_after();
     grid_dependency_wait();  // s_g is written by the preceding sharq_prep
@@ -516,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       record_error(args.err, kErrTimeout);
       abort_sh = 1;
     } else if (!kSplit) {
-      const float scale = __fmul_rn(kFused ? sg_sh : *args.s_g, args.s_w[expert]);
+      const float scale = __fmul_rn(kFused ? fstats.s : *args.s_g, args.s_w[expert]);
       const int row = mt * 128 + rl;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
@@ -552,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   }
 
   if (threadIdx.x == 64) TRACE_POINT(6);
-  if (kFused) __syncthreads();  // sg_sh visible to every warp
+  if (kFused) __syncthreads();  // fstats.s visible to every warp
   if (kSplit && my_n > 0) {
     grid_dependency_wait();
     // ------------------------ owner: sum the S received slices in rank order
@@ -563,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     if (!ok) {
       if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
     } else {
-      const float scale = __fmul_rn(kFused ? sg_sh : *args.s_g, args.s_w[expert]);
+      const float scale = __fmul_rn(kFused ? fstats.s : *args.s_g, args.s_w[expert]);
       const float* recv = reinterpret_cast<const float*>(smem + C::kRingBytes);
       constexpr int q4 = BN / 4;
       for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
