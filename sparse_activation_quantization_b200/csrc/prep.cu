@@ -20,7 +20,7 @@
 // threads (adjacent lanes), reduced with warp shuffles.  The residual never
 // leaves registers; every output is stored in the MMA-ready tiled layout of
 // include/sharq.h.
-#include "quant.cuh"
+#include "strip.cuh"
 
 namespace sharq {
 
@@ -68,54 +68,143 @@ __device__ __forceinline__ float block_max_f(float v, float* sh) {
   return r;
 }
 
-constexpr int kStatsThreads = 256;
+constexpr int kRowThreads = 256;
+constexpr int kRowChunk = 8;  // 16-byte loads in flight per lane
 
-__global__ void __launch_bounds__(kStatsThreads) prep_stats_kernel(
+// bf16 (upper / lower half of a word) -> its value times 2^128 as a double,
+// by moving the exponent and mantissa fields (no conversion unit): exact for
+// normal numbers.  Zeros and subnormals come out as (1 + m/128) * 2^-127
+// (times 2^128) instead; see prep_rowstats_kernel for why that is harmless.
+__device__ __forceinline__ double bf16_hi_x2p128(uint32_t w) {
+  return __hiloint2double((int)(((w >> 3) & 0x0FFFE000u) | 0x40000000u), 0);
+}
+__device__ __forceinline__ double bf16_lo_x2p128(uint32_t w) {
+  return __hiloint2double((int)(((w << 13) & 0x0FFFE000u) | 0x40000000u), 0);
+}
+
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Wide form, first launch: one warp per row (rows strided over a grid that
+// fits the GPU), 8 loads of 16 bytes in flight per lane.
+//   RMSNorm rows: float64 sum of squares -> 1/rms, then max |Xn| (Xn
+//   recomputed from L1/L2 as in the quantizer: bf16(f32(f32(x/rms) g))).
+//   Rows without RMSNorm: max |x| on packed bf16 bits.
+// The device-wide max goes to gmax_bits[0] with one atomicMax per CTA.
+// Sum of squares: each square of a bf16 value is exact in float64, and the
+// values enter scaled by 2^128 (bf16_*_x2p128, squares scaled by 2^256,
+// undone exactly at the end).  A zero or subnormal element then adds at most
+// 2^-252 (unscaled) instead of its true square, i.e. at most K 2^-252 per
+// row -- far below one ulp of mean(x^2) + eps for any eps >= 2^-60, where
+// the result is that of an exact-input float64 sum in this lane order.  For
+// eps < 2^-60 (`exact`) the elements are converted exactly instead.
+template <bool kGamma>
+__global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
-    const int* __restrict__ row_index, int K, float* __restrict__ inv_rms,
+    const int* __restrict__ row_index, int T, int K, int exact, float* __restrict__ inv_rms,
     unsigned int* __restrict__ gmax_bits) {
-  __shared__ double sh_d[kStatsThreads / 32];
-  __shared__ float sh_f[kStatsThreads / 32];
-  const int t = blockIdx.x;
-  const int src = row_index ? row_index[t] : t;
-  const int nch = K >> 3;
-  float inv = 1.0f;
-  if (src < 0) {  // zero padding row: Xn = 0 contributes nothing to gmax
-    if (threadIdx.x == 0 && gamma) inv_rms[t] = (float)(1.0 / sqrt((double)eps));
-    else if (threadIdx.x == 0) inv_rms[t] = 1.0f;
-    return;
-  }
-  const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K);
-  const uint4* gr = reinterpret_cast<const uint4*>(gamma);
-  if (gamma) {
-    double ss = 0.0;
-    for (int c = threadIdx.x; c < nch; c += kStatsThreads) {
-      float f[8];
-      bf16x8_to_float(xr[c], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ss += (double)f[i] * (double)f[i];
+  __shared__ uint32_t wmax[kRowThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = gridDim.x * (kRowThreads / 32);
+  const int nv = K >> 3;  // 16-byte vectors per row
+  uint32_t mx = 0;        // max |Xn| so far: bf16 bit patterns, one per half
+  for (int t = blockIdx.x * (kRowThreads / 32) + warp; t < T; t += nw) {
+    const int src = row_index ? row_index[t] : t;  // warp-uniform
+    if (src < 0) {  // zero padding row of the grouped form: Xn = 0
+      if (lane == 0) inv_rms[t] = kGamma ? (float)(1.0 / sqrt((double)eps)) : 1.0f;
+      continue;
     }
-    ss = block_sum_d<kStatsThreads / 32>(ss, sh_d);
-    inv = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
-  }
-  float amax = 0.0f;
-  for (int c = threadIdx.x; c < nch; c += kStatsThreads) {
-    float f[8];
-    bf16x8_to_float(xr[c], f);
-    if (gamma) {
-      float g[8];
-      bf16x8_to_float(gr[c], g);
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K);
+    if (kGamma) {
+      double acc0 = 0.0, acc1 = 0.0;
+      for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunk) {
+        uint4 v[kRowChunk];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(norm_one(f[i], inv, g[i])));
+        for (int u = 0; u < kRowChunk; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+        if (!exact) {
+#pragma unroll
+          for (int u = 0; u < kRowChunk; ++u) {
+            if (c0 + 32 * u < nv) {
+              const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const double dl = bf16_lo_x2p128(w[i]), dh = bf16_hi_x2p128(w[i]);
+                acc0 = fma(dl, dl, acc0);
+                acc1 = fma(dh, dh, acc1);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < kRowChunk; ++u) {
+            float f[8];
+            bf16x8_to_float(v[u], f);  // zero-filled beyond the row: adds 0
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              acc0 = fma((double)f[e], (double)f[e], acc0);
+              acc1 = fma((double)f[e + 1], (double)f[e + 1], acc1);
+            }
+          }
+        }
+      }
+      double acc = acc0 + acc1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      const double ss = exact ? acc : acc * 0x1p-256;
+      const float inv = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
+      if (lane == 0) inv_rms[t] = inv;
+      const f2_t inv2 = f2_make(inv, inv);
+      const uint4* gr = reinterpret_cast<const uint4*>(gamma);
+      for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunk) {
+        uint4 v[kRowChunk], g[kRowChunk];
+#pragma unroll
+        for (int u = 0; u < kRowChunk; ++u) {
+          const bool in = c0 + 32 * u < nv;
+          v[u] = in ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+          g[u] = in ? gr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kRowChunk; ++u) {
+          const uint32_t xw[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          const uint32_t gw[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t n =
+                bf16x2_from_f2(f2_mul(f2_mul(f2_from_bf16x2(xw[i]), inv2), f2_from_bf16x2(gw[i])));
+            mx = vmax_u16x2(mx, n & 0x7FFF7FFFu);
+          }
+        }
+      }
     } else {
+      for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunk) {
+        uint4 v[kRowChunk];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        for (int u = 0; u < kRowChunk; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < kRowChunk; ++u) {
+          mx = vmax_u16x2(mx, v[u].x & 0x7FFF7FFFu);
+          mx = vmax_u16x2(mx, v[u].y & 0x7FFF7FFFu);
+          mx = vmax_u16x2(mx, v[u].z & 0x7FFF7FFFu);
+          mx = vmax_u16x2(mx, v[u].w & 0x7FFF7FFFu);
+        }
+      }
+      if (lane == 0) inv_rms[t] = 1.0f;
     }
   }
-  amax = block_max_f<kStatsThreads / 32>(amax, sh_f);
+  // CTA max -> device-wide max (non-negative floats order as their bits)
+  uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) wmax[warp] = m;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    inv_rms[t] = inv;
-    atomicMax(gmax_bits, __float_as_uint(amax));  // non-negative floats order as uints
+    uint32_t cm = 0;
+#pragma unroll
+    for (int w = 0; w < kRowThreads / 32; ++w) cm = max(cm, wmax[w]);
+    if (cm) atomicMax(gmax_bits, cm << 16);
   }
 }
 
@@ -137,34 +226,93 @@ __device__ __forceinline__ void depart_and_reset(unsigned int* sync) {
   }
 }
 
-constexpr int kQuantThreads = 256;
+constexpr int kStripThreads = 256;
 
-// Two-launch form, second launch: one thread per 32 consecutive K (four runs
-// of 8; every quantization block inside the thread), flat over rows.
-template <bool kSharq>
-__global__ void __launch_bounds__(kQuantThreads) prep_quant_kernel(
+// Wide form, second launch: one thread per 32-K strip of a row.  Warp w of
+// the grid owns strip group w % G (32 adjacent strips = 2 KB of a row, G
+// groups per row) and walks the rows w / G, w / G + nw / G, ... (nw, the
+// warps used, is a multiple of G), so its lanes load and unpack gamma once
+// and prefetch the next row's 64 bytes while quantizing the current one.
+template <bool kSharq, bool kGamma>
+__global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
-    const int* __restrict__ row_index, int T, int Tp, int K, const float* __restrict__ inv_rms,
-    const unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
-  __shared__ float gmax_sh;
+    const int* __restrict__ row_index, int T, int K, int nw, const float* __restrict__ inv_rms,
+    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
+  __shared__ float2 tab[128];
+  __shared__ uint32_t msel[16];
   allow_dependents();
-  const int segs = K >> 5;
-  const long long gid = (long long)blockIdx.x * kQuantThreads + threadIdx.x;
-  if (threadIdx.x == 0) gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
-  __syncthreads();
-  const float gmax = gmax_sh;
+  const float gmax = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
-  if (gid == 0) *s_g_out = s;  // published even when there are no rows
-  if (gid < (long long)T * segs) {
-    const int t = (int)(gid / segs);
-    const int c0 = (int)(gid - (long long)t * segs) * 4;
-    const int src = row_index ? row_index[t] : t;
-    float x[32];
-    load_runs<4>(x, X, src, K, c0);
-    if (gamma && src >= 0) normalise_runs<4>(x, gamma, c0, inv_rms[t]);
-    quant_runs<4, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;  // published even when there are no rows
+  strip_tables_init(s, tab, msel);
+  __syncthreads();
+  const StripCtx ctx = strip_ctx(s, tab, msel);
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (kStripThreads / 32) + (threadIdx.x >> 5);
+  const int nstrips = K >> 5, G = (nstrips + 31) >> 5, KS = K >> 8;
+  if (gw < nw && T > 0) {
+    const int j = (gw % G) * 32 + lane;
+    const bool active = j < nstrips;
+    const int rstride = nw / G;
+    f2_t gm[16];
+    if (kGamma && active) {
+      const uint4* gp = reinterpret_cast<const uint4*>(gamma + 32 * (size_t)j);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint4 v = gp[u];
+        gm[4 * u] = f2_from_bf16x2(v.x);
+        gm[4 * u + 1] = f2_from_bf16x2(v.y);
+        gm[4 * u + 2] = f2_from_bf16x2(v.z);
+        gm[4 * u + 3] = f2_from_bf16x2(v.w);
+      }
+    }
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    int t = gw / G;  // < T: the host uses at most T warps per strip group
+    int src = row_index ? row_index[t] : t;
+    uint4 cur[4];
+    float inv = 1.0f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      cur[u] = (active && src >= 0) ? reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * (size_t)j)[u] : z4;
+    if (kGamma) inv = inv_rms[t];
+    while (t < T) {
+      // prefetch the next row of this warp
+      const int tn = t + rstride;
+      int srcn = -1;
+      uint4 nxt[4] = {z4, z4, z4, z4};
+      float invn = 1.0f;
+      if (tn < T) {
+        srcn = row_index ? row_index[tn] : tn;
+        if (active && srcn >= 0) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) nxt[u] = reinterpret_cast<const uint4*>(X + (size_t)srcn * K + 32 * (size_t)j)[u];
+        }
+        if (kGamma) invn = inv_rms[tn];
+      }
+      if (active) {
+        f2_t P[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          P[4 * u] = f2_from_bf16x2(cur[u].x);
+          P[4 * u + 1] = f2_from_bf16x2(cur[u].y);
+          P[4 * u + 2] = f2_from_bf16x2(cur[u].z);
+          P[4 * u + 3] = f2_from_bf16x2(cur[u].w);
+        }
+        if (kGamma && src >= 0) {
+          const f2_t inv2 = f2_make(inv, inv);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) P[i] = f2_norm(P[i], inv2, gm[i]);
+        }
+        quant_strip<kSharq>(P, t, j, KS, ctx, out);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
+      src = srcn;
+      inv = invn;
+      t = tn;
+    }
   }
-  if (threadIdx.x == 0) depart_and_reset(const_cast<unsigned int*>(gmax_bits));
+  if (threadIdx.x == 0) depart_and_reset(gmax_bits);
 }
 
 // ---------------------------------------------------------------------------
@@ -361,6 +509,29 @@ cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, floa
   }
 }
 
+// CTAs of `fn` resident per SM at `threads` threads (cached per device and
+// kernel); the maximum shared-memory carveout is requested first so that an
+// SM running them keeps room for a GEMM CTA launched as their dependent.
+template <class F>
+int resident_ctas(F* fn, int threads, int dev) {
+  static F* fns[16] = {};
+  static int cache[16][64] = {};
+  int slot = 0;
+  while (slot < 16 && fns[slot] && fns[slot] != fn) ++slot;
+  if (slot == 16) return 1;
+  if (!fns[slot]) fns[slot] = fn;
+  if (cache[slot][dev] == 0) {
+    prefer_max_shared(fn);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, 0) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = 1;
+    }
+    cache[slot][dev] = n;
+  }
+  return cache[slot][dev];
+}
+
 }  // namespace
 
 #ifdef SHARQ_TRACE
@@ -390,25 +561,36 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
     if (launched) return cudaSuccess;
   }
 
-  static bool carveout_set[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !carveout_set[dev]) {
-    prefer_max_shared(prep_quant_kernel<true>);
-    prefer_max_shared(prep_quant_kernel<false>);
-    carveout_set[dev] = true;
-  }
+  // wide form: row statistics, then the strip quantizer
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const bool g = Gb != nullptr;
+  const int exact = eps < 0x1p-60f ? 1 : 0;
   if (T > 0) {
-    prep_stats_kernel<<<T, kStatsThreads, 0, stream>>>(Xb, Gb, eps, row_index, K, inv_rms, gmax_bits);
+    const int per_sm = g ? resident_ctas(prep_rowstats_kernel<true>, kRowThreads, dev)
+                         : resident_ctas(prep_rowstats_kernel<false>, kRowThreads, dev);
+    const int rows_per_cta = kRowThreads / 32;
+    int grid = (T + rows_per_cta - 1) / rows_per_cta;
+    if (grid > sms * per_sm) grid = sms * per_sm;
+    if (g)
+      prep_rowstats_kernel<true><<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms,
+                                                                   gmax_bits);
+    else
+      prep_rowstats_kernel<false><<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms,
+                                                                    gmax_bits);
   }
-  const long long n = (long long)T * (K >> 5);
-  // at least one block so that s_g is published (= 1) even for T == 0
-  const unsigned grid = n > 0 ? (unsigned)((n + kQuantThreads - 1) / kQuantThreads) : 1u;
-  if (sharq_mode)
-    prep_quant_kernel<true><<<grid, kQuantThreads, 0, stream>>>(Xb, Gb, row_index, T, Tp, K, inv_rms, gmax_bits,
-                                                                 s_g, p);
-  else
-    prep_quant_kernel<false><<<grid, kQuantThreads, 0, stream>>>(Xb, Gb, row_index, T, Tp, K, inv_rms,
-                                                                  gmax_bits, s_g, p);
+  auto strip_fn = sharq_mode ? (g ? prep_strip_kernel<true, true> : prep_strip_kernel<true, false>)
+                             : (g ? prep_strip_kernel<false, true> : prep_strip_kernel<false, false>);
+  const int G = ((K >> 5) + 31) >> 5;  // strip groups (warps) per row
+  const int max_warps = sms * resident_ctas(strip_fn, kStripThreads, dev) * (kStripThreads / 32);
+  long long rows = max_warps / G;
+  if (rows < 1) rows = 1;
+  if (rows > T) rows = T;
+  const int nw = (int)(rows * G);  // 0 when T == 0: one CTA still publishes s_g
+  const int grid = nw > 0 ? (nw + kStripThreads / 32 - 1) / (kStripThreads / 32) : 1;
+  strip_fn<<<grid, kStripThreads, 0, stream>>>(Xb, Gb, row_index, T, K, nw, inv_rms, gmax_bits, s_g, p);
   return cudaGetLastError();
 }
 
