@@ -179,6 +179,27 @@ __device__ __forceinline__ void store4(void* Y, int out_f32, size_t off, float4 
   }
 }
 
+// Expert that owns m-tile mt in the grouped form (offsets are 128-row
+// aligned), 0 without groups, -1 if the offsets do not cover the tile.
+__device__ __forceinline__ int tile_expert(const GemmArgs& args, int mt) {
+  if (!args.group_offsets) return 0;
+  const int row0 = mt * 128;
+  int e = -1;
+  int lo = 0, hi = args.E - 1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    if (args.group_offsets[mid] <= row0) {
+      e = mid;
+      lo = mid + 1;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  while (e >= 0 && e < args.E && args.group_offsets[e + 1] <= row0) ++e;
+  if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
+  return e;
+}
+
 // Programmatic dependent launch: wait until the preceding grid in the stream
 // has completed and its memory is visible (returns at once if there is none).
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -458,20 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     mbar_init(&recv_bar, kSplit && my_n > 0 ? (uint32_t)(S * my_n) : 1u);
     fence_mbar_init();
     abort_sh = 0;
-    // expert of this m-tile (grouped form): offsets are 128-row aligned
-    int e = 0;
-    if (args.group_offsets) {
-      const int row0 = mt * 128;
-      e = -1;
-      int lo = 0, hi = args.E - 1;
-      while (lo <= hi) {
-        const int mid = (lo + hi) >> 1;
-        if (args.group_offsets[mid] <= row0) { e = mid; lo = mid + 1; } else { hi = mid - 1; }
-      }
-      while (e >= 0 && e < args.E && args.group_offsets[e + 1] <= row0) ++e;
-      if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
-    }
-    expert_sh = e;
+    expert_sh = tile_expert(args, mt);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, C::kTmemCols);
@@ -729,6 +737,273 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent form (no split-K, activation already prepared: prefill and the
+// grouped expert shapes).  One CTA per SM walks the output tiles t =
+// blockIdx.x, blockIdx.x + gridDim.x, ... (row-major over (m-tile, n-tile),
+// so CTAs running at the same time share activation tiles in L2).  The
+// shared-memory ring and its phases run on across tiles, so the producer
+// streams the next tile's stages while the current one finishes, and the
+// accumulator is handed back to the MMA warp as soon as the epilogue has
+// moved it into registers (bf16 output: the tile's row in 128 packed
+// registers per thread) -- the global stores of tile k overlap the MMAs of
+// tile k + 1.  Set-up (barriers, TMEM allocation) is paid once per SM.
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(const GemmArgs args, int m_tiles) {
+  using C = Cfg<BN, false>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::kStages];
+  __shared__ __align__(8) uint64_t empty_bar[C::kStages];
+  __shared__ __align__(8) uint64_t acc_full;
+  __shared__ __align__(8) uint64_t acc_empty;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KS = args.K >> 8;
+  const int NB = args.D >> 7;
+  const int n_tiles = args.D / BN;
+  const int ntiles = m_tiles * n_tiles;
+  const bool sharq = args.sharq_mode != 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, 128);  // every epilogue thread, once per tile
+    fence_mbar_init();
+    abort_sh = 0;
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (sharq) {
+    // Metadata rows past a partial tile's valid rows are never copied in: give
+    // every row a valid pattern (pairs 0 and 1) once; later tiles leave
+    // metadata written by sharq_prep there, which is valid as well.
+    for (int idx = threadIdx.x; idx < C::kStages * 128; idx += kThreads) {
+      const int st = idx >> 7, row = idx & 127;
+      *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE + row * 16) =
+          make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- producer ----
+    if (lane == 0) {
+      grid_dependency_wait();  // the activation comes from the preceding sharq_prep
+      if (blockIdx.x == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
+      uint32_t g = 0;  // stage counter across tiles
+      for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
+        const int mt = tile / n_tiles, nt = tile - mt * n_tiles;
+        const int expert = tile_expert(args, mt);
+        if (expert < 0) {
+          if (nt == 0) record_error(args.err, kErrInvalid);
+          continue;
+        }
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        const int valid = min(128, args.T - mt * 128);
+        const uint32_t a_rows = (uint32_t)valid;
+        const uint32_t tx = (sharq ? C::kTxSharq : C::kTxNvfp4) - (128u - a_rows) * (sharq ? 208u : 128u);
+        const size_t a_tile0 = (size_t)mt * KS;
+        const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages;
+          if (g >= (uint32_t)C::kStages &&
+              !mbar_wait(&empty_bar[s], ((g / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          uint8_t* st = smem + s * C::kStageBytes;
+          mbar_arrive_expect_tx(&full_bar[s], tx);
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            const size_t bt = b_tile0 + (size_t)h * KS + i;
+            bulk_g2s(st + C::kOffB + h * kCodesTile, args.w_codes + bt * kCodesTile, kCodesTile, &full_bar[s]);
+            bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, &full_bar[s]);
+            if (sharq)
+              bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, &full_bar[s]);
+          }
+          const size_t at = a_tile0 + i;
+          bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, a_rows * 128u, &full_bar[s]);
+          bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, &full_bar[s]);
+          if (sharq) {
+            bulk_g2s(st + C::kOffASP, args.a_sp + at * kSpTile, a_rows * 64u, &full_bar[s]);
+            bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, a_rows * 16u, &full_bar[s]);
+            bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, &full_bar[s]);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_dn = idesc_nvf4(128, BN, false);
+      constexpr uint32_t idesc_sp = idesc_nvf4(128, BN, true);
+      uint32_t g = 0, k = 0;  // stage counter, tiles done
+      for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
+        if (tile_expert(args, tile / n_tiles) < 0) continue;
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        // the epilogue has taken the previous tile's accumulator
+        if (k > 0 && !mbar_wait(&acc_empty, (k - 1) & 1, deadline, &abort_sh)) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        tc_fence_after();
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages;
+          if (!mbar_wait(&full_bar[s], (g / C::kStages) & 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t sf = tmem + C::kColSf0 + (g & 1u) * C::kSfRegion;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
+                               smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+          if (sharq) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h)
+                tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
+                                 smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
+            tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffASP + 32 * j, 16, 512, kSw64),
+                          smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + C::kSfE + 2 * j, idesc_sp,
+                          sf + C::kSfASP + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, (i > 0 || j > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffAR + 32 * j, 16, 1024, kSw128),
+                     smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + C::kSfAR + 4 * j,
+                     sf + C::kSfB16 + j * C::kSfbCols, (sharq || i > 0 || j > 0) ? 1u : 0u);
+          tc_commit(&empty_bar[s]);
+        }
+        tc_commit(&acc_full);  // accumulator of this tile complete
+        ++k;
+      }
+    }
+  } else {
+    // ------------------------------------------------------- epilogue ----
+    const int sp = warp & 3;  // TMEM lane quarter this warp may access
+    const int rl = sp * 32 + lane;
+    grid_dependency_wait();  // s_g is written by the preceding sharq_prep
+    const float s_g = *args.s_g;
+    uint32_t k = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
+      const int mt = tile / n_tiles, nt = tile - mt * n_tiles;
+      const int expert = tile_expert(args, mt);
+      if (expert < 0) continue;
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+      if (!mbar_wait(&acc_full, k & 1, deadline, &abort_sh)) {
+        record_error(args.err, kErrTimeout);
+        abort_sh = 1;
+        break;
+      }
+      tc_fence_after();
+      const float scale = __fmul_rn(s_g, args.s_w[expert]);
+      const int valid = min(128, args.T - mt * 128);
+      const size_t off = (size_t)(mt * 128 + rl) * args.D + (size_t)nt * BN;
+      if (!args.out_f32) {
+        uint32_t pk[BN / 2];  // the row as packed bf16, then the accumulator is free
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * q]), scale),
+                                                      __fmul_rn(__uint_as_float(v[2 * q + 1]), scale));
+            pk[c / 2 + q] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive_local(&acc_empty);
+        if (rl < valid) {
+          uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off);
+#pragma unroll
+          for (int q = 0; q < BN / 8; ++q) y[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+          tmem_ld_wait();
+          if (rl < valid) store_row32(args.Y, 1, off + c, v, scale);
+        }
+        tc_fence_before();
+        mbar_arrive_local(&acc_empty);
+      }
+      ++k;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN>
+cudaError_t launch_persistent(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
+  using C = Cfg<BN, false>;
+  static int sms[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (sms[dev] == 0) {
+    e = cudaFuncSetAttribute(sharq_gemm_persistent_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    sms[dev] = n;
+  }
+  const long long ntiles = (long long)m_tiles * (a.D / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(ntiles < sms[dev] ? ntiles : sms[dev]));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sharq_gemm_persistent_kernel<BN>, a, m_tiles);
+}
+
 template <int BN, bool kSplit, bool kFused>
 cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   using C = Cfg<BN, kSplit>;
@@ -813,8 +1088,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
     if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
     return launch_cfg<128, true, false>(a, m_tiles, stream);
   }
-  return bn == 256 ? launch_cfg<256, false, false>(a, m_tiles, stream)
-                   : launch_cfg<128, false, false>(a, m_tiles, stream);
+  return bn == 256 ? launch_persistent<256>(a, m_tiles, stream) : launch_persistent<128>(a, m_tiles, stream);
 }
 
 }  // namespace sharq
