@@ -871,37 +871,33 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
           tc_fence_after();
           const uint32_t st = smem_u32(smem + s * C::kStageBytes);
           const uint32_t sf = tmem + C::kColSf0 + (g & 1u) * C::kSfRegion;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int h = 0; h < C::kHalves; ++h)
-              tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
-                               smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+          // each MMA's scale copies right before it: the copies for MMA j + 1
+          // can run while MMA j computes
           if (sharq) {
+            tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int j = 0; j < 2; ++j) {
+              tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
 #pragma unroll
               for (int h = 0; h < C::kHalves; ++h)
                 tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
                                  smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
-            tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-              tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
               mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffASP + 32 * j, 16, 512, kSw64),
                           smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + C::kSfE + 2 * j, idesc_sp,
                           sf + C::kSfASP + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, (i > 0 || j > 0) ? 1u : 0u);
+            }
           }
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < 4; ++j) {
+            tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
+                               smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
             mma_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffAR + 32 * j, 16, 1024, kSw128),
                      smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + C::kSfAR + 4 * j,
                      sf + C::kSfB16 + j * C::kSfbCols, (sharq || i > 0 || j > 0) ? 1u : 0u);
+          }
           tc_commit(&empty_bar[s]);
         }
         tc_commit(&acc_full);  // accumulator of this tile complete
