@@ -216,7 +216,40 @@ def linear(p, wq):
     w16 = (e2m1_decode(wq["codes"]).reshape(D, K // 16, 16)
            * e4m3_decode(wq["sf16"])[..., None]).reshape(D, K).T
     y = a_sp @ w32 + a_dn @ w16
-    return y * (np.float64(p["s_g"]) * np.float64(wq["s_w"]))
+    return y * (_row_scale(p["s_g"], y.shape[0]) * np.float64(wq["s_w"]))
+
+
+def _row_scale(s_g, T):
+    """The global activation scale as a float64 column: one value for the
+    per-tensor scale, one per row for the per-token reading."""
+    s = np.asarray(s_g, dtype=np.float64)
+    return s if s.ndim == 0 else s.reshape(T, 1)
+
+
+def prep_per_token(x, gamma=None, eps=1e-5):
+    """SharQ preparation with the global scale read as per-TOKEN (the
+    alternative expansion of "PTS", xllm-io review, sections 3.1 and 3.5): every
+    row gets its own s_t = max|Xn[t]| / (6*448) (1 for an all-zero row), and
+    each row is prepared exactly as the per-tensor prep() of that row alone
+    with s_g = s_t.  Both activation paths of a row share s_t, so the two
+    MMAs still add into one accumulator row.  Returns the prep() dict with
+    s_g (and gmax) as float32 arrays [T]."""
+    x = np.asarray(x, dtype=np.float32)
+    T = x.shape[0]
+    xn, _ = rmsnorm(x, gamma, eps)
+    scales = [pts_scale(xn[t:t + 1]) for t in range(T)]
+    rows = [prep(x[t:t + 1], gamma, eps, s_g=scales[t][0]) for t in range(T)]
+    out = {}
+    for k, v in prep(x[:1] if T else x, gamma, eps).items():
+        if k == "s_g":
+            out[k] = np.array([sc[0] for sc in scales], np.float32)
+        elif k == "gmax":
+            out[k] = np.array([sc[1] for sc in scales], np.float32)
+        elif v is None or not T:
+            out[k] = v
+        else:
+            out[k] = np.concatenate([r[k] for r in rows], axis=0)
+    return out
 
 
 def epilogue_f32(y64, s_g, s_w):
@@ -270,4 +303,4 @@ def linear_nvfp4(p, wq):
     D = wq["w_t"].shape[1]
     w16 = (e2m1_decode(wq["codes"]).reshape(D, K // 16, 16)
            * e4m3_decode(wq["sf16"])[..., None]).reshape(D, K).T
-    return (a @ w16) * (np.float64(p["s_g"]) * np.float64(wq["s_w"]))
+    return (a @ w16) * (_row_scale(p["s_g"], a.shape[0]) * np.float64(wq["s_w"]))
