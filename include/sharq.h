@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define SHARQ_ABI_VERSION 1
+#define SHARQ_ABI_VERSION 2
 
 typedef struct CUstream_st *sharq_stream_t; /* same type as cudaStream_t */
 
@@ -65,8 +65,13 @@ enum { SHARQ_OUT_BF16 = 0, SHARQ_OUT_F32 = 1 };
 /* Activation path.  SHARQ: sparse backbone + dense residual (the method).
  * NVFP4: plain NVFP4 of Xn (16-element blocks, same PTS scale) and a dense
  * FP4 GEMM only -- the "NVFP4" comparator of the xllm-io review's Table 1 and
- * the official repository's NVFP4 mode (kasblo.com explainer). */
-enum { SHARQ_MODE_SHARQ = 0, SHARQ_MODE_NVFP4 = 1 };
+ * the official repository's NVFP4 mode (kasblo.com explainer).
+ * SHARQ_TOKEN: the SharQ path with the global activation scale read as
+ * per-TOKEN rather than per-tensor (the pages never expand "PTS", xllm-io
+ * review, sections 3.1 and 3.5): row t gets s_t = max|Xn[t]| / (6*448) and is
+ * prepared exactly as a one-row tensor; no device-wide reduction.  Its codes
+ * are not those of the per-tensor mode.  Supported for K <= 20480. */
+enum { SHARQ_MODE_SHARQ = 0, SHARQ_MODE_NVFP4 = 1, SHARQ_MODE_SHARQ_TOKEN = 2 };
 
 /* Tile geometry of every packed operand: 128 rows x 256 logical K. */
 #define SHARQ_TILE_ROWS 128
@@ -105,21 +110,23 @@ typedef struct {
  *   r_codes: 16384-byte tiles, 128-byte lines, 128-byte swizzle (as weight
  *            codes).  SHARQ: residual codes.  NVFP4: codes of Xn.
  *   r_sf:    2048-byte tiles, one scale per 16 K (as weight sf16).
- *   sp_codes (SHARQ only): 8192-byte tiles; row r is the 64-byte line at
+ *   sp_codes (SHARQ, SHARQ_TOKEN): 8192-byte tiles; row r is the 64-byte line at
  *            r*64 holding the 128 kept values of its 256 logical K in
  *            ascending K order, byte j/2 for kept value j; 16-byte chunks
  *            permuted by chunk ^= (r/2) % 4 (64-byte swizzle).
- *   meta (SHARQ only): 2048-byte tiles, row r at r*16; chunk of 8 logical K
+ *   meta (SHARQ, SHARQ_TOKEN): 2048-byte tiles, row r at r*16; chunk of 8 logical K
  *            g = c/8 in byte g/2 (low nibble = lower chunk); nibble =
  *            p_lo | p_hi << 2, the kept pair indices, p_lo < p_hi.
- *   sp_sf (SHARQ only): 1024-byte tiles, one scale per 32 logical K (16 kept
+ *   sp_sf (SHARQ, SHARQ_TOKEN): 1024-byte tiles, one scale per 32 logical K (16 kept
  *            values), atom layout as weight sf32.
  *   inv_rms: Tp floats (1/rms per row; 1 when RMSNorm is off).
- *   s_g:     the per-tensor global scale gmax / (6*448) (1 if gmax == 0).
+ *   s_g:     the per-tensor global scale gmax / (6*448) (1 if gmax == 0);
+ *            SHARQ_TOKEN: Tp floats, s_t of row t (rows >= T unused).
  *   gmax_bits: 16 bytes of scratch: device-wide amax, grid-barrier count,
  *            departure count, and an error word that sharq_linear forwards
  *            to its workspace (a prep whose grid barrier timed out).
- *   The 256-byte scalar block that starts at s_g (s_g, gmax_bits[0..3])
+ *   The 256-byte scalar block that holds gmax_bits (and s_g outside
+ *   SHARQ_TOKEN)
  *   must be zero before the first sharq_prep on a buffer (zero the whole
  *   buffer once after allocation); sharq_prep leaves gmax_bits[0..2] zero
  *   again, so no per-call memset is needed.

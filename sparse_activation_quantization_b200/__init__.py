@@ -15,7 +15,7 @@ import os
 
 __all__ = [
     "SharqError", "SharqAct", "SharqWeight", "lib", "library_path",
-    "SHARQ_MODE_SHARQ", "SHARQ_MODE_NVFP4", "SHARQ_OUT_BF16", "SHARQ_OUT_F32",
+    "SHARQ_MODE_SHARQ", "SHARQ_MODE_NVFP4", "SHARQ_MODE_SHARQ_TOKEN", "SHARQ_OUT_BF16", "SHARQ_OUT_F32",
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes",
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
@@ -25,6 +25,7 @@ __all__ = [
 
 SHARQ_MODE_SHARQ = 0
 SHARQ_MODE_NVFP4 = 1
+SHARQ_MODE_SHARQ_TOKEN = 2
 SHARQ_OUT_BF16 = 0
 SHARQ_OUT_F32 = 1
 
@@ -221,9 +222,11 @@ class PreparedAct:
         self.reset()
 
     def reset(self):
-        """Zero the scalar block (s_g and the prep's sync words), as the C ABI
-        requires before the first sharq_prep on a buffer."""
-        self.region("s_g", 256).zero_()
+        """Zero the 256-byte scalar block (the prep's sync words, and s_g
+        outside the per-token mode), as the C ABI requires before the first
+        sharq_prep on a buffer."""
+        off = self.view.gmax_bits - 16 - self.buf.data_ptr()
+        self.buf[off:off + 256].zero_()
 
     def prep(self, X, gamma=None, eps=1e-5, row_index=None, stream=None):
         sharq_prep(X.data_ptr() if X is not None else None,

@@ -11,7 +11,8 @@
 
 namespace sharq {
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp, int K,
-                        bool sharq_mode, float* inv_rms, float* s_g, unsigned int* gmax_bits, uint8_t* sp_codes,
+                        bool sharq_mode, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
+                        uint8_t* sp_codes,
                         uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, cudaStream_t stream);
 cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf32, uint8_t* sf16,
                                float* s_w, unsigned int* amax_bits, cudaStream_t stream);
@@ -20,10 +21,11 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
                           int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
-                          const void* gamma_fused, float eps_fused);
+                          const void* gamma_fused, float eps_fused, bool per_token);
 int noalloc_max_rows();
+bool prep_per_token_supported(int K);
 cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
-                                int K, bool sharq_mode, float* s_g, uint8_t* sp_codes, uint8_t* meta,
+                                int K, bool sharq_mode, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
                                 uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, unsigned int* err_out,
                                 cudaStream_t stream);
 }  // namespace sharq
@@ -45,9 +47,14 @@ bool shape_ok_d(int D) { return D > 0 && D <= kMaxD && D % 128 == 0; }
 bool shape_ok_t(int T) { return T >= 0 && T <= kMaxT; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+bool mode_ok(int mode) {
+  return mode == SHARQ_MODE_SHARQ || mode == SHARQ_MODE_NVFP4 || mode == SHARQ_MODE_SHARQ_TOKEN;
+}
+bool has_sparse(int mode) { return mode != SHARQ_MODE_NVFP4; }
+
 // layout sizes, shared by the *_bytes and *_view functions
 struct ActLayout {
-  size_t r_codes, r_sf, sp_codes, meta, sp_sf, inv, scal, total;
+  size_t r_codes, r_sf, sp_codes, meta, sp_sf, inv, s_tok, scal, total;
 };
 ActLayout act_layout(int T, int K, int mode) {
   ActLayout L{};
@@ -57,12 +64,14 @@ ActLayout act_layout(int T, int K, int mode) {
   L.r_codes = off; off += tiles * sharq::kCodesTile;
   L.r_sf = off;    off += tiles * sharq::kSf16Tile;
   L.sp_codes = off;
-  if (mode == SHARQ_MODE_SHARQ) off += tiles * sharq::kSpTile;
+  if (has_sparse(mode)) off += tiles * sharq::kSpTile;
   L.meta = off;
-  if (mode == SHARQ_MODE_SHARQ) off += tiles * sharq::kMetaTile;
+  if (has_sparse(mode)) off += tiles * sharq::kMetaTile;
   L.sp_sf = off;
-  if (mode == SHARQ_MODE_SHARQ) off += tiles * sharq::kSf32Tile;
+  if (has_sparse(mode)) off += tiles * sharq::kSf32Tile;
   L.inv = off;     off = round_up(off + Tp * sizeof(float), kAlign);
+  L.s_tok = off;   // per-token scales (SHARQ_TOKEN only)
+  if (mode == SHARQ_MODE_SHARQ_TOKEN) off = round_up(off + Tp * sizeof(float), kAlign);
   L.scal = off;    off += kAlign;  // s_g, gmax_bits
   L.total = off;
   return L;
@@ -132,10 +141,10 @@ int check_device() {
 int act_ok(const sharq_act* a) {
   if (!a) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(a->T) || !shape_ok_k(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
-  if (a->mode != SHARQ_MODE_SHARQ && a->mode != SHARQ_MODE_NVFP4) return SHARQ_ERR_INVALID_ARG;
+  if (!mode_ok(a->mode)) return SHARQ_ERR_INVALID_ARG;
   if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
   if (!a->r_codes || !a->r_sf || !a->inv_rms || !a->s_g || !a->gmax_bits) return SHARQ_ERR_INVALID_ARG;
-  if (a->mode == SHARQ_MODE_SHARQ && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  if (has_sparse(a->mode) && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
   const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf};
   for (const void* q : p)
     if (q && !aligned(q, 16)) return SHARQ_ERR_INVALID_ARG;
@@ -167,12 +176,12 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
   cudaError_t e = sharq::launch_linear(
       static_cast<const uint8_t*>(a->sp_codes), static_cast<const uint8_t*>(a->meta),
       static_cast<const uint8_t*>(a->sp_sf), static_cast<const uint8_t*>(a->r_codes),
-      static_cast<const uint8_t*>(a->r_sf), a->s_g, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ ? 1 : 0,
+      static_cast<const uint8_t*>(a->r_sf), a->s_g, a->T, a->Tp, a->K, has_sparse(a->mode) ? 1 : 0,
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
       out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, static_cast<int*>(d_ws),
       reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr,
-      0.0f);
+      0.0f, a->mode == SHARQ_MODE_SHARQ_TOKEN);
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 
@@ -202,7 +211,7 @@ size_t sharq_weight_bytes(int K, int D, int E) {
 
 size_t sharq_act_bytes(int T, int K, int mode) {
   if (!shape_ok_t(T) || !shape_ok_k(K)) return 0;
-  if (mode != SHARQ_MODE_SHARQ && mode != SHARQ_MODE_NVFP4) return 0;
+  if (!mode_ok(mode)) return 0;
   return act_layout(T, K, mode).total;
 }
 
@@ -230,18 +239,18 @@ int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {
 int sharq_act_view(void* d_buf, int T, int K, int mode, sharq_act* out) {
   if (!d_buf || !out) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(T) || !shape_ok_k(K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
-  if (mode != SHARQ_MODE_SHARQ && mode != SHARQ_MODE_NVFP4) return SHARQ_ERR_INVALID_ARG;
+  if (!mode_ok(mode)) return SHARQ_ERR_INVALID_ARG;
   if (!aligned(d_buf, kAlign)) return SHARQ_ERR_INVALID_ARG;
   const ActLayout L = act_layout(T, K, mode);
   uint8_t* b = static_cast<uint8_t*>(d_buf);
-  const bool sq = mode == SHARQ_MODE_SHARQ;
+  const bool sq = has_sparse(mode);
   out->r_codes = b + L.r_codes;
   out->r_sf = b + L.r_sf;
   out->sp_codes = sq ? b + L.sp_codes : nullptr;
   out->meta = sq ? b + L.meta : nullptr;
   out->sp_sf = sq ? b + L.sp_sf : nullptr;
   out->inv_rms = reinterpret_cast<float*>(b + L.inv);
-  out->s_g = reinterpret_cast<float*>(b + L.scal);
+  out->s_g = reinterpret_cast<float*>(b + (mode == SHARQ_MODE_SHARQ_TOKEN ? L.s_tok : L.scal));
   out->gmax_bits = reinterpret_cast<unsigned int*>(b + L.scal + 16);
   out->T = T;
   out->Tp = (int)round_up((size_t)T, 128);
@@ -270,9 +279,11 @@ int sharq_prep(const void* d_X, const void* d_gamma, float eps, const int* d_row
   if (a->T > 0 && (!d_X || !aligned(d_X, 16))) return SHARQ_ERR_INVALID_ARG;
   if (d_gamma && !aligned(d_gamma, 16)) return SHARQ_ERR_INVALID_ARG;
   if (!(eps >= 0.0f)) return SHARQ_ERR_INVALID_ARG;
+  const bool per_token = a->mode == SHARQ_MODE_SHARQ_TOKEN;
+  if (per_token && !sharq::prep_per_token_supported(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if ((st = check_device())) return st;
   cudaError_t e = sharq::launch_prep(
-      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ, a->inv_rms, a->s_g,
+      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, has_sparse(a->mode), per_token, a->inv_rms, a->s_g,
       a->gmax_bits, static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta),
       static_cast<uint8_t*>(a->sp_sf), static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf),
       reinterpret_cast<cudaStream_t>(stream));
@@ -284,10 +295,11 @@ int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const in
   if (!a) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(a->T) || !shape_ok_k(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if (a->T > sharq::noalloc_max_rows()) return SHARQ_ERR_UNSUPPORTED_SHAPE;
-  if (a->mode != SHARQ_MODE_SHARQ && a->mode != SHARQ_MODE_NVFP4) return SHARQ_ERR_INVALID_ARG;
+  if (!mode_ok(a->mode)) return SHARQ_ERR_INVALID_ARG;
   if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
   if (!a->r_codes || !a->r_sf || !a->s_g) return SHARQ_ERR_INVALID_ARG;
-  if (a->mode == SHARQ_MODE_SHARQ && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  if (has_sparse(a->mode) && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  if (a->mode == SHARQ_MODE_SHARQ_TOKEN && !sharq::prep_per_token_supported(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf};
   for (const void* q : p)
     if (q && !aligned(q, 16)) return SHARQ_ERR_INVALID_ARG;
@@ -297,7 +309,8 @@ int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const in
   int st = check_device();
   if (st) return st;
   cudaError_t e = sharq::launch_prep_noalloc(
-      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, a->mode == SHARQ_MODE_SHARQ, a->s_g,
+      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, has_sparse(a->mode), a->mode == SHARQ_MODE_SHARQ_TOKEN,
+      a->s_g,
       static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta), static_cast<uint8_t*>(a->sp_sf),
       static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf), a->gmax_bits ? a->gmax_bits + 3 : nullptr,
       reinterpret_cast<cudaStream_t>(stream));
@@ -312,7 +325,7 @@ int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, co
   if (w->E != 1) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(T)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if (T > SHARQ_FUSED_MAX_T) {  // larger batches: the two-call path through `a`
-    if (!a || a->T != T || a->K != w->K || a->mode != SHARQ_MODE_SHARQ) return SHARQ_ERR_INVALID_ARG;
+    if (!a || a->T != T || a->K != w->K || !has_sparse(a->mode)) return SHARQ_ERR_INVALID_ARG;
     if ((st = sharq_prep(d_X, d_gamma, eps, nullptr, a, stream))) return st;
     return sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream);
   }
@@ -328,7 +341,8 @@ int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, co
       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, T, (int)round_up((size_t)T, 128), w->K, 1,
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, 1, nullptr, d_Y, out_dtype == SHARQ_OUT_F32 ? 1 : 0,
-      g.bn, g.splits, static_cast<int*>(d_ws), nullptr, reinterpret_cast<cudaStream_t>(stream), d_X, d_gamma, eps);
+      g.bn, g.splits, static_cast<int*>(d_ws), nullptr, reinterpret_cast<cudaStream_t>(stream), d_X, d_gamma, eps,
+      false);
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 

@@ -86,6 +86,7 @@ struct GemmArgs {
   int out_f32;
   int sharq_mode;
   int splits;
+  int per_token;  // s_g holds one scale per activation row
   // fused decode form: raw activations are prepared inside the GEMM
   const __nv_bfloat16* X;      // [T][K] bf16
   const __nv_bfloat16* gamma;  // [K] bf16 or nullptr
@@ -662,8 +663,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       record_error(args.err, kErrTimeout);
       abort_sh = 1;
     } else if (!kSplit) {
-      const float scale = __fmul_rn(kFused ? fstats.s : *args.s_g, args.s_w[expert]);
       const int row = mt * 128 + rl;
+      const float scale =
+          __fmul_rn(kFused ? fstats.s : args.s_g[args.per_token ? row : 0], args.s_w[expert]);
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t v[32];
@@ -709,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
     if (!ok) {
       if (threadIdx.x == 0) record_error(args.err, kErrTimeout);
     } else {
-      const float scale = __fmul_rn(kFused ? fstats.s : *args.s_g, args.s_w[expert]);
+      const float sw = args.s_w[expert];
       const float* recv = reinterpret_cast<const float*>(smem + C::kRingBytes);
       constexpr int q4 = BN / 4;
       for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
@@ -723,7 +725,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
           acc.z = __fadd_rn(acc.z, q.z);
           acc.w = __fadd_rn(acc.w, q.w);
         }
-        store4(args.Y, args.out_f32, (size_t)(mt * 128 + my0 + r) * args.D + nt * BN + 4 * c4, acc, scale);
+        const int row = mt * 128 + my0 + r;
+        const float scale = __fmul_rn(kFused ? fstats.s : args.s_g[args.per_token ? row : 0], sw);
+        store4(args.Y, args.out_f32, (size_t)row * args.D + nt * BN + 4 * c4, acc, scale);
       }
     }
   }
@@ -909,7 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
     const int sp = warp & 3;  // TMEM lane quarter this warp may access
     const int rl = sp * 32 + lane;
     grid_dependency_wait();  // s_g is written by the preceding sharq_prep
-    const float s_g = *args.s_g;
+    const float s_tensor = args.per_token ? 0.0f : *args.s_g;
     uint32_t k = 0;
     for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
       const int mt = tile / n_tiles, nt = tile - mt * n_tiles;
@@ -922,7 +926,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
         break;
       }
       tc_fence_after();
-      const float scale = __fmul_rn(s_g, args.s_w[expert]);
+      const float scale =
+          __fmul_rn(args.per_token ? args.s_g[mt * 128 + rl] : s_tensor, args.s_w[expert]);
       const int valid = min(128, args.T - mt * 128);
       const size_t off = (size_t)(mt * 128 + rl) * args.D + (size_t)nt * BN;
       if (!args.out_f32) {
@@ -1043,7 +1048,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
                           int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
-                          const void* gamma_fused, float eps_fused) {
+                          const void* gamma_fused, float eps_fused, bool per_token) {
   GemmArgs a = {};
   a.a_sp = a_sp;
   a.a_meta = a_meta;
@@ -1066,13 +1071,14 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.out_f32 = out_f32;
   a.sharq_mode = sharq_mode;
   a.splits = splits;
+  a.per_token = per_token ? 1 : 0;
   a.X = static_cast<const __nv_bfloat16*>(X_fused);
   a.gamma = static_cast<const __nv_bfloat16*>(gamma_fused);
   a.eps = eps_fused;
   const int m_tiles = Tp / 128;
   if (m_tiles == 0) return cudaSuccess;
   if (X_fused) {  // fused decode form
-    if (T > 32 || m_tiles != 1 || !sharq_mode || group_offsets) return cudaErrorInvalidValue;
+    if (T > 32 || m_tiles != 1 || !sharq_mode || group_offsets || per_token) return cudaErrorInvalidValue;
     if (splits > 1) {
       if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
       return launch_cfg<128, true, true>(a, m_tiles, stream);

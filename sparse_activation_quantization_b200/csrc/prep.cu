@@ -323,7 +323,7 @@ constexpr uint64_t kBarrierLimitNs = 2000000000ull;
 template <int NC>
 constexpr int fused_max_threads() { return NC == 4 ? 640 : kFusedMaxThreads; }
 
-template <int NC, bool kSharq>
+template <int NC, bool kSharq, bool kPerToken = false>
 __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     inv_rms[t] = 1.0f;
   }
 
-  // CTA max |Xn| -> device-wide max
+  // CTA max |Xn| -> device-wide max (per-token: the row max)
   float a = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8 * NC; ++i) a = fmaxf(a, fabsf(x[i]));
@@ -392,6 +392,15 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if (lane == 0) wmax[warp] = a;
   __syncthreads();
+  if (kPerToken) {
+    // every row is its own tensor: s_t from the row's warps, no grid barrier
+    float m = 0.0f;
+    for (int w = 0; w < wpr; ++w) m = fmaxf(m, wmax[rl * wpr + w]);
+    const float s = m > 0.0f ? __fdiv_rn(m, kGlobalDiv) : 1.0f;
+    if (live && li == 0) s_g_out[t] = s;
+    if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
+    return;
+  }
   if (threadIdx.x == 0) {
     float m = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
@@ -497,6 +506,23 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   return cudaSuccess;
 }
 
+// Per-token scales need no device-wide max: the single-launch kernel serves
+// every T (CTAs are independent, so the grid need not fit the GPU).
+template <int NC>
+cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index,
+                                int T, int Tp, int K, float* inv_rms, unsigned int* sync, float* s_t, QuantPtrs p,
+                                cudaStream_t stream) {
+  const int tpr = (((K >> 3) / NC) + 31) & ~31;
+  int rpc = 512 / tpr;
+  rpc = rpc < 1 ? 1 : rpc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((T + rpc - 1) / rpc);
+  cfg.blockDim = dim3(rpc * tpr);
+  cfg.stream = stream;
+  return cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, true, true>, Xb, Gb, eps, row_index, T, Tp, K, rpc, inv_rms,
+                            sync, s_t, p);
+}
+
 template <bool kSharq>
 cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
                           int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
@@ -540,8 +566,10 @@ extern "C" int sharq_debug_set_trace_prep(void* p) {
 }
 #endif
 
+bool prep_per_token_supported(int K) { return fused_runs_per_thread(K) != 0; }
+
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
-                        int K, bool sharq_mode, float* inv_rms, float* s_g, unsigned int* gmax_bits,
+                        int K, bool sharq_mode, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
                         cudaStream_t stream) {
   // gmax_bits[0..3]: device-wide max, barrier arrivals, departures, error
@@ -550,6 +578,15 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf};
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
+  if (per_token) {  // s_g: Tp floats, one per row (SharQ mode only)
+    if (T == 0) return cudaSuccess;
+    switch (fused_runs_per_thread(K)) {
+      case 1: return launch_per_token_nc<1>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream);
+      case 2: return launch_per_token_nc<2>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream);
+      case 4: return launch_per_token_nc<4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
 
   if (T > 0) {
     bool launched = false;
@@ -626,7 +663,7 @@ static cudaError_t noalloc_scratch(unsigned char** out) {
 }
 
 cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
-                                int K, bool sharq_mode, float* s_g, uint8_t* sp_codes, uint8_t* meta,
+                                int K, bool sharq_mode, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
                                 uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, unsigned int* err_out,
                                 cudaStream_t stream) {
   if (T > kNoAllocMaxRows) return cudaErrorInvalidValue;
@@ -638,8 +675,8 @@ cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, con
   // the array keeps the last call's contents: start every call from zero
   e = cudaMemsetAsync(sync, 0, 4 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
-  e = launch_prep(X, gamma, eps, row_index, T, Tp, K, sharq_mode, inv, s_g, sync, sp_codes, meta, sp_sf, r_codes,
-                  r_sf, stream);
+  e = launch_prep(X, gamma, eps, row_index, T, Tp, K, sharq_mode, per_token, inv, s_g, sync, sp_codes, meta, sp_sf,
+                  r_codes, r_sf, stream);
   if (e != cudaSuccess) return e;
   // forward the error word to where sharq_linear looks for it
   if (err_out) e = cudaMemcpyAsync(err_out, sync + 3, sizeof(unsigned int), cudaMemcpyDeviceToDevice, stream);

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(sq.EXPORTED_SYMBOLS)
-    assert sq.sharq_abi_version() == 1
+    assert sq.sharq_abi_version() == 2
 
 
 def test_sizes(L):
@@ -70,6 +70,15 @@ def test_views_carve_inside_the_buffer(L):
     assert (a.T, a.Tp, a.K, a.mode) == (300, 384, 768, 0)
     b = sq.sharq_act_view(base, T, K, 1)
     assert b.sp_codes is None and b.meta is None
+    # per-token: the SharQ operands plus Tp per-row scales outside the
+    # 256-byte scalar block that holds the sync words
+    nt = sq.sharq_act_bytes(T, K, sq.SHARQ_MODE_SHARQ_TOKEN)
+    assert nt >= n + 384 * 4
+    c = sq.sharq_act_view(base, T, K, sq.SHARQ_MODE_SHARQ_TOKEN)
+    assert c.sp_codes and c.meta and c.sp_sf
+    assert base <= c.s_g and c.s_g + 384 * 4 <= c.gmax_bits - 16
+    assert c.gmax_bits + 240 <= base + nt
+    assert c.mode == sq.SHARQ_MODE_SHARQ_TOKEN
     w = sq.sharq_weight_view(base, K, 256, 3)
     assert (w.K, w.D, w.E) == (768, 256, 3)
     assert base <= w.s_w < base + sq.sharq_weight_bytes(K, 256, 3)
