@@ -280,6 +280,95 @@ def linear_grouped(p, wqs, offsets):
     return y
 
 
+# ------------------------------------------------- Table-5 path modes ----
+# The xllm-io review's ablation (section 5.3, Table 5) compares the SharQ
+# decomposition with three other ways of splitting the activation into two
+# FP4 operands.  The page names them only; the plainest reading, used here,
+# keeps every other step of the method (RMSNorm, the per-tensor scale, the
+# block quantizer, the 4:8 in-pairs rule):
+#   Sparse only    the backbone alone (no residual operand);
+#   Dense+Dense    dense NVFP4 of Xn (16-element blocks), then dense NVFP4 of
+#                  its residual Xn - dequant;
+#   Sparse+Sparse  the SharQ backbone, then the residual R pruned by the same
+#                  4:8 in-pairs rule (scores max|R|) and quantized as a
+#                  sparse operand (one scale per 32 logical K).
+
+def prep_dense_dense(x, gamma=None, eps=1e-5):
+    """Dense+Dense mode.  Returns dict xn, inv, s_g, gmax, b_codes [T,K],
+    b_sf [T,K/16], b_t (dequantized first level), r [T,K] = Xn - b_t
+    (float32), r_codes [T,K], r_sf [T,K/16], r_t."""
+    xn, inv = rmsnorm(x, gamma, eps)
+    T, K = xn.shape
+    s_g, gmax = pts_scale(xn)
+    bc, bsb, bdeq = nvfp4_quant(xn.reshape(T, K // 16, 16), s_g)
+    b_t = bdeq.reshape(T, K)
+    r = (xn - b_t).astype(np.float32)
+    rc, rsb, rdeq = nvfp4_quant(r.reshape(T, K // 16, 16), s_g)
+    return dict(xn=xn, inv=inv, s_g=s_g, gmax=gmax, b_codes=bc.reshape(T, K), b_sf=bsb, b_t=b_t, r=r,
+                r_codes=rc.reshape(T, K), r_sf=rsb, r_t=rdeq.reshape(T, K))
+
+
+def prep_sparse_sparse(x, gamma=None, eps=1e-5):
+    """Sparse+Sparse mode: prep() for the backbone and R, then R pruned and
+    quantized like the backbone.  Adds r_keep [T,K/8,4], r_meta [T,K/8],
+    r_sp_vals [T,K/2], r_sp_codes [T,K/2], r_sp_sf [T,K/32], r_sp_t [T,K]
+    (dequantized residual scattered to its kept positions)."""
+    p = prep(x, gamma, eps)
+    r = p["r"]
+    T, K = r.shape
+    keep, meta = pair_mask(r)
+    keep_el = np.repeat(keep, 2, axis=-1).reshape(T, K)
+    vals = r[keep_el].reshape(T, K // 2)
+    codes, sb, deq = nvfp4_quant(vals.reshape(T, K // 32, 16), p["s_g"])
+    r_sp_t = np.zeros((T, K), dtype=np.float32)
+    r_sp_t[keep_el] = deq.reshape(-1)
+    out = {k: v for k, v in p.items() if k not in ("r_codes", "r_sf", "r_t")}
+    out.update(r_keep=keep, r_meta=meta, r_sp_vals=vals, r_sp_codes=codes.reshape(T, K // 2), r_sp_sf=sb,
+               r_sp_t=r_sp_t)
+    return out
+
+
+def approx_activation(x, gamma=None, eps=1e-5, mode="sharq"):
+    """The activation each mode hands to the GEMMs, dequantized, float64
+    without the global scale folded out: X~ with Y~ = X~ W.  Modes: "nvfp4",
+    "sharq", "sparse_only", "dense_dense", "sparse_sparse"."""
+    if mode == "nvfp4":
+        return prep_nvfp4(x, gamma, eps)["x_t"].astype(np.float64)
+    if mode == "dense_dense":
+        p = prep_dense_dense(x, gamma, eps)
+        return p["b_t"].astype(np.float64) + p["r_t"].astype(np.float64)
+    if mode == "sparse_sparse":
+        p = prep_sparse_sparse(x, gamma, eps)
+        return p["xsp_t"].astype(np.float64) + p["r_sp_t"].astype(np.float64)
+    p = prep(x, gamma, eps)
+    if mode == "sparse_only":
+        return p["xsp_t"].astype(np.float64)
+    return p["xsp_t"].astype(np.float64) + p["r_t"].astype(np.float64)
+
+
+def linear_mode(p, wq, mode):
+    """Float64 GEMM of a Table-5 mode from its prep dict: the operands the
+    GPU multiplies (dequantized codes times scale values) times the weight
+    view each operand is paired with, times s_g * s_w."""
+    K, D = wq["w_t"].shape
+    w32 = wq["w_t"]
+    w16 = (e2m1_decode(wq["codes"]).reshape(D, K // 16, 16)
+           * e4m3_decode(wq["sf16"])[..., None]).reshape(D, K).T
+    if mode == "sparse_only":
+        y = dequant_sparse(p) @ w32
+    elif mode == "dense_dense":
+        T = p["xn"].shape[0]
+        dq = lambda c, sf: (e2m1_decode(c).reshape(T, K // 16, 16) * e4m3_decode(sf)[..., None]).reshape(T, K)
+        y = dq(p["b_codes"], p["b_sf"]) @ w16 + dq(p["r_codes"], p["r_sf"]) @ w16
+    elif mode == "sparse_sparse":
+        T = p["xn"].shape[0]
+        r = {"xn": p["xn"], "keep": p["r_keep"], "sp_codes": p["r_sp_codes"], "sp_sf": p["r_sp_sf"]}
+        y = dequant_sparse(p) @ w32 + dequant_sparse(r) @ w32
+    else:
+        raise ValueError(mode)
+    return y * (_row_scale(p["s_g"], y.shape[0]) * np.float64(wq["s_w"]))
+
+
 def prep_nvfp4(x, gamma=None, eps=1e-5):
     """Plain NVFP4 preparation, the comparator the SharQ evaluation reports
     as "NVFP4" (xllm-io review, Table 1; the kasblo.com explainer lists the
