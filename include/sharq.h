@@ -73,6 +73,23 @@ enum { SHARQ_OUT_BF16 = 0, SHARQ_OUT_F32 = 1 };
  * are not those of the per-tensor mode.  Supported for K <= 20480. */
 enum { SHARQ_MODE_SHARQ = 0, SHARQ_MODE_NVFP4 = 1, SHARQ_MODE_SHARQ_TOKEN = 2 };
 
+/* The other operand splits of the xllm-io review's ablation (section 5.3,
+ * Table 5), under the plainest reading of their names; every other step
+ * (RMSNorm, the per-tensor scale, the block quantizer, the 4:8 in-pairs rule)
+ * is the method's:
+ *   SPARSE_ONLY    the SharQ backbone alone: sharq_prep writes the SharQ
+ *                  operands, sharq_linear multiplies only the backbone.
+ *   DENSE_DENSE    first operand: dense NVFP4 of Xn (16-element blocks) in
+ *                  sp_codes / sp_sf (laid out as r_codes / r_sf); second:
+ *                  dense NVFP4 of Xn minus its dequantized value.
+ *   SPARSE_SPARSE  the SharQ backbone, and the residual pruned by the same
+ *                  4:8 in-pairs rule (scores max|R|) and quantized as a
+ *                  sparse operand: r_codes laid out as sp_codes, r_sf as
+ *                  sp_sf, its metadata in r_meta.
+ * These modes always run the persistent GEMM (no split-K decode form) and
+ * are not accepted by sharq_prep_linear. */
+enum { SHARQ_MODE_SPARSE_ONLY = 3, SHARQ_MODE_DENSE_DENSE = 4, SHARQ_MODE_SPARSE_SPARSE = 5 };
+
 /* Tile geometry of every packed operand: 128 rows x 256 logical K. */
 #define SHARQ_TILE_ROWS 128
 #define SHARQ_TILE_K 256
@@ -141,6 +158,7 @@ typedef struct {
   float *s_g;
   unsigned int *gmax_bits;
   int T, Tp, K, mode;
+  void *r_meta; /* SPARSE_SPARSE only: the residual's metadata (layout as meta) */
 } sharq_act;
 
 /* Host-only size queries (pure functions; 0 on invalid shape). */

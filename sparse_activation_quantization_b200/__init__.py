@@ -15,7 +15,8 @@ import os
 
 __all__ = [
     "SharqError", "SharqAct", "SharqWeight", "lib", "library_path",
-    "SHARQ_MODE_SHARQ", "SHARQ_MODE_NVFP4", "SHARQ_MODE_SHARQ_TOKEN", "SHARQ_OUT_BF16", "SHARQ_OUT_F32",
+    "SHARQ_MODE_SHARQ", "SHARQ_MODE_NVFP4", "SHARQ_MODE_SHARQ_TOKEN", "SHARQ_MODE_SPARSE_ONLY",
+    "SHARQ_MODE_DENSE_DENSE", "SHARQ_MODE_SPARSE_SPARSE", "SHARQ_OUT_BF16", "SHARQ_OUT_F32",
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes",
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
@@ -26,6 +27,9 @@ __all__ = [
 SHARQ_MODE_SHARQ = 0
 SHARQ_MODE_NVFP4 = 1
 SHARQ_MODE_SHARQ_TOKEN = 2
+SHARQ_MODE_SPARSE_ONLY = 3
+SHARQ_MODE_DENSE_DENSE = 4
+SHARQ_MODE_SPARSE_SPARSE = 5
 SHARQ_OUT_BF16 = 0
 SHARQ_OUT_F32 = 1
 
@@ -57,7 +61,8 @@ class SharqAct(ctypes.Structure):
     _fields_ = [("sp_codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("sp_sf", ctypes.c_void_p),
                 ("r_codes", ctypes.c_void_p), ("r_sf", ctypes.c_void_p), ("inv_rms", ctypes.c_void_p),
                 ("s_g", ctypes.c_void_p), ("gmax_bits", ctypes.c_void_p),
-                ("T", ctypes.c_int), ("Tp", ctypes.c_int), ("K", ctypes.c_int), ("mode", ctypes.c_int)]
+                ("T", ctypes.c_int), ("Tp", ctypes.c_int), ("K", ctypes.c_int), ("mode", ctypes.c_int),
+                ("r_meta", ctypes.c_void_p)]
 
 
 def lib():

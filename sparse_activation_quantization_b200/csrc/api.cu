@@ -11,13 +11,14 @@
 
 namespace sharq {
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp, int K,
-                        bool sharq_mode, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
-                        uint8_t* sp_codes,
-                        uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, cudaStream_t stream);
+                        int kind, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
+                        uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
+                        uint8_t* r_meta, cudaStream_t stream);
 cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf32, uint8_t* sf16,
                                float* s_w, unsigned int* amax_bits, cudaStream_t stream);
 cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
-                          const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
+                          const uint8_t* a_rsf, const uint8_t* a_rmeta, const float* s_g, int T, int Tp, int K,
+                          int gmode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
                           int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
@@ -25,9 +26,9 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
 int noalloc_max_rows();
 bool prep_per_token_supported(int K);
 cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
-                                int K, bool sharq_mode, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
-                                uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, unsigned int* err_out,
-                                cudaStream_t stream);
+                                int K, int kind, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
+                                uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, uint8_t* r_meta,
+                                unsigned int* err_out, cudaStream_t stream);
 }  // namespace sharq
 
 namespace {
@@ -47,28 +48,51 @@ bool shape_ok_d(int D) { return D > 0 && D <= kMaxD && D % 128 == 0; }
 bool shape_ok_t(int T) { return T >= 0 && T <= kMaxT; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool mode_ok(int mode) {
-  return mode == SHARQ_MODE_SHARQ || mode == SHARQ_MODE_NVFP4 || mode == SHARQ_MODE_SHARQ_TOKEN;
+bool mode_ok(int mode) { return mode >= SHARQ_MODE_SHARQ && mode <= SHARQ_MODE_SPARSE_SPARSE; }
+// operand sets per mode: first operand (sp_codes/meta/sp_sf) sparse or dense,
+// second operand (r_codes/r_sf, r_meta) dense or sparse
+bool has_first(int mode) { return mode != SHARQ_MODE_NVFP4; }
+bool first_sparse(int mode) { return has_first(mode) && mode != SHARQ_MODE_DENSE_DENSE; }
+bool second_sparse(int mode) { return mode == SHARQ_MODE_SPARSE_SPARSE; }
+// prep operand kind (csrc/quant.cuh) and GEMM operand set (csrc/gemm.cu)
+int prep_kind(int mode) {
+  switch (mode) {
+    case SHARQ_MODE_NVFP4: return 0;
+    case SHARQ_MODE_DENSE_DENSE: return 2;
+    case SHARQ_MODE_SPARSE_SPARSE: return 3;
+    default: return 1;  // SHARQ, SHARQ_TOKEN, SPARSE_ONLY
+  }
 }
-bool has_sparse(int mode) { return mode != SHARQ_MODE_NVFP4; }
+int gemm_mode(int mode) {
+  switch (mode) {
+    case SHARQ_MODE_NVFP4: return 1;
+    case SHARQ_MODE_SPARSE_ONLY: return 2;
+    case SHARQ_MODE_DENSE_DENSE: return 3;
+    case SHARQ_MODE_SPARSE_SPARSE: return 4;
+    default: return 0;  // SHARQ, SHARQ_TOKEN
+  }
+}
 
 // layout sizes, shared by the *_bytes and *_view functions
 struct ActLayout {
-  size_t r_codes, r_sf, sp_codes, meta, sp_sf, inv, s_tok, scal, total;
+  size_t r_codes, r_sf, sp_codes, meta, sp_sf, r_meta, inv, s_tok, scal, total;
 };
 ActLayout act_layout(int T, int K, int mode) {
   ActLayout L{};
   const size_t Tp = round_up((size_t)T, 128);
   const size_t tiles = (Tp / 128) * (size_t)(K / 256);
   size_t off = 0;
-  L.r_codes = off; off += tiles * sharq::kCodesTile;
-  L.r_sf = off;    off += tiles * sharq::kSf16Tile;
+  const bool s2 = second_sparse(mode);
+  L.r_codes = off; off += tiles * (s2 ? sharq::kSpTile : sharq::kCodesTile);
+  L.r_sf = off;    off += tiles * (s2 ? sharq::kSf32Tile : sharq::kSf16Tile);
   L.sp_codes = off;
-  if (has_sparse(mode)) off += tiles * sharq::kSpTile;
+  if (has_first(mode)) off += tiles * (first_sparse(mode) ? sharq::kSpTile : sharq::kCodesTile);
   L.meta = off;
-  if (has_sparse(mode)) off += tiles * sharq::kMetaTile;
+  if (first_sparse(mode)) off += tiles * sharq::kMetaTile;
   L.sp_sf = off;
-  if (has_sparse(mode)) off += tiles * sharq::kSf32Tile;
+  if (has_first(mode)) off += tiles * (first_sparse(mode) ? sharq::kSf32Tile : sharq::kSf16Tile);
+  L.r_meta = off;
+  if (s2) off += tiles * sharq::kMetaTile;
   L.inv = off;     off = round_up(off + Tp * sizeof(float), kAlign);
   L.s_tok = off;   // per-token scales (SHARQ_TOKEN only)
   if (mode == SHARQ_MODE_SHARQ_TOKEN) off = round_up(off + Tp * sizeof(float), kAlign);
@@ -144,8 +168,10 @@ int act_ok(const sharq_act* a) {
   if (!mode_ok(a->mode)) return SHARQ_ERR_INVALID_ARG;
   if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
   if (!a->r_codes || !a->r_sf || !a->inv_rms || !a->s_g || !a->gmax_bits) return SHARQ_ERR_INVALID_ARG;
-  if (has_sparse(a->mode) && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
-  const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf};
+  if (has_first(a->mode) && (!a->sp_codes || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  if (first_sparse(a->mode) && !a->meta) return SHARQ_ERR_INVALID_ARG;
+  if (second_sparse(a->mode) && !a->r_meta) return SHARQ_ERR_INVALID_ARG;
+  const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf, a->r_meta};
   for (const void* q : p)
     if (q && !aligned(q, 16)) return SHARQ_ERR_INVALID_ARG;
   return SHARQ_OK;
@@ -176,7 +202,8 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
   cudaError_t e = sharq::launch_linear(
       static_cast<const uint8_t*>(a->sp_codes), static_cast<const uint8_t*>(a->meta),
       static_cast<const uint8_t*>(a->sp_sf), static_cast<const uint8_t*>(a->r_codes),
-      static_cast<const uint8_t*>(a->r_sf), a->s_g, a->T, a->Tp, a->K, has_sparse(a->mode) ? 1 : 0,
+      static_cast<const uint8_t*>(a->r_sf), static_cast<const uint8_t*>(a->r_meta), a->s_g, a->T, a->Tp, a->K,
+      gemm_mode(a->mode),
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
       out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, static_cast<int*>(d_ws),
@@ -243,12 +270,12 @@ int sharq_act_view(void* d_buf, int T, int K, int mode, sharq_act* out) {
   if (!aligned(d_buf, kAlign)) return SHARQ_ERR_INVALID_ARG;
   const ActLayout L = act_layout(T, K, mode);
   uint8_t* b = static_cast<uint8_t*>(d_buf);
-  const bool sq = has_sparse(mode);
   out->r_codes = b + L.r_codes;
   out->r_sf = b + L.r_sf;
-  out->sp_codes = sq ? b + L.sp_codes : nullptr;
-  out->meta = sq ? b + L.meta : nullptr;
-  out->sp_sf = sq ? b + L.sp_sf : nullptr;
+  out->sp_codes = has_first(mode) ? b + L.sp_codes : nullptr;
+  out->meta = first_sparse(mode) ? b + L.meta : nullptr;
+  out->sp_sf = has_first(mode) ? b + L.sp_sf : nullptr;
+  out->r_meta = second_sparse(mode) ? b + L.r_meta : nullptr;
   out->inv_rms = reinterpret_cast<float*>(b + L.inv);
   out->s_g = reinterpret_cast<float*>(b + (mode == SHARQ_MODE_SHARQ_TOKEN ? L.s_tok : L.scal));
   out->gmax_bits = reinterpret_cast<unsigned int*>(b + L.scal + 16);
@@ -283,10 +310,10 @@ int sharq_prep(const void* d_X, const void* d_gamma, float eps, const int* d_row
   if (per_token && !sharq::prep_per_token_supported(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if ((st = check_device())) return st;
   cudaError_t e = sharq::launch_prep(
-      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, has_sparse(a->mode), per_token, a->inv_rms, a->s_g,
+      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, prep_kind(a->mode), per_token, a->inv_rms, a->s_g,
       a->gmax_bits, static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta),
       static_cast<uint8_t*>(a->sp_sf), static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf),
-      reinterpret_cast<cudaStream_t>(stream));
+      static_cast<uint8_t*>(a->r_meta), reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 
@@ -298,9 +325,11 @@ int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const in
   if (!mode_ok(a->mode)) return SHARQ_ERR_INVALID_ARG;
   if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
   if (!a->r_codes || !a->r_sf || !a->s_g) return SHARQ_ERR_INVALID_ARG;
-  if (has_sparse(a->mode) && (!a->sp_codes || !a->meta || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  if (has_first(a->mode) && (!a->sp_codes || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
+  if (first_sparse(a->mode) && !a->meta) return SHARQ_ERR_INVALID_ARG;
+  if (second_sparse(a->mode) && !a->r_meta) return SHARQ_ERR_INVALID_ARG;
   if (a->mode == SHARQ_MODE_SHARQ_TOKEN && !sharq::prep_per_token_supported(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
-  const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf};
+  const void* p[] = {a->r_codes, a->r_sf, a->sp_codes, a->meta, a->sp_sf, a->r_meta};
   for (const void* q : p)
     if (q && !aligned(q, 16)) return SHARQ_ERR_INVALID_ARG;
   if (a->T > 0 && (!d_X || !aligned(d_X, 16))) return SHARQ_ERR_INVALID_ARG;
@@ -309,10 +338,10 @@ int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const in
   int st = check_device();
   if (st) return st;
   cudaError_t e = sharq::launch_prep_noalloc(
-      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, has_sparse(a->mode), a->mode == SHARQ_MODE_SHARQ_TOKEN,
-      a->s_g,
-      static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta), static_cast<uint8_t*>(a->sp_sf),
-      static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf), a->gmax_bits ? a->gmax_bits + 3 : nullptr,
+      d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, prep_kind(a->mode), a->mode == SHARQ_MODE_SHARQ_TOKEN,
+      a->s_g, static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta), static_cast<uint8_t*>(a->sp_sf),
+      static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf), static_cast<uint8_t*>(a->r_meta),
+      a->gmax_bits ? a->gmax_bits + 3 : nullptr,
       reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
@@ -325,7 +354,8 @@ int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, co
   if (w->E != 1) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(T)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if (T > SHARQ_FUSED_MAX_T) {  // larger batches: the two-call path through `a`
-    if (!a || a->T != T || a->K != w->K || !has_sparse(a->mode)) return SHARQ_ERR_INVALID_ARG;
+    if (!a || a->T != T || a->K != w->K || (a->mode != SHARQ_MODE_SHARQ && a->mode != SHARQ_MODE_SHARQ_TOKEN))
+      return SHARQ_ERR_INVALID_ARG;
     if ((st = sharq_prep(d_X, d_gamma, eps, nullptr, a, stream))) return st;
     return sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream);
   }
@@ -338,7 +368,8 @@ int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, co
   if (T == 0) return SHARQ_OK;
   const GemmShape g = gemm_shape(T, w->K, w->D, 1);
   cudaError_t e = sharq::launch_linear(
-      nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, T, (int)round_up((size_t)T, 128), w->K, 1,
+      nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, T, (int)round_up((size_t)T, 128), w->K,
+      0 /* SharQ operands */,
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, 1, nullptr, d_Y, out_dtype == SHARQ_OUT_F32 ? 1 : 0,
       g.bn, g.splits, static_cast<int*>(d_ws), nullptr, reinterpret_cast<cudaStream_t>(stream), d_X, d_gamma, eps,

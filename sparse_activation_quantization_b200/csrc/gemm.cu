@@ -73,6 +73,7 @@ struct GemmArgs {
   const uint8_t* a_spsf;
   const uint8_t* a_r;
   const uint8_t* a_rsf;
+  const uint8_t* a_rmeta;  // Sparse+Sparse: the residual's metadata
   const float* s_g;
   const uint8_t* w_codes;
   const uint8_t* w_sf32;
@@ -413,7 +414,7 @@ __device__ __forceinline__ bool fused_prep(const GemmArgs& args, uint8_t* smem, 
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = norm_one(x[e], inv, gm[e]);
         }
-        quant_runs<1, true>(x, r, lane, 256, s, six_s, q);  // one 256-K tile: tile index 0
+        quant_runs<1, kKindSharq>(x, r, lane, 256, s, six_s, q);  // one 256-K tile: tile index 0
       }
     }
     fence_proxy_async_smem();   // generic writes -> visible to tcgen05.cp / MMA
@@ -742,19 +743,74 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
 }
 
 // ---------------------------------------------------------------------------
-// Persistent form (no split-K, activation already prepared: prefill and the
-// grouped expert shapes).  One CTA per SM walks the output tiles t =
-// blockIdx.x, blockIdx.x + gridDim.x, ... (row-major over (m-tile, n-tile),
-// so CTAs running at the same time share activation tiles in L2).  The
-// shared-memory ring and its phases run on across tiles, so the producer
-// streams the next tile's stages while the current one finishes, and the
-// accumulator is handed back to the MMA warp as soon as the epilogue has
-// moved it into registers (bf16 output: the tile's row in 128 packed
-// registers per thread) -- the global stores of tile k overlap the MMAs of
-// tile k + 1.  Set-up (barriers, TMEM allocation) is paid once per SM.
-template <int BN>
+// Persistent form (no split-K, activation already prepared: prefill, the
+// grouped expert shapes, and every shape of the Table-5 operand modes).  One
+// CTA per SM walks the output tiles t = blockIdx.x, blockIdx.x + gridDim.x,
+// ... (row-major over (m-tile, n-tile), so CTAs running at the same time
+// share activation tiles in L2).  The shared-memory ring and its phases run on
+// across tiles, so the producer streams the next tile's stages while the
+// current one finishes, and the accumulator is handed back to the MMA warp as
+// soon as the epilogue has moved it into registers (bf16 output: the tile's
+// row in 128 packed registers per thread) -- the global stores of tile k
+// overlap the MMAs of tile k + 1.  Set-up (barriers, TMEM allocation) is paid
+// once per SM.
+//
+// Operand sets (kG): both FP4 operands of the activation accumulate into one
+// TMEM tile and read the same weight tile; a sparse operand (4:8 in-pairs,
+// one scale per 32 logical K) pairs with the weight's per-32 scale view, a
+// dense one (one scale per 16 K) with the per-16 view.
+enum : int { kGemmSharq = 0, kGemmNvfp4 = 1, kGemmSparseOnly = 2, kGemmDenseDense = 3, kGemmSparseSparse = 4 };
+
+template <int BN, int kG>
+struct PCfg {
+  static constexpr int kHalves = BN / 128;
+  static constexpr bool kHas1 = kG != kGemmNvfp4;       // first operand (backbone)
+  static constexpr bool kSp1 = kG != kGemmDenseDense;   // ... sparse
+  static constexpr bool kHas2 = kG != kGemmSparseOnly;  // second operand (residual)
+  static constexpr bool kSp2 = kG == kGemmSparseSparse;
+  static constexpr bool kB32 = (kHas1 && kSp1) || (kHas2 && kSp2);
+  static constexpr bool kB16 = (kHas1 && !kSp1) || (kHas2 && !kSp2);
+  static constexpr int kA1 = kHas1 ? (kSp1 ? kSpTile : kCodesTile) : 0;
+  static constexpr int kE1 = kHas1 && kSp1 ? kMetaTile : 0;
+  static constexpr int kS1 = kHas1 ? (kSp1 ? kSf32Tile : kSf16Tile) : 0;
+  static constexpr int kA2 = kHas2 ? (kSp2 ? kSpTile : kCodesTile) : 0;
+  static constexpr int kE2 = kHas2 && kSp2 ? kMetaTile : 0;
+  static constexpr int kS2 = kHas2 ? (kSp2 ? kSf32Tile : kSf16Tile) : 0;
+  // stage layout (every size a multiple of 1 KB: swizzled tiles stay aligned)
+  static constexpr int kOffB = 0;
+  static constexpr int kOffA2 = kOffB + BN * 128;
+  static constexpr int kOffA1 = kOffA2 + kA2;
+  static constexpr int kOffE1 = kOffA1 + kA1;
+  static constexpr int kOffE2 = kOffE1 + kE1;
+  static constexpr int kOffS1 = kOffE2 + kE2;
+  static constexpr int kOffS2 = kOffS1 + kS1;
+  static constexpr int kOffSFB32 = kOffS2 + kS2;
+  static constexpr int kOffSFB16 = kOffSFB32 + (kB32 ? kHalves * kSf32Tile : 0);
+  static constexpr int kStageBytes = kOffSFB16 + (kB16 ? kHalves * kSf16Tile : 0);
+  static constexpr int kStages = (BN == 128 && 4 * kStageBytes + 1024 <= 232448) ? 4 : 3;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  // TMEM: accumulator, then two scale regions (alternating by stage) of 32
+  // activation columns + the weight scale columns
+  static constexpr uint32_t kColAcc = 0;
+  static constexpr uint32_t kSfbCols = BN / 32;
+  static constexpr uint32_t kSfE1 = 0, kSfE2 = 4, kSfS1 = kSp1 ? 8 : 0, kSfS2 = 16;
+  static constexpr uint32_t kSfB32 = 32, kSfB16 = 32 + 2 * kSfbCols;
+  static constexpr uint32_t kSfRegion = 32 + 6 * kSfbCols;
+  static constexpr uint32_t kColSf0 = BN;
+  static constexpr uint32_t kTmemCols = BN + 2 * kSfRegion <= 256 ? 256 : 512;
+  // transaction bytes per stage with `rows` valid activation rows
+  __host__ __device__ static constexpr uint32_t tx(uint32_t rows) {
+    return BN * 128 + (kB32 ? kHalves * kSf32Tile : 0) + (kB16 ? kHalves * kSf16Tile : 0) +
+           rows * (uint32_t)(kA1 / 128 + kE1 / 128 + kA2 / 128 + kE2 / 128) + kS1 + kS2;
+  }
+  static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory overflow");
+  static_assert(BN + 2 * kSfRegion <= 512, "TMEM overflow");
+};
+
+template <int BN, int kG>
 __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(const GemmArgs args, int m_tiles) {
-  using C = Cfg<BN, false>;
+  using C = PCfg<BN, kG>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::kStages];
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
@@ -769,7 +825,6 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
   const int NB = args.D >> 7;
   const int n_tiles = args.D / BN;
   const int ntiles = m_tiles * n_tiles;
-  const bool sharq = args.sharq_mode != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -785,14 +840,15 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
     tmem_alloc(&tmem_base_sh, C::kTmemCols);
     tmem_relinquish();
   }
-  if (sharq) {
+  if (C::kE1 || C::kE2) {
     // Metadata rows past a partial tile's valid rows are never copied in: give
     // every row a valid pattern (pairs 0 and 1) once; later tiles leave
     // metadata written by sharq_prep there, which is valid as well.
     for (int idx = threadIdx.x; idx < C::kStages * 128; idx += kThreads) {
       const int st = idx >> 7, row = idx & 127;
-      *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE + row * 16) =
-          make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+      const uint4 v = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+      if (C::kE1) *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE1 + row * 16) = v;
+      if (C::kE2) *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE2 + row * 16) = v;
     }
     fence_proxy_async_smem();
   }
@@ -815,9 +871,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
           continue;
         }
         const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
-        const int valid = min(128, args.T - mt * 128);
-        const uint32_t a_rows = (uint32_t)valid;
-        const uint32_t tx = (sharq ? C::kTxSharq : C::kTxNvfp4) - (128u - a_rows) * (sharq ? 208u : 128u);
+        const uint32_t rows = (uint32_t)min(128, args.T - mt * 128);
+        const uint32_t tx = C::tx(rows);
         const size_t a_tile0 = (size_t)mt * KS;
         const size_t b_tile0 = ((size_t)expert * NB + (size_t)nt * C::kHalves) * KS;
         for (int i = 0; i < KS; ++i, ++g) {
@@ -829,22 +884,25 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
             break;
           }
           uint8_t* st = smem + s * C::kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[s], tx);
+          uint64_t* fb = &full_bar[s];
+          mbar_arrive_expect_tx(fb, tx);
 #pragma unroll
           for (int h = 0; h < C::kHalves; ++h) {
             const size_t bt = b_tile0 + (size_t)h * KS + i;
-            bulk_g2s(st + C::kOffB + h * kCodesTile, args.w_codes + bt * kCodesTile, kCodesTile, &full_bar[s]);
-            bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, &full_bar[s]);
-            if (sharq)
-              bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, &full_bar[s]);
+            bulk_g2s(st + C::kOffB + h * kCodesTile, args.w_codes + bt * kCodesTile, kCodesTile, fb);
+            if (C::kB16) bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, fb);
+            if (C::kB32) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
           }
           const size_t at = a_tile0 + i;
-          bulk_g2s(st + C::kOffAR, args.a_r + at * kCodesTile, a_rows * 128u, &full_bar[s]);
-          bulk_g2s(st + C::kOffSFAR, args.a_rsf + at * kSf16Tile, kSf16Tile, &full_bar[s]);
-          if (sharq) {
-            bulk_g2s(st + C::kOffASP, args.a_sp + at * kSpTile, a_rows * 64u, &full_bar[s]);
-            bulk_g2s(st + C::kOffE, args.a_meta + at * kMetaTile, a_rows * 16u, &full_bar[s]);
-            bulk_g2s(st + C::kOffSFASP, args.a_spsf + at * kSf32Tile, kSf32Tile, &full_bar[s]);
+          if (C::kHas1) {
+            bulk_g2s(st + C::kOffA1, args.a_sp + at * C::kA1, rows * (C::kA1 / 128), fb);
+            if (C::kE1) bulk_g2s(st + C::kOffE1, args.a_meta + at * kMetaTile, rows * 16u, fb);
+            bulk_g2s(st + C::kOffS1, args.a_spsf + at * C::kS1, C::kS1, fb);
+          }
+          if (C::kHas2) {
+            bulk_g2s(st + C::kOffA2, args.a_r + at * C::kA2, rows * (C::kA2 / 128), fb);
+            if (C::kE2) bulk_g2s(st + C::kOffE2, args.a_rmeta + at * kMetaTile, rows * 16u, fb);
+            bulk_g2s(st + C::kOffS2, args.a_rsf + at * C::kS2, C::kS2, fb);
           }
         }
       }
@@ -875,32 +933,53 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
           tc_fence_after();
           const uint32_t st = smem_u32(smem + s * C::kStageBytes);
           const uint32_t sf = tmem + C::kColSf0 + (g & 1u) * C::kSfRegion;
-          // each MMA's scale copies right before it: the copies for MMA j + 1
-          // can run while MMA j computes
-          if (sharq) {
-            tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
+          bool acc = i > 0;  // the tile's first MMA overwrites the accumulator
+          // a sparse operand: 2 x (128 x BN x 128 logical K); its metadata
+          // and scales, and the weight's per-32 view (once per stage), right
+          // before each MMA so copies overlap the previous MMA
+          auto sparse_op = [&](uint32_t a_off, uint32_t e_off, uint32_t s_off, uint32_t e_col, uint32_t s_col,
+                               bool copy_b) {
+            tc_cp_128x128b(sf + e_col, smem_desc(st + e_off, 0, 128, kSwNone));
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
+              tc_cp_32x128b_x4(sf + s_col + 4 * j, smem_desc(st + s_off + 512 * j, 0, 128, kSwNone));
+              if (copy_b) {
 #pragma unroll
-              for (int h = 0; h < C::kHalves; ++h)
-                tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
-                                 smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
-              mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffASP + 32 * j, 16, 512, kSw64),
-                          smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + C::kSfE + 2 * j, idesc_sp,
-                          sf + C::kSfASP + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, (i > 0 || j > 0) ? 1u : 0u);
+                for (int h = 0; h < C::kHalves; ++h)
+                  tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
+                                   smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
+              }
+              mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + a_off + 32 * j, 16, 512, kSw64),
+                          smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + e_col + 2 * j, idesc_sp,
+                          sf + s_col + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, acc ? 1u : 0u);
+              acc = true;
             }
+          };
+          // a dense operand: 4 x (128 x BN x 64 K), weight per-16 view
+          auto dense_op = [&](uint32_t a_off, uint32_t s_off, uint32_t s_col, bool copy_b) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_32x128b_x4(sf + s_col + 4 * j, smem_desc(st + s_off + 512 * j, 0, 128, kSwNone));
+              if (copy_b) {
+#pragma unroll
+                for (int h = 0; h < C::kHalves; ++h)
+                  tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
+                                   smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
+              }
+              mma_nvf4(tmem + C::kColAcc, smem_desc(st + a_off + 32 * j, 16, 1024, kSw128),
+                       smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + s_col + 4 * j,
+                       sf + C::kSfB16 + j * C::kSfbCols, acc ? 1u : 0u);
+              acc = true;
+            }
+          };
+          if (C::kHas1) {
+            if (C::kSp1) sparse_op(C::kOffA1, C::kOffE1, C::kOffS1, C::kSfE1, C::kSfS1, true);
+            else dense_op(C::kOffA1, C::kOffS1, C::kSfS1, true);
           }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
-#pragma unroll
-            for (int h = 0; h < C::kHalves; ++h)
-              tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
-                               smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
-            mma_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffAR + 32 * j, 16, 1024, kSw128),
-                     smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + C::kSfAR + 4 * j,
-                     sf + C::kSfB16 + j * C::kSfbCols, (sharq || i > 0 || j > 0) ? 1u : 0u);
+          if (C::kHas2) {
+            // the weight view is already in TMEM when both operands share it
+            if (C::kSp2) sparse_op(C::kOffA2, C::kOffE2, C::kOffS2, C::kSfE2, C::kSfS2, !(C::kHas1 && C::kSp1));
+            else dense_op(C::kOffA2, C::kOffS2, C::kSfS2, !(C::kHas1 && !C::kSp1));
           }
           tc_commit(&empty_bar[s]);
         }
@@ -974,16 +1053,16 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
   }
 }
 
-template <int BN>
+template <int BN, int kG>
 cudaError_t launch_persistent(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
-  using C = Cfg<BN, false>;
+  using C = PCfg<BN, kG>;
   static int sms[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64) return cudaErrorInvalidDevice;
   if (sms[dev] == 0) {
-    e = cudaFuncSetAttribute(sharq_gemm_persistent_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(sharq_gemm_persistent_kernel<BN, kG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes);
     if (e != cudaSuccess) return e;
     int n = 0;
@@ -1002,7 +1081,19 @@ cudaError_t launch_persistent(const GemmArgs& a, int m_tiles, cudaStream_t strea
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sharq_gemm_persistent_kernel<BN>, a, m_tiles);
+  return cudaLaunchKernelEx(&cfg, sharq_gemm_persistent_kernel<BN, kG>, a, m_tiles);
+}
+
+template <int BN>
+cudaError_t launch_persistent_mode(const GemmArgs& a, int m_tiles, int gmode, cudaStream_t stream) {
+  switch (gmode) {
+    case kGemmSharq: return launch_persistent<BN, kGemmSharq>(a, m_tiles, stream);
+    case kGemmNvfp4: return launch_persistent<BN, kGemmNvfp4>(a, m_tiles, stream);
+    case kGemmSparseOnly: return launch_persistent<BN, kGemmSparseOnly>(a, m_tiles, stream);
+    case kGemmDenseDense: return launch_persistent<BN, kGemmDenseDense>(a, m_tiles, stream);
+    case kGemmSparseSparse: return launch_persistent<BN, kGemmSparseSparse>(a, m_tiles, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int BN, bool kSplit, bool kFused>
@@ -1044,7 +1135,8 @@ extern "C" int sharq_debug_set_trace(void* p) {
 #endif
 
 cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
-                          const uint8_t* a_rsf, const float* s_g, int T, int Tp, int K, int sharq_mode,
+                          const uint8_t* a_rsf, const uint8_t* a_rmeta, const float* s_g, int T, int Tp, int K,
+                          int gmode,
                           const uint8_t* w_codes, const uint8_t* w_sf32, const uint8_t* w_sf16, const float* s_w,
                           int D, int E, const int* group_offsets, void* Y, int out_f32, int bn, int splits,
                           int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
@@ -1055,6 +1147,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.a_spsf = a_spsf;
   a.a_r = a_r;
   a.a_rsf = a_rsf;
+  a.a_rmeta = a_rmeta;
   a.s_g = s_g;
   a.w_codes = w_codes;
   a.w_sf32 = w_sf32;
@@ -1069,7 +1162,8 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.D = D;
   a.E = E;
   a.out_f32 = out_f32;
-  a.sharq_mode = sharq_mode;
+  a.sharq_mode = gmode == kGemmSharq ? 1 : 0;
+  const bool two_way = gmode == kGemmSharq || gmode == kGemmNvfp4;  // the split-K/fused kernels' modes
   a.splits = splits;
   a.per_token = per_token ? 1 : 0;
   a.X = static_cast<const __nv_bfloat16*>(X_fused);
@@ -1078,7 +1172,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   const int m_tiles = Tp / 128;
   if (m_tiles == 0) return cudaSuccess;
   if (X_fused) {  // fused decode form
-    if (T > 32 || m_tiles != 1 || !sharq_mode || group_offsets || per_token) return cudaErrorInvalidValue;
+    if (T > 32 || m_tiles != 1 || gmode != kGemmSharq || group_offsets || per_token) return cudaErrorInvalidValue;
     if (splits > 1) {
       if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
       return launch_cfg<128, true, true>(a, m_tiles, stream);
@@ -1086,11 +1180,15 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
     return bn == 256 ? launch_cfg<256, false, true>(a, m_tiles, stream)
                      : launch_cfg<128, false, true>(a, m_tiles, stream);
   }
-  if (splits > 1) {
+  if (splits > 1 && two_way) {
     if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
     return launch_cfg<128, true, false>(a, m_tiles, stream);
   }
-  return bn == 256 ? launch_persistent<256>(a, m_tiles, stream) : launch_persistent<128>(a, m_tiles, stream);
+  // the Table-5 modes run the persistent form at every size
+  const int pbn = (a.D % 256 == 0) ? 256 : 128;
+  const int use_bn = two_way ? bn : pbn;
+  return use_bn == 256 ? launch_persistent_mode<256>(a, m_tiles, gmode, stream)
+                       : launch_persistent_mode<128>(a, m_tiles, gmode, stream);
 }
 
 }  // namespace sharq

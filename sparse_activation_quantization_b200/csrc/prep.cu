@@ -315,6 +315,36 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
   if (threadIdx.x == 0) depart_and_reset(gmax_bits);
 }
 
+// Two-launch form of the Table-5 operand kinds (Dense+Dense, Sparse+Sparse):
+// after prep_rowstats_kernel, one thread per 32 consecutive K (four runs,
+// every block inside the thread), flat over rows.
+constexpr int kRunsThreads = 256;
+template <int kKind>
+__global__ void __launch_bounds__(kRunsThreads) prep_runs_kernel(
+    const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
+    const int* __restrict__ row_index, int T, int K, const float* __restrict__ inv_rms,
+    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
+  __shared__ float gmax_sh;
+  allow_dependents();
+  const int segs = K >> 5;
+  const long long gid = (long long)blockIdx.x * kRunsThreads + threadIdx.x;
+  if (threadIdx.x == 0) gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
+  __syncthreads();
+  const float gmax = gmax_sh;
+  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
+  if (gid == 0) *s_g_out = s;
+  if (gid < (long long)T * segs) {
+    const int t = (int)(gid / segs);
+    const int c0 = (int)(gid - (long long)t * segs) * 4;
+    const int src = row_index ? row_index[t] : t;
+    float x[32];
+    load_runs<4>(x, X, src, K, c0);
+    if (gamma && src >= 0) normalise_runs<4>(x, gamma, c0, inv_rms[t]);
+    quant_runs<4, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
+  }
+  if (threadIdx.x == 0) depart_and_reset(gmax_bits);
+}
+
 // ---------------------------------------------------------------------------
 // Single-launch form (cooperative grid; whole rows inside a CTA).
 constexpr int kFusedMaxThreads = 1024;
@@ -323,7 +353,7 @@ constexpr uint64_t kBarrierLimitNs = 2000000000ull;
 template <int NC>
 constexpr int fused_max_threads() { return NC == 4 ? 640 : kFusedMaxThreads; }
 
-template <int NC, bool kSharq, bool kPerToken = false>
+template <int NC, int kKind, bool kPerToken = false>
 __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
@@ -398,7 +428,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     for (int w = 0; w < wpr; ++w) m = fmaxf(m, wmax[rl * wpr + w]);
     const float s = m > 0.0f ? __fdiv_rn(m, kGlobalDiv) : 1.0f;
     if (live && li == 0) s_g_out[t] = s;
-    if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
+    if (live) quant_runs<NC, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
     return;
   }
   if (threadIdx.x == 0) {
@@ -432,7 +462,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
   // rows past T: whole warps (rows span whole warps), so they can skip
-  if (live) quant_runs<NC, kSharq>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
+  if (live) quant_runs<NC, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
   if (threadIdx.x == 0 && gridDim.x > 1) depart_and_reset(sync);
 #ifdef SHARQ_TRACE
   __syncthreads();
@@ -458,16 +488,16 @@ void prefer_max_shared(F* fn) {
   cudaGetLastError();
 }
 
-template <int NC, bool kSharq>
+template <int NC, int kKind>
 int fused_max_ctas_t(int threads) {
   static int cache[kFusedMaxThreads + 1][64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
   int& c = cache[threads][dev];
   if (c == 0) {
-    prefer_max_shared(prep_fused_kernel<NC, kSharq>);
+    prefer_max_shared(prep_fused_kernel<NC, kKind>);
     int per_sm = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<NC, kSharq>, threads, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prep_fused_kernel<NC, kKind>, threads, 0) !=
             cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
       cudaGetLastError();
@@ -478,7 +508,7 @@ int fused_max_ctas_t(int threads) {
   return c > 0 ? c : 0;
 }
 
-template <int NC, bool kSharq>
+template <int NC, int kKind>
 cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
                       int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
                       cudaStream_t stream, bool* launched) {
@@ -488,7 +518,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   rpc = rpc < 1 ? 1 : rpc;
   const int threads = rpc * tpr;
   const int ctas = (T + rpc - 1) / rpc;
-  if (ctas > fused_max_ctas_t<NC, kSharq>(threads)) return cudaSuccess;
+  if (ctas > fused_max_ctas_t<NC, kKind>(threads)) return cudaSuccess;
   // A plain launch: the grid fits the GPU at once (checked above), so all
   // CTAs are resident together when the stream reaches this kernel; the
   // GEMM that follows as a programmatic dependent can start only after every
@@ -499,7 +529,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(threads);
   cfg.stream = stream;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kSharq>, Xb, Gb, eps, row_index, T, Tp, K, rpc,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKind>, Xb, Gb, eps, row_index, T, Tp, K, rpc,
                                      inv_rms, sync, s_g, p);
   if (e == cudaSuccess) *launched = true;
   else cudaGetLastError();  // fall back to the two-launch form
@@ -519,18 +549,18 @@ cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb
   cfg.gridDim = dim3((T + rpc - 1) / rpc);
   cfg.blockDim = dim3(rpc * tpr);
   cfg.stream = stream;
-  return cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, true, true>, Xb, Gb, eps, row_index, T, Tp, K, rpc, inv_rms,
+  return cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKindSharq, true>, Xb, Gb, eps, row_index, T, Tp, K, rpc, inv_rms,
                             sync, s_t, p);
 }
 
-template <bool kSharq>
+template <int kKind>
 cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
                           int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
                           cudaStream_t stream, bool* launched) {
   switch (fused_runs_per_thread(K)) {
-    case 1: return try_fused<1, kSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
-    case 2: return try_fused<2, kSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
-    case 4: return try_fused<4, kSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    case 1: return try_fused<1, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    case 2: return try_fused<2, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    case 4: return try_fused<4, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
     default: *launched = false; return cudaSuccess;
   }
 }
@@ -569,13 +599,13 @@ extern "C" int sharq_debug_set_trace_prep(void* p) {
 bool prep_per_token_supported(int K) { return fused_runs_per_thread(K) != 0; }
 
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
-                        int K, bool sharq_mode, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
+                        int K, int kind, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
-                        cudaStream_t stream) {
+                        uint8_t* r_meta, cudaStream_t stream) {
   // gmax_bits[0..3]: device-wide max, barrier arrivals, departures, error
   // word; zero at rest (the kernels reset them), so no memset is needed
   cudaError_t e = cudaSuccess;
-  QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf};
+  QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf, r_meta};
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
   if (per_token) {  // s_g: Tp floats, one per row (SharQ mode only)
@@ -590,10 +620,24 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
 
   if (T > 0) {
     bool launched = false;
-    e = sharq_mode ? try_fused_any<true>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
-                                         &launched)
-                   : try_fused_any<false>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
-                                          &launched);
+    switch (kind) {
+      case kKindNvfp4:
+        e = try_fused_any<kKindNvfp4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream, &launched);
+        break;
+      case kKindSharq:
+        e = try_fused_any<kKindSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream, &launched);
+        break;
+      case kKindDenseDense:
+        e = try_fused_any<kKindDenseDense>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+                                           &launched);
+        break;
+      case kKindSparseSparse:
+        e = try_fused_any<kKindSparseSparse>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+                                             &launched);
+        break;
+      default:
+        return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
     if (launched) return cudaSuccess;
   }
@@ -618,6 +662,18 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
       prep_rowstats_kernel<false><<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms,
                                                                     gmax_bits);
   }
+  if (kind == kKindDenseDense || kind == kKindSparseSparse) {
+    const long long n = (long long)T * (K >> 5);
+    const unsigned grid = n > 0 ? (unsigned)((n + kRunsThreads - 1) / kRunsThreads) : 1u;
+    if (kind == kKindDenseDense)
+      prep_runs_kernel<kKindDenseDense><<<grid, kRunsThreads, 0, stream>>>(Xb, Gb, row_index, T, K, inv_rms,
+                                                                          gmax_bits, s_g, p);
+    else
+      prep_runs_kernel<kKindSparseSparse><<<grid, kRunsThreads, 0, stream>>>(Xb, Gb, row_index, T, K, inv_rms,
+                                                                            gmax_bits, s_g, p);
+    return cudaGetLastError();
+  }
+  const bool sharq_mode = kind == kKindSharq;
   auto strip_fn = sharq_mode ? (g ? prep_strip_kernel<true, true> : prep_strip_kernel<true, false>)
                              : (g ? prep_strip_kernel<false, true> : prep_strip_kernel<false, false>);
   const int G = ((K >> 5) + 31) >> 5;  // strip groups (warps) per row
@@ -663,9 +719,9 @@ static cudaError_t noalloc_scratch(unsigned char** out) {
 }
 
 cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
-                                int K, bool sharq_mode, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
-                                uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, unsigned int* err_out,
-                                cudaStream_t stream) {
+                                int K, int kind, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
+                                uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf, uint8_t* r_meta,
+                                unsigned int* err_out, cudaStream_t stream) {
   if (T > kNoAllocMaxRows) return cudaErrorInvalidValue;
   unsigned char* scr = nullptr;
   cudaError_t e = noalloc_scratch(&scr);
@@ -675,8 +731,8 @@ cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, con
   // the array keeps the last call's contents: start every call from zero
   e = cudaMemsetAsync(sync, 0, 4 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
-  e = launch_prep(X, gamma, eps, row_index, T, Tp, K, sharq_mode, per_token, inv, s_g, sync, sp_codes, meta, sp_sf,
-                  r_codes, r_sf, stream);
+  e = launch_prep(X, gamma, eps, row_index, T, Tp, K, kind, per_token, inv, s_g, sync, sp_codes, meta, sp_sf,
+                  r_codes, r_sf, r_meta, stream);
   if (e != cudaSuccess) return e;
   // forward the error word to where sharq_linear looks for it
   if (err_out) e = cudaMemcpyAsync(err_out, sync + 3, sizeof(unsigned int), cudaMemcpyDeviceToDevice, stream);

@@ -34,6 +34,17 @@ struct QuantPtrs {
   uint8_t* sp_sf;
   uint8_t* r_codes;
   uint8_t* r_sf;
+  uint8_t* r_meta;  // Sparse+Sparse only: the residual's metadata
+};
+
+// How the activation is split into its two FP4 operands (xllm-io review,
+// section 3 for SharQ; section 5.3, Table 5, for the others; plain NVFP4 is
+// the comparator of Table 1).
+enum : int {
+  kKindNvfp4 = 0,        // one dense operand: NVFP4 of Xn
+  kKindSharq = 1,        // sparse backbone + dense residual (also Sparse only: the GEMM drops the residual)
+  kKindDenseDense = 2,   // dense NVFP4 of Xn + dense NVFP4 of its residual
+  kKindSparseSparse = 3  // sparse backbone + sparse (4:8 in-pairs) residual
 };
 
 // max over the `width` adjacent lanes of an aligned lane group
@@ -62,86 +73,93 @@ __device__ __forceinline__ float2 e2m1x2_values(uint32_t byte) {
   return __half22float2(*reinterpret_cast<__half2*>(&h2));
 }
 
-// Quantize NC consecutive runs of 8 logical K of row t, held in registers
-// (x[8*c + e] = run c, element e), starting at run index c0 of the row.
-// NC = 4: every block is inside the thread.  NC = 1, 2: the 32-K block spans
-// 4 / NC adjacent lanes and (NC = 1) the 16-K block 2 lanes; all 32 lanes of
-// the warp must call it then (warp shuffles).
-template <int NC, bool kSharq>
-__device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int c0, int K, float s, float six_s,
-                                           const QuantPtrs& out, bool store = true) {
+// Sparse operand of NC consecutive runs of 8 logical K of row t, held in
+// registers (v[8*c + e] = run c, element e), starting at run c0 of the row:
+// the 4:8 in-pairs mask (keep the 2 of 4 pairs with the largest max|v|, ties
+// to the lower pair), the kept values' NVFP4 codes with one scale per 32
+// logical K, the metadata; out[] = v - f32(val * dec * s) at kept positions
+// and v elsewhere (exact).  Tiles: codes 8 KB (64-byte swizzle), metadata
+// 2 KB, scales 1 KB.  NC = 1, 2: the 32-K block spans 4 / NC adjacent lanes
+// (all 32 lanes of the warp must call it).
+template <int NC>
+__device__ __forceinline__ void sparse_operand(const float (&x)[8 * NC], float (&res)[8 * NC], int t, int c0, int K,
+                                               float s, float six_s, uint8_t* codes_out, uint8_t* meta_out,
+                                               uint8_t* sf_out, bool store) {
   const int KS = K >> 8;
   const int r = t & 127;
-  float res[8 * NC];
 #pragma unroll
   for (int i = 0; i < 8 * NC; ++i) res[i] = x[i];
-
-  if (kSharq) {
-    // --- 4:8 in-pairs mask per run: keep the 2 of 4 pairs with the largest max|x|
-    float v[4 * NC];
-    uint32_t km[NC];
+  float v[4 * NC];
+  uint32_t km[NC];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      float sc[4];
+  for (int c = 0; c < NC; ++c) {
+    float sc[4];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) sc[p] = fmaxf(fabsf(x[8 * c + 2 * p]), fabsf(x[8 * c + 2 * p + 1]));
-      km[c] = keep_mask4(sc);
-      const bool k0 = km[c] & 1u, k1 = km[c] & 2u, k3 = km[c] & 8u;
-      // lowest kept pair (0..2) and highest kept pair (1..3)
-      const float* xc = x + 8 * c;
-      v[4 * c + 0] = k0 ? xc[0] : (k1 ? xc[2] : xc[4]);
-      v[4 * c + 1] = k0 ? xc[1] : (k1 ? xc[3] : xc[5]);
-      v[4 * c + 2] = k3 ? xc[6] : ((km[c] & 4u) ? xc[4] : xc[2]);
-      v[4 * c + 3] = k3 ? xc[7] : ((km[c] & 4u) ? xc[5] : xc[3]);
-    }
-    // --- backbone NVFP4: one scale per 32 logical K (4 runs = 16 kept values)
-    float am = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4 * NC; ++i) am = fmaxf(am, fabsf(v[i]));
-    if (NC < 4) am = group_max(am, 4 / NC);
-    const BlockScale bs = block_scale(am, six_s, s);
-    uint32_t cb[2 * NC];  // code bytes: kept values (2i, 2i+1)
-#pragma unroll
-    for (int i = 0; i < 2 * NC; ++i) cb[i] = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
-    // --- residual R = Xn - dequant(backbone) at kept positions (exact fp32)
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      const float2 lo2 = e2m1x2_values(cb[2 * c]), hi2 = e2m1x2_values(cb[2 * c + 1]);
-      const float t0 = __fmul_rn(__fmul_rn(lo2.x, bs.dec), s), t1 = __fmul_rn(__fmul_rn(lo2.y, bs.dec), s);
-      const float t2 = __fmul_rn(__fmul_rn(hi2.x, bs.dec), s), t3 = __fmul_rn(__fmul_rn(hi2.y, bs.dec), s);
-      const uint32_t m = km[c];
-      const bool k0 = m & 1u, k1 = m & 2u, k2 = m & 4u, k3 = m & 8u;
-      // pair p holds (t0,t1) if it is the lowest kept pair, (t2,t3) if the highest
-      float* rc = res + 8 * c;
-      if (k0) { rc[0] = __fsub_rn(rc[0], t0); rc[1] = __fsub_rn(rc[1], t1); }
-      if (k1) { rc[2] = __fsub_rn(rc[2], k0 ? t2 : t0); rc[3] = __fsub_rn(rc[3], k0 ? t3 : t1); }
-      if (k2) { rc[4] = __fsub_rn(rc[4], k3 ? t0 : t2); rc[5] = __fsub_rn(rc[5], k3 ? t1 : t3); }
-      if (k3) { rc[6] = __fsub_rn(rc[6], t2); rc[7] = __fsub_rn(rc[7], t3); }
-    }
-    // --- stores: per run 2 bytes of kept codes, one metadata nibble
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      const int g = c0 + c;               // run index in the row
-      const int kt = g >> 5, w = g & 31;  // K tile, run within the 256-K tile
-      const size_t tile = (size_t)(t >> 7) * KS + kt;
-      if (store)
-        *reinterpret_cast<uint16_t*>(out.sp_codes + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
-            (uint16_t)(cb[2 * c] | (cb[2 * c + 1] << 8));
-      const uint32_t m = km[c];
-      const uint32_t nib = (uint32_t)((__ffs(m) - 1) | ((31 - __clz(m)) << 2));
-      if (NC == 1) {
-        const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
-        if (store && (w & 1) == 0) out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
-      } else if (store && (c & 1) == 0) {
-        const uint32_t m2 = km[c + 1 < NC ? c + 1 : c];
-        const uint32_t other = (uint32_t)((__ffs(m2) - 1) | ((31 - __clz(m2)) << 2));
-        out.meta[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
-      }
-      if (store && (w & 3) == 0) out.sp_sf[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
-    }
+    for (int p = 0; p < 4; ++p) sc[p] = fmaxf(fabsf(x[8 * c + 2 * p]), fabsf(x[8 * c + 2 * p + 1]));
+    km[c] = keep_mask4(sc);
+    const bool k0 = km[c] & 1u, k1 = km[c] & 2u, k3 = km[c] & 8u;
+    // lowest kept pair (0..2) and highest kept pair (1..3)
+    const float* xc = x + 8 * c;
+    v[4 * c + 0] = k0 ? xc[0] : (k1 ? xc[2] : xc[4]);
+    v[4 * c + 1] = k0 ? xc[1] : (k1 ? xc[3] : xc[5]);
+    v[4 * c + 2] = k3 ? xc[6] : ((km[c] & 4u) ? xc[4] : xc[2]);
+    v[4 * c + 3] = k3 ? xc[7] : ((km[c] & 4u) ? xc[5] : xc[3]);
   }
+  // one scale per 32 logical K (4 runs = 16 kept values)
+  float am = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4 * NC; ++i) am = fmaxf(am, fabsf(v[i]));
+  if (NC < 4) am = group_max(am, 4 / NC);
+  const BlockScale bs = block_scale(am, six_s, s);
+  uint32_t cb[2 * NC];  // code bytes: kept values (2i, 2i+1)
+#pragma unroll
+  for (int i = 0; i < 2 * NC; ++i) cb[i] = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
+  // residual w.r.t. the quantized operand at kept positions (exact fp32)
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const float2 lo2 = e2m1x2_values(cb[2 * c]), hi2 = e2m1x2_values(cb[2 * c + 1]);
+    const float t0 = __fmul_rn(__fmul_rn(lo2.x, bs.dec), s), t1 = __fmul_rn(__fmul_rn(lo2.y, bs.dec), s);
+    const float t2 = __fmul_rn(__fmul_rn(hi2.x, bs.dec), s), t3 = __fmul_rn(__fmul_rn(hi2.y, bs.dec), s);
+    const uint32_t m = km[c];
+    const bool k0 = m & 1u, k1 = m & 2u, k2 = m & 4u, k3 = m & 8u;
+    // pair p holds (t0,t1) if it is the lowest kept pair, (t2,t3) if the highest
+    float* rc = res + 8 * c;
+    if (k0) { rc[0] = __fsub_rn(rc[0], t0); rc[1] = __fsub_rn(rc[1], t1); }
+    if (k1) { rc[2] = __fsub_rn(rc[2], k0 ? t2 : t0); rc[3] = __fsub_rn(rc[3], k0 ? t3 : t1); }
+    if (k2) { rc[4] = __fsub_rn(rc[4], k3 ? t0 : t2); rc[5] = __fsub_rn(rc[5], k3 ? t1 : t3); }
+    if (k3) { rc[6] = __fsub_rn(rc[6], t2); rc[7] = __fsub_rn(rc[7], t3); }
+  }
+  // stores: per run 2 bytes of kept codes, one metadata nibble
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int g = c0 + c;               // run index in the row
+    const int kt = g >> 5, w = g & 31;  // K tile, run within the 256-K tile
+    const size_t tile = (size_t)(t >> 7) * KS + kt;
+    if (store)
+      *reinterpret_cast<uint16_t*>(codes_out + tile * kSpTile + sp_chunk_off(r, w >> 3) + 2 * (w & 7)) =
+          (uint16_t)(cb[2 * c] | (cb[2 * c + 1] << 8));
+    const uint32_t m = km[c];
+    const uint32_t nib = (uint32_t)((__ffs(m) - 1) | ((31 - __clz(m)) << 2));
+    if (NC == 1) {
+      const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
+      if (store && (w & 1) == 0) meta_out[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
+    } else if (store && (c & 1) == 0) {
+      const uint32_t m2 = km[c + 1 < NC ? c + 1 : c];
+      const uint32_t other = (uint32_t)((__ffs(m2) - 1) | ((31 - __clz(m2)) << 2));
+      meta_out[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
+    }
+    if (store && (w & 3) == 0) sf_out[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
+  }
+}
 
-  // --- dense NVFP4 of R (or of Xn in NVFP4 mode): 16-element blocks
+// Dense operand: NVFP4 of v in 16-element blocks; with kDeq, deq[] receives
+// f32(val * dec * s) of every element.  Tiles: codes 16 KB (128-byte
+// swizzle), scales 2 KB.  NC = 1: the 16-K block spans 2 adjacent lanes.
+template <int NC, bool kDeq>
+__device__ __forceinline__ void dense_operand(const float (&res)[8 * NC], float (&deq)[8 * NC], int t, int c0, int K,
+                                              float s, float six_s, uint8_t* codes_out, uint8_t* sf_out, bool store) {
+  const int KS = K >> 8;
+  const int r = t & 127;
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     if (NC > 1 && (c & 1)) continue;  // the even run handles its block of two runs
@@ -155,18 +173,50 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
     for (int h = 0; h < nr; ++h) {
       uint32_t word = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        word |= cvt_e2m1x2(__fmul_rn(res[8 * (c + h) + 2 * i], bs.inv), __fmul_rn(res[8 * (c + h) + 2 * i + 1], bs.inv))
-                << (8 * i);
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t b = cvt_e2m1x2(__fmul_rn(res[8 * (c + h) + 2 * i], bs.inv),
+                                      __fmul_rn(res[8 * (c + h) + 2 * i + 1], bs.inv));
+        word |= b << (8 * i);
+        if (kDeq) {
+          const float2 q = e2m1x2_values(b);
+          deq[8 * (c + h) + 2 * i] = __fmul_rn(__fmul_rn(q.x, bs.dec), s);
+          deq[8 * (c + h) + 2 * i + 1] = __fmul_rn(__fmul_rn(q.y, bs.dec), s);
+        }
+      }
       const int g = c0 + c + h;
       const int kt = g >> 5, w = g & 31;
       const size_t tile = (size_t)(t >> 7) * KS + kt;
       if (store) {
-        *reinterpret_cast<uint32_t*>(out.r_codes + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
+        *reinterpret_cast<uint32_t*>(codes_out + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
             word;
-        if ((w & 1) == 0) out.r_sf[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+        if ((w & 1) == 0) sf_out[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
       }
     }
+  }
+}
+
+// Quantize NC consecutive runs of 8 logical K of row t into the two operands
+// of kKind (see the enum).  NC = 4: every block is inside the thread; NC = 1,
+// 2: blocks span adjacent lanes and all 32 lanes of the warp must call it.
+template <int NC, int kKind>
+__device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int c0, int K, float s, float six_s,
+                                           const QuantPtrs& out, bool store = true) {
+  float res[8 * NC];
+  if (kKind == kKindNvfp4) {
+    dense_operand<NC, false>(x, res, t, c0, K, s, six_s, out.r_codes, out.r_sf, store);
+  } else if (kKind == kKindSharq) {
+    sparse_operand<NC>(x, res, t, c0, K, s, six_s, out.sp_codes, out.meta, out.sp_sf, store);
+    dense_operand<NC, false>(res, res, t, c0, K, s, six_s, out.r_codes, out.r_sf, store);
+  } else if (kKind == kKindDenseDense) {
+    float deq[8 * NC];
+    dense_operand<NC, true>(x, deq, t, c0, K, s, six_s, out.sp_codes, out.sp_sf, store);
+#pragma unroll
+    for (int i = 0; i < 8 * NC; ++i) res[i] = __fsub_rn(x[i], deq[i]);
+    dense_operand<NC, false>(res, deq, t, c0, K, s, six_s, out.r_codes, out.r_sf, store);
+  } else {
+    float res2[8 * NC];
+    sparse_operand<NC>(x, res, t, c0, K, s, six_s, out.sp_codes, out.meta, out.sp_sf, store);
+    sparse_operand<NC>(res, res2, t, c0, K, s, six_s, out.r_codes, out.r_meta, out.r_sf, store);
   }
 }
 
