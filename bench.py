@@ -410,7 +410,44 @@ def run_gpu(args, world, rank, local):
         dist.all_reduce(t_, op=dist.ReduceOp.MAX)
         e2e_ms = t_.item()
 
-    # --- comparators on the same box: plain NVFP4 (dense FP4 GEMM only, same
+    # --- every activation mode of the library on one layer: prep + GEMM time,
+    # and the relative Frobenius error of Y (float32 output) against the
+    # unquantized float32 product Xn W (weight quantization included, the
+    # same for every mode) on the first input copy
+    MODES = {"sharq": sq.SHARQ_MODE_SHARQ, "nvfp4": sq.SHARQ_MODE_NVFP4, "sharq_per_token": sq.SHARQ_MODE_SHARQ_TOKEN,
+             "sparse_only": sq.SHARQ_MODE_SPARSE_ONLY, "dense_dense": sq.SHARQ_MODE_DENSE_DENSE,
+             "sparse_sparse": sq.SHARQ_MODE_SPARSE_SPARSE}
+
+    def mode_table(L, li, src, W0):
+        x0 = xs[src][0].float()
+        if gammas[src] is not None:
+            ss = (xs[src][0].double() ** 2).sum(dim=1)
+            inv = (1.0 / torch.sqrt(ss / L.K + float(torch.tensor(EPS, dtype=torch.float32)))).float()
+            xn = ((x0 * inv[:, None]) * gammas[src].float()).to(torch.bfloat16).float()
+        else:
+            xn = x0
+        torch.backends.cuda.matmul.allow_tf32 = False  # a true float32 reference product
+        yref = xn @ W0.float()
+        y32 = torch.empty((L.T, L.D), dtype=torch.float32, device=dev)
+        out = {}
+        for name, mode in MODES.items():
+            try:
+                a_m = sq.PreparedAct(L.T, L.K, mode=mode, device=dev)
+            except Exception as e:  # a shape the mode does not support
+                out[name] = {"unsupported": str(e)}
+                continue
+            us = kernel_us(lambda i: (a_m.prep(xs[src][i], gammas[src], EPS, stream=stream),
+                                      sq.linear(a_m, weights[L.name][i], out=outs[L.name], ws=wss[L.name],
+                                                stream=stream)), n_rot, stream)
+            a_m.prep(xs[src][0], gammas[src], EPS, stream=stream)
+            sq.linear(a_m, weights[L.name][0], out_dtype=torch.float32, out=y32, ws=wss[L.name], stream=stream)
+            torch.cuda.synchronize()
+            err = (torch.linalg.norm(y32 - yref) / torch.linalg.norm(yref)).item()
+            out[name] = {"layer_us": round(us, 3), "y_rel_err": round(err, 5)}
+            del a_m
+        return out
+
+    # --- comparators on the same box: plain NVFP4 (dense FP4 GEMM only, same    # --- comparators on the same box: plain NVFP4 (dense FP4 GEMM only, same
     # kernels in SHARQ_MODE_NVFP4) and bf16 cuBLAS (torch.matmul) ---------
     comparators = None
     if args.compare:
@@ -427,7 +464,8 @@ def run_gpu(args, world, rank, local):
             ob = torch.empty((L.T, L.D), dtype=torch.bfloat16, device=dev)
             bf = kernel_us(lambda i, L=L: torch.matmul(xs[src][i], Wb[i % len(Wb)], out=ob), n_rot, stream)
             comparators[L.name] = {"sharq_layer_us": round(per[L.name]["layer_us"], 3),
-                                   "nvfp4_layer_us": round(nv, 3), "bf16_cublas_us": round(bf, 3)}
+                                   "nvfp4_layer_us": round(nv, 3), "bf16_cublas_us": round(bf, 3),
+                                   "modes": mode_table(L, li, src, Wb[0])}
             del Wb, act_n
 
     flops_step = sum(L.flops for L in layers)
