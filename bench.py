@@ -62,7 +62,10 @@ def prep_alg_bytes(T, K):
 # kernel per launch, from the ncu capture summarised in
 # profiles/sharq_gemm_qproj_decode.md; reset to None whenever that kernel
 # changes until it is captured again.
-NCU_TRAFFIC = {"q_proj_T128": None}
+# DRAM bytes (read + write) per launch of the dominant GEMM, from ncu captures
+# of this script's workloads (profiles/sharq_gemm_qproj_decode.md,
+# profiles/sharq_gemm_persistent_mlp2048.md); None where none was taken.
+NCU_TRAFFIC = {"q_proj_T128": 10470912, "gate_T2048": 65486592, "up_T2048": 65486592}
 
 
 def read_peaks():
@@ -478,7 +481,7 @@ def run_gpu(args, world, rank, local):
                 "achieved": per[dom.name]["gemm_tflops"], "peak": pk["effective_pflops"] * 1e3,
                 "unit": "TFLOP/s", "frac": per[dom.name]["gemm_tflops"] / (pk["effective_pflops"] * 1e3),
                 "peak_kind": "measured tcgen05 FP4 (dense %.2f, sparse %.2f PFLOP/s; dual-GEMM effective)"
-                             % (pk["dense_pflops"], pk["sparse_pflops"]), "traffic": None}
+                             % (pk["dense_pflops"], pk["sparse_pflops"]), "traffic": NCU_TRAFFIC.get(dom.name)}
     else:
         peak_gbs, peak_kind = read_peaks()
         ach = per[dom.name]["gemm_gbs"]
