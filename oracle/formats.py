@@ -92,6 +92,36 @@ def e4m3_encode_nonneg(x):
 # ---------------------------------------------------------------- bf16 -----
 
 
+# ---------------------------------------------------------------- E8M0 -----
+# The MX scale type (OCP Microscaling Formats specification v1.0, "E8M0"):
+# 8 exponent bits, bias 127, no sign, no mantissa; 0xFF is NaN.  Byte e is
+# 2^(e - 127).  MXFP4 (the same specification) is 32 E2M1 elements sharing
+# one E8M0 scale X = 2^(floor(log2(amax)) - emax_elem), emax_elem = 2 for
+# E2M1 (largest normal 6 = 1.5 * 2^2); the elements are x / X rounded to
+# E2M1 (round to nearest even, saturating).
+
+
+def e8m0_decode(b):
+    """Value of each E8M0 byte (array of ints 0..254) as float64."""
+    b = np.asarray(b, dtype=np.int64)
+    return np.ldexp(1.0, b - 127)
+
+
+def mx_scale_exponent(amax):
+    """Shared exponent of an MX block from its float32 amax: floor(log2(amax))
+    - 2, clamped to the E8M0 range [-127, 127]; -127 for an all-zero block.
+    floor(log2) is read off the float32 encoding exactly (no logarithm)."""
+    a = np.asarray(amax, dtype=np.float32)
+    bits = a.view(np.uint32).astype(np.int64)
+    e_field = (bits >> 23) & 0xFF
+    mant = bits & 0x7FFFFF
+    # normal: e_field - 127; subnormal: position of the highest mantissa bit
+    sub = np.where(mant > 0, np.floor(np.log2(np.maximum(mant, 1))).astype(np.int64) - 149, -1000)
+    fl = np.where(e_field > 0, e_field - 127, sub)
+    e = np.where(a > 0, fl - 2, -127)
+    return np.clip(e, -127, 127)
+
+
 def bf16_round(x):
     """Round float32 to the nearest bfloat16 (ties to even); returns float32.
 

@@ -26,7 +26,7 @@ bytes comparable bit for bit:
 import numpy as np
 
 from .formats import (bf16_round, e2m1_decode, e2m1_encode, e4m3_decode,
-                      e4m3_encode_nonneg, f32)
+                      e4m3_encode_nonneg, f32, e8m0_decode, mx_scale_exponent)
 
 E2M1_MAX = 6.0
 E4M3_MAX = 448.0
@@ -367,6 +367,90 @@ def linear_mode(p, wq, mode):
     else:
         raise ValueError(mode)
     return y * (_row_scale(p["s_g"], y.shape[0]) * np.float64(wq["s_w"]))
+
+
+# ------------------------------------------------------------- MXFP4 -----
+# The xllm-io review (section 5.3, "FP4 format generalisation") runs SharQ on
+# NVFP4, HiF4 and MXFP4.  MXFP4 is the OCP Microscaling format: E2M1 elements,
+# one E8M0 (power-of-two) scale per 32 elements, no second-level scale.  The
+# pages pair MXFP4 with 2:4 sparsity; the sparse FP4 MMA of sm_100 takes only
+# the 4:8 in-pairs pattern, so the backbone keeps the 4:8 in-pairs mask, and
+# its scale covers 64 logical K (32 kept values), the granularity of that
+# MMA for E8M0 scales; the dense residual uses the MXFP4 32-element blocks.
+
+def mx_quant(v):
+    """MXFP4 quantization of blocks (last axis): X = 2^e, e = floor(log2
+    amax) - 2 (E8M0 byte e + 127), codes = E2M1(v / X) with round to nearest
+    even and saturation, deq = f32(val * X) (exact).  Returns (codes, sb,
+    deq)."""
+    v = np.asarray(v, dtype=np.float32)
+    e = mx_scale_exponent(np.max(np.abs(v), axis=-1))
+    y = (v.astype(np.float64) * np.ldexp(1.0, -e)[..., None]).astype(np.float32)
+    codes = e2m1_encode(y)
+    deq = f32(e2m1_decode(codes) * np.ldexp(1.0, e)[..., None])
+    return codes, (e + 127).astype(np.uint8), deq
+
+
+def prep_mxfp4(x, gamma=None, eps=1e-5):
+    """SharQ with MXFP4 operands: RMSNorm, the 4:8 in-pairs mask, the kept
+    values quantized with one E8M0 scale per 64 logical K, the residual
+    R = Xn - X~_sp (exact) in MXFP4 32-element blocks.  s_g = 1 (MX formats
+    have no tensor scale).  Same keys as prep()."""
+    xn, inv = rmsnorm(x, gamma, eps)
+    T, K = xn.shape
+    keep, meta = pair_mask(xn)
+    keep_el = np.repeat(keep, 2, axis=-1).reshape(T, K)
+    xsp = np.where(keep_el, xn, np.float32(0)).astype(np.float32)
+    sp_vals = xn[keep_el].reshape(T, K // 2)
+    codes, sb, deq = mx_quant(sp_vals.reshape(T, K // 64, 32))
+    xsp_t = np.zeros((T, K), dtype=np.float32)
+    xsp_t[keep_el] = deq.reshape(-1)
+    r = np.where(keep_el, (xn - xsp_t).astype(np.float32), xn).astype(np.float32)
+    rc, rsb, rdeq = mx_quant(r.reshape(T, K // 32, 32))
+    return dict(xn=xn, inv=inv, s_g=np.float32(1.0), gmax=None, keep=keep, meta=meta, sp_vals=sp_vals,
+                sp_codes=codes.reshape(T, K // 2), sp_sf=sb, xsp=xsp, xsp_t=xsp_t, r=r, r_codes=rc.reshape(T, K),
+                r_sf=rsb, r_t=rdeq.reshape(T, K))
+
+
+def prep_mxfp4_plain(x, gamma=None, eps=1e-5):
+    """Plain MXFP4 of Xn (32-element blocks), the MXFP4 comparator.  Returns
+    dict xn, inv, s_g (= 1), codes [T,K], sf [T,K/32], x_t."""
+    xn, inv = rmsnorm(x, gamma, eps)
+    T, K = xn.shape
+    c, sb, deq = mx_quant(xn.reshape(T, K // 32, 32))
+    return dict(xn=xn, inv=inv, s_g=np.float32(1.0), codes=c.reshape(T, K), sf=sb, x_t=deq.reshape(T, K))
+
+
+def pack_weight_mx(w):
+    """The shared weight payload in MXFP4: W in R^{K x D} quantized per
+    output column with one E8M0 scale per 64 K (the sparse path's
+    granularity); the dense path's per-32 view repeats each scale byte.
+    Returns codes [D,K], sf64 [D,K/64], sf32 [D,K/32], s_w = 1, w_t [K,D]
+    dequantized (float64)."""
+    w = np.asarray(w, dtype=np.float32)
+    K, D = w.shape
+    c, sb, deq = mx_quant(w.T.reshape(D, K // 64, 64))
+    return dict(codes=c.reshape(D, K), sf64=sb, sf32=np.repeat(sb, 2, axis=-1), s_w=np.float32(1.0),
+                w_t=deq.reshape(D, K).T.astype(np.float64))
+
+
+def linear_mx(p, wq):
+    """Float64 GEMM of MXFP4-SharQ (or of the plain MXFP4 comparator when p
+    has "codes"): each operand's dequantized values times the weight view it
+    is paired with (per-64 for the backbone, per-32 for dense operands)."""
+    K, D = wq["w_t"].shape
+    T = p["xn"].shape[0]
+    w64 = (e2m1_decode(wq["codes"]).reshape(D, K // 64, 64) * e8m0_decode(wq["sf64"])[..., None]).reshape(D, K).T
+    w32 = (e2m1_decode(wq["codes"]).reshape(D, K // 32, 32) * e8m0_decode(wq["sf32"])[..., None]).reshape(D, K).T
+    if "codes" in p:  # plain MXFP4
+        a = (e2m1_decode(p["codes"]).reshape(T, K // 32, 32) * e8m0_decode(p["sf"])[..., None]).reshape(T, K)
+        return a @ w32
+    vals = (e2m1_decode(p["sp_codes"]).reshape(T, K // 64, 32) * e8m0_decode(p["sp_sf"])[..., None]).reshape(T, K // 2)
+    keep_el = np.repeat(p["keep"], 2, axis=-1).reshape(T, K)
+    a_sp = np.zeros((T, K), dtype=np.float64)
+    a_sp[keep_el] = vals.reshape(-1)
+    a_r = (e2m1_decode(p["r_codes"]).reshape(T, K // 32, 32) * e8m0_decode(p["r_sf"])[..., None]).reshape(T, K)
+    return a_sp @ w64 + a_r @ w32
 
 
 def prep_nvfp4(x, gamma=None, eps=1e-5):
