@@ -90,6 +90,25 @@ enum { SHARQ_MODE_SHARQ = 0, SHARQ_MODE_NVFP4 = 1, SHARQ_MODE_SHARQ_TOKEN = 2 };
  * are not accepted by sharq_prep_linear. */
 enum { SHARQ_MODE_SPARSE_ONLY = 3, SHARQ_MODE_DENSE_DENSE = 4, SHARQ_MODE_SPARSE_SPARSE = 5 };
 
+/* MXFP4 (xllm-io review, section 5.3: SharQ on the NVFP4, HiF4 and MXFP4
+ * formats).  MXFP4 is the OCP Microscaling format: E2M1 elements and one E8M0
+ * (power-of-two) scale X = 2^(floor(log2 amax) - 2) per block, no tensor
+ * scale (s_g = 1, s_w = 1).  The pages pair MXFP4 with 2:4 sparsity; the
+ * sparse FP4 MMA of sm_100 takes the 4:8 in-pairs pattern, so:
+ *   MXFP4        the SharQ decomposition in MXFP4: 4:8 in-pairs backbone with
+ *                one E8M0 scale per 64 logical K (sp_sf: 512-byte tiles, one
+ *                atom), dense MXFP4 residual with one per 32 K (r_sf: 1024-
+ *                byte tiles).
+ *   MXFP4_PLAIN  plain MXFP4 of Xn (r_codes, r_sf as above), the comparator.
+ * Both need a weight packed in SHARQ_FMT_MXFP4. */
+enum { SHARQ_MODE_MXFP4 = 6, SHARQ_MODE_MXFP4_PLAIN = 7 };
+
+/* Weight payload format.  NVFP4: E4M3 scales, sparse view per 32 K, dense
+ * view per 16 K, FP32 s_w.  MXFP4: E8M0 scales per 64 K (the sparse MXFP4
+ * MMA's granularity) in sf32 (512-byte tiles), the dense view per 32 K in sf16
+ * (1024-byte tiles, each byte twice), s_w = 1. */
+enum { SHARQ_FMT_NVFP4 = 0, SHARQ_FMT_MXFP4 = 1 };
+
 /* Tile geometry of every packed operand: 128 rows x 256 logical K. */
 #define SHARQ_TILE_ROWS 128
 #define SHARQ_TILE_K 256
@@ -116,6 +135,7 @@ typedef struct {
   void *sf16;
   float *s_w;
   int K, D, E;
+  int fmt; /* SHARQ_FMT_NVFP4 (set by sharq_weight_view) or SHARQ_FMT_MXFP4 */
 } sharq_weight;
 
 /*
@@ -162,7 +182,9 @@ typedef struct {
 } sharq_act;
 
 /* Host-only size queries (pure functions; 0 on invalid shape). */
-size_t sharq_weight_bytes(int K, int D, int E);
+size_t sharq_weight_bytes(int K, int D, int E); /* SHARQ_FMT_NVFP4 */
+/* Bytes of a packed weight in format fmt (SHARQ_FMT_*); 0 on an invalid shape or format. */
+size_t sharq_weight_bytes_fmt(int K, int D, int E, int fmt);
 size_t sharq_act_bytes(int T, int K, int mode);
 /* Workspace of sharq_linear (E = 1) / sharq_linear_grouped (E experts):
  * the device-side error word (256 bytes reserved).  The caller zeroes it
@@ -171,7 +193,11 @@ size_t sharq_workspace_bytes(int T, int K, int D, int E);
 
 /* Carve the views of a caller-owned device buffer of at least the size
  * returned above (no device access). */
-int sharq_weight_view(void *d_buf, int K, int D, int E, sharq_weight *out);
+int sharq_weight_view(void *d_buf, int K, int D, int E, sharq_weight *out); /* SHARQ_FMT_NVFP4 */
+/* Views of a weight buffer in format fmt; sharq_pack_weight packs in w->fmt.
+ * Errors: SHARQ_ERR_INVALID_ARG (null, misaligned, unknown fmt),
+ * SHARQ_ERR_UNSUPPORTED_SHAPE. */
+int sharq_weight_view_fmt(void *d_buf, int K, int D, int E, int fmt, sharq_weight *out);
 int sharq_act_view(void *d_buf, int T, int K, int mode, sharq_act *out);
 
 /*

@@ -16,7 +16,9 @@ import os
 __all__ = [
     "SharqError", "SharqAct", "SharqWeight", "lib", "library_path",
     "SHARQ_MODE_SHARQ", "SHARQ_MODE_NVFP4", "SHARQ_MODE_SHARQ_TOKEN", "SHARQ_MODE_SPARSE_ONLY",
-    "SHARQ_MODE_DENSE_DENSE", "SHARQ_MODE_SPARSE_SPARSE", "SHARQ_OUT_BF16", "SHARQ_OUT_F32",
+    "SHARQ_MODE_DENSE_DENSE", "SHARQ_MODE_SPARSE_SPARSE", "SHARQ_MODE_MXFP4", "SHARQ_MODE_MXFP4_PLAIN",
+    "SHARQ_FMT_NVFP4", "SHARQ_FMT_MXFP4", "SHARQ_OUT_BF16", "SHARQ_OUT_F32",
+    "sharq_weight_bytes_fmt", "sharq_weight_view_fmt",
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes",
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
@@ -30,6 +32,10 @@ SHARQ_MODE_SHARQ_TOKEN = 2
 SHARQ_MODE_SPARSE_ONLY = 3
 SHARQ_MODE_DENSE_DENSE = 4
 SHARQ_MODE_SPARSE_SPARSE = 5
+SHARQ_MODE_MXFP4 = 6
+SHARQ_MODE_MXFP4_PLAIN = 7
+SHARQ_FMT_NVFP4 = 0
+SHARQ_FMT_MXFP4 = 1
 SHARQ_OUT_BF16 = 0
 SHARQ_OUT_F32 = 1
 
@@ -37,7 +43,7 @@ EXPORTED_SYMBOLS = (
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes", "sharq_weight_view",
     "sharq_act_view", "sharq_pack_weight", "sharq_prep", "sharq_linear", "sharq_linear_grouped",
     "sharq_check_status", "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
-    "sharq_prep_linear",
+    "sharq_prep_linear", "sharq_weight_bytes_fmt", "sharq_weight_view_fmt",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -54,7 +60,8 @@ class SharqError(RuntimeError):
 
 class SharqWeight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("sf32", ctypes.c_void_p), ("sf16", ctypes.c_void_p),
-                ("s_w", ctypes.c_void_p), ("K", ctypes.c_int), ("D", ctypes.c_int), ("E", ctypes.c_int)]
+                ("s_w", ctypes.c_void_p), ("K", ctypes.c_int), ("D", ctypes.c_int), ("E", ctypes.c_int),
+                ("fmt", ctypes.c_int)]
 
 
 class SharqAct(ctypes.Structure):
@@ -80,6 +87,8 @@ def lib():
             "sharq_act_bytes": (sz, [i, i, i]),
             "sharq_workspace_bytes": (sz, [i, i, i, i]),
             "sharq_weight_view": (i, [vp, i, i, i, W]),
+            "sharq_weight_bytes_fmt": (sz, [i, i, i, i]),
+            "sharq_weight_view_fmt": (i, [vp, i, i, i, i, W]),
             "sharq_act_view": (i, [vp, i, i, i, A]),
             "sharq_pack_weight": (i, [vp, W, vp]),
             "sharq_prep": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
@@ -118,6 +127,10 @@ def sharq_weight_bytes(K, D, E=1):
     return lib().sharq_weight_bytes(K, D, E)
 
 
+def sharq_weight_bytes_fmt(K, D, E=1, fmt=SHARQ_FMT_NVFP4):
+    return lib().sharq_weight_bytes_fmt(K, D, E, fmt)
+
+
 def sharq_act_bytes(T, K, mode=SHARQ_MODE_SHARQ):
     return lib().sharq_act_bytes(T, K, mode)
 
@@ -129,6 +142,12 @@ def sharq_workspace_bytes(T, K, D, E=1):
 def sharq_weight_view(d_buf, K, D, E=1):
     w = SharqWeight()
     _check(lib().sharq_weight_view(d_buf, K, D, E, ctypes.byref(w)), "sharq_weight_view")
+    return w
+
+
+def sharq_weight_view_fmt(d_buf, K, D, E=1, fmt=SHARQ_FMT_NVFP4):
+    w = SharqWeight()
+    _check(lib().sharq_weight_view_fmt(d_buf, K, D, E, fmt, ctypes.byref(w)), "sharq_weight_view_fmt")
     return w
 
 
@@ -192,20 +211,21 @@ def _buffer(nbytes, device):
 class PackedWeight:
     """Device buffer + view of a packed weight (sharq_pack_weight).
 
-    W: bf16 CUDA tensor [K, D] (or [E, K, D] for grouped experts)."""
+    W: bf16 CUDA tensor [K, D] (or [E, K, D] for grouped experts); fmt:
+    SHARQ_FMT_NVFP4 or SHARQ_FMT_MXFP4 (for the MXFP4 activation modes)."""
 
-    def __init__(self, W, stream=None):
+    def __init__(self, W, stream=None, fmt=SHARQ_FMT_NVFP4):
         torch = _torch()
         if W.dtype != torch.bfloat16 or not W.is_cuda:
             raise TypeError("W must be a bf16 CUDA tensor")
         W = W.contiguous()
         E, K, D = (1, *W.shape) if W.dim() == 2 else W.shape
-        self.K, self.D, self.E = K, D, E
-        nbytes = sharq_weight_bytes(K, D, E)
+        self.K, self.D, self.E, self.fmt = K, D, E, fmt
+        nbytes = sharq_weight_bytes_fmt(K, D, E, fmt)
         if nbytes == 0:
-            raise SharqError(-2, "sharq_weight_bytes")
+            raise SharqError(-2, "sharq_weight_bytes_fmt")
         self.buf = _buffer(nbytes, W.device)
-        self.view = sharq_weight_view(self.buf.data_ptr(), K, D, E)
+        self.view = sharq_weight_view_fmt(self.buf.data_ptr(), K, D, E, fmt)
         sharq_pack_weight(W.data_ptr(), self.view, _stream_ptr(stream))
 
     def s_w(self):

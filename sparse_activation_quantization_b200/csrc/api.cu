@@ -16,6 +16,8 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
                         uint8_t* r_meta, cudaStream_t stream);
 cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf32, uint8_t* sf16,
                                float* s_w, unsigned int* amax_bits, cudaStream_t stream);
+cudaError_t launch_pack_weight_mx(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf64, uint8_t* sf32,
+                                  float* s_w, cudaStream_t stream);
 cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint8_t* a_spsf, const uint8_t* a_r,
                           const uint8_t* a_rsf, const uint8_t* a_rmeta, const float* s_g, int T, int Tp, int K,
                           int gmode,
@@ -48,10 +50,11 @@ bool shape_ok_d(int D) { return D > 0 && D <= kMaxD && D % 128 == 0; }
 bool shape_ok_t(int T) { return T >= 0 && T <= kMaxT; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool mode_ok(int mode) { return mode >= SHARQ_MODE_SHARQ && mode <= SHARQ_MODE_SPARSE_SPARSE; }
+bool mode_ok(int mode) { return mode >= SHARQ_MODE_SHARQ && mode <= SHARQ_MODE_MXFP4_PLAIN; }
+bool mode_is_mx(int mode) { return mode == SHARQ_MODE_MXFP4 || mode == SHARQ_MODE_MXFP4_PLAIN; }
 // operand sets per mode: first operand (sp_codes/meta/sp_sf) sparse or dense,
 // second operand (r_codes/r_sf, r_meta) dense or sparse
-bool has_first(int mode) { return mode != SHARQ_MODE_NVFP4; }
+bool has_first(int mode) { return mode != SHARQ_MODE_NVFP4 && mode != SHARQ_MODE_MXFP4_PLAIN; }
 bool first_sparse(int mode) { return has_first(mode) && mode != SHARQ_MODE_DENSE_DENSE; }
 bool second_sparse(int mode) { return mode == SHARQ_MODE_SPARSE_SPARSE; }
 // prep operand kind (csrc/quant.cuh) and GEMM operand set (csrc/gemm.cu)
@@ -60,6 +63,8 @@ int prep_kind(int mode) {
     case SHARQ_MODE_NVFP4: return 0;
     case SHARQ_MODE_DENSE_DENSE: return 2;
     case SHARQ_MODE_SPARSE_SPARSE: return 3;
+    case SHARQ_MODE_MXFP4: return 4;
+    case SHARQ_MODE_MXFP4_PLAIN: return 5;
     default: return 1;  // SHARQ, SHARQ_TOKEN, SPARSE_ONLY
   }
 }
@@ -69,6 +74,8 @@ int gemm_mode(int mode) {
     case SHARQ_MODE_SPARSE_ONLY: return 2;
     case SHARQ_MODE_DENSE_DENSE: return 3;
     case SHARQ_MODE_SPARSE_SPARSE: return 4;
+    case SHARQ_MODE_MXFP4: return 5;
+    case SHARQ_MODE_MXFP4_PLAIN: return 6;
     default: return 0;  // SHARQ, SHARQ_TOKEN
   }
 }
@@ -83,14 +90,18 @@ ActLayout act_layout(int T, int K, int mode) {
   const size_t tiles = (Tp / 128) * (size_t)(K / 256);
   size_t off = 0;
   const bool s2 = second_sparse(mode);
+  // scale tiles: NVFP4 sparse operand 1 KB (per 32 logical K), dense 2 KB
+  // (per 16); MXFP4 sparse 512 B (per 64 logical K), dense 1 KB (per 32)
+  const size_t sf_sp = mode_is_mx(mode) ? sharq::kSf64Tile : sharq::kSf32Tile;
+  const size_t sf_dn = mode_is_mx(mode) ? sharq::kSf32Tile : sharq::kSf16Tile;
   L.r_codes = off; off += tiles * (s2 ? sharq::kSpTile : sharq::kCodesTile);
-  L.r_sf = off;    off += tiles * (s2 ? sharq::kSf32Tile : sharq::kSf16Tile);
+  L.r_sf = off;    off += tiles * (s2 ? sf_sp : sf_dn);
   L.sp_codes = off;
   if (has_first(mode)) off += tiles * (first_sparse(mode) ? sharq::kSpTile : sharq::kCodesTile);
   L.meta = off;
   if (first_sparse(mode)) off += tiles * sharq::kMetaTile;
   L.sp_sf = off;
-  if (has_first(mode)) off += tiles * (first_sparse(mode) ? sharq::kSf32Tile : sharq::kSf16Tile);
+  if (has_first(mode)) off += round_up(tiles * (first_sparse(mode) ? sf_sp : sf_dn), 16);
   L.r_meta = off;
   if (s2) off += tiles * sharq::kMetaTile;
   L.inv = off;     off = round_up(off + Tp * sizeof(float), kAlign);
@@ -104,13 +115,16 @@ ActLayout act_layout(int T, int K, int mode) {
 struct WeightLayout {
   size_t codes, sf32, sf16, s_w, scratch, total;
 };
-WeightLayout weight_layout(int K, int D, int E) {
+// fmt: SHARQ_FMT_NVFP4 (sparse view per 32 K, dense view per 16) or
+// SHARQ_FMT_MXFP4 (sparse view per 64 K, dense view per 32)
+WeightLayout weight_layout(int K, int D, int E, int fmt = SHARQ_FMT_NVFP4) {
   WeightLayout L{};
   const size_t tiles = (size_t)E * (D / 128) * (K / 256);
+  const bool mx = fmt == SHARQ_FMT_MXFP4;
   size_t off = 0;
   L.codes = off; off += tiles * sharq::kCodesTile;
-  L.sf32 = off;  off += tiles * sharq::kSf32Tile;
-  L.sf16 = off;  off += tiles * sharq::kSf16Tile;
+  L.sf32 = off;  off += tiles * (mx ? sharq::kSf64Tile : sharq::kSf32Tile);
+  L.sf16 = off;  off += tiles * (mx ? sharq::kSf32Tile : sharq::kSf16Tile);
   L.s_w = off;   off = round_up(off + (size_t)E * sizeof(float), kAlign);
   L.scratch = off; off = round_up(off + (size_t)E * sizeof(unsigned), kAlign);
   L.total = off;
@@ -182,6 +196,7 @@ int weight_ok(const sharq_weight* w) {
   if (!shape_ok_k(w->K) || !shape_ok_d(w->D) || w->E < 1 || w->E > kMaxE) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if (!w->codes || !w->sf32 || !w->sf16 || !w->s_w) return SHARQ_ERR_INVALID_ARG;
   if (!aligned(w->codes, 16) || !aligned(w->sf32, 16) || !aligned(w->sf16, 16)) return SHARQ_ERR_INVALID_ARG;
+  if (w->fmt != SHARQ_FMT_NVFP4 && w->fmt != SHARQ_FMT_MXFP4) return SHARQ_ERR_INVALID_ARG;
   return SHARQ_OK;
 }
 
@@ -191,6 +206,7 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
   if (st) return st;
   if ((st = weight_ok(w))) return st;
   if (a->K != w->K) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (mode_is_mx(a->mode) != (w->fmt == SHARQ_FMT_MXFP4)) return SHARQ_ERR_INVALID_ARG;  // formats must match
   if (!grouped && w->E != 1) return SHARQ_ERR_INVALID_ARG;
   if (grouped && !d_offsets) return SHARQ_ERR_INVALID_ARG;
   if (out_dtype != SHARQ_OUT_BF16 && out_dtype != SHARQ_OUT_F32) return SHARQ_ERR_INVALID_ARG;
@@ -231,10 +247,13 @@ const char* sharq_status_string(int status) {
   }
 }
 
-size_t sharq_weight_bytes(int K, int D, int E) {
+size_t sharq_weight_bytes_fmt(int K, int D, int E, int fmt) {
   if (!shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return 0;
-  return weight_layout(K, D, E).total;
+  if (fmt != SHARQ_FMT_NVFP4 && fmt != SHARQ_FMT_MXFP4) return 0;
+  return weight_layout(K, D, E, fmt).total;
 }
+
+size_t sharq_weight_bytes(int K, int D, int E) { return sharq_weight_bytes_fmt(K, D, E, SHARQ_FMT_NVFP4); }
 
 size_t sharq_act_bytes(int T, int K, int mode) {
   if (!shape_ok_t(T) || !shape_ok_k(K)) return 0;
@@ -247,11 +266,12 @@ size_t sharq_workspace_bytes(int T, int K, int D, int E) {
   return kWsHeader;
 }
 
-int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {
+int sharq_weight_view_fmt(void* d_buf, int K, int D, int E, int fmt, sharq_weight* out) {
   if (!d_buf || !out) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_k(K) || !shape_ok_d(D) || E < 1 || E > kMaxE) return SHARQ_ERR_UNSUPPORTED_SHAPE;
+  if (fmt != SHARQ_FMT_NVFP4 && fmt != SHARQ_FMT_MXFP4) return SHARQ_ERR_INVALID_ARG;
   if (!aligned(d_buf, kAlign)) return SHARQ_ERR_INVALID_ARG;
-  const WeightLayout L = weight_layout(K, D, E);
+  const WeightLayout L = weight_layout(K, D, E, fmt);
   uint8_t* b = static_cast<uint8_t*>(d_buf);
   out->codes = b + L.codes;
   out->sf32 = b + L.sf32;
@@ -260,7 +280,12 @@ int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {
   out->K = K;
   out->D = D;
   out->E = E;
+  out->fmt = fmt;
   return SHARQ_OK;
+}
+
+int sharq_weight_view(void* d_buf, int K, int D, int E, sharq_weight* out) {
+  return sharq_weight_view_fmt(d_buf, K, D, E, SHARQ_FMT_NVFP4, out);
 }
 
 int sharq_act_view(void* d_buf, int T, int K, int mode, sharq_act* out) {
@@ -291,6 +316,12 @@ int sharq_pack_weight(const void* d_W, const sharq_weight* w, sharq_stream_t str
   if (st) return st;
   if (!d_W || !aligned(d_W, 2)) return SHARQ_ERR_INVALID_ARG;
   if ((st = check_device())) return st;
+  if (w->fmt == SHARQ_FMT_MXFP4) {
+    cudaError_t e = sharq::launch_pack_weight_mx(d_W, w->K, w->D, w->E, static_cast<uint8_t*>(w->codes),
+                                                 static_cast<uint8_t*>(w->sf32), static_cast<uint8_t*>(w->sf16),
+                                                 w->s_w, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
+  }
   const WeightLayout L = weight_layout(w->K, w->D, w->E);
   unsigned int* scratch = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(w->s_w) + (L.scratch - L.s_w));
   cudaError_t e = sharq::launch_pack_weight(d_W, w->K, w->D, w->E, static_cast<uint8_t*>(w->codes),
@@ -351,7 +382,7 @@ int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, co
                       sharq_stream_t stream) {
   int st = weight_ok(w);
   if (st) return st;
-  if (w->E != 1) return SHARQ_ERR_INVALID_ARG;
+  if (w->E != 1 || w->fmt != SHARQ_FMT_NVFP4) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(T)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if (T > SHARQ_FUSED_MAX_T) {  // larger batches: the two-call path through `a`
     if (!a || a->T != T || a->K != w->K || (a->mode != SHARQ_MODE_SHARQ && a->mode != SHARQ_MODE_SHARQ_TOKEN))

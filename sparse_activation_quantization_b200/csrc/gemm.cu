@@ -759,24 +759,34 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
 // TMEM tile and read the same weight tile; a sparse operand (4:8 in-pairs,
 // one scale per 32 logical K) pairs with the weight's per-32 scale view, a
 // dense one (one scale per 16 K) with the per-16 view.
-enum : int { kGemmSharq = 0, kGemmNvfp4 = 1, kGemmSparseOnly = 2, kGemmDenseDense = 3, kGemmSparseSparse = 4 };
+enum : int {
+  kGemmSharq = 0, kGemmNvfp4 = 1, kGemmSparseOnly = 2, kGemmDenseDense = 3, kGemmSparseSparse = 4,
+  kGemmSharqMx = 5,  // MXFP4 operands (kind::mxf4, E8M0): sparse backbone + dense residual
+  kGemmMxfp4 = 6     // plain MXFP4: one dense operand
+};
 
 template <int BN, int kG>
 struct PCfg {
   static constexpr int kHalves = BN / 128;
-  static constexpr bool kHas1 = kG != kGemmNvfp4;       // first operand (backbone)
-  static constexpr bool kSp1 = kG != kGemmDenseDense;   // ... sparse
-  static constexpr bool kHas2 = kG != kGemmSparseOnly;  // second operand (residual)
+  static constexpr bool kMx = kG == kGemmSharqMx || kG == kGemmMxfp4;
+  static constexpr bool kHas1 = kG != kGemmNvfp4 && kG != kGemmMxfp4;  // first operand (backbone)
+  static constexpr bool kSp1 = kG != kGemmDenseDense;                 // ... sparse
+  static constexpr bool kHas2 = kG != kGemmSparseOnly;                // second operand (residual)
   static constexpr bool kSp2 = kG == kGemmSparseSparse;
-  static constexpr bool kB32 = (kHas1 && kSp1) || (kHas2 && kSp2);
-  static constexpr bool kB16 = (kHas1 && !kSp1) || (kHas2 && !kSp2);
+  static constexpr bool kB32 = (kHas1 && kSp1) || (kHas2 && kSp2);    // weight sparse-path view
+  static constexpr bool kB16 = (kHas1 && !kSp1) || (kHas2 && !kSp2);  // weight dense-path view
+  // scale tiles: NVFP4 sparse 1 KB (per 32 logical K), dense 2 KB (per 16);
+  // MXFP4 sparse 512 B (per 64 logical K), dense 1 KB (per 32)
+  static constexpr int kSfSp = kMx ? kSf64Tile : kSf32Tile;
+  static constexpr int kSfDn = kMx ? kSf32Tile : kSf16Tile;
   static constexpr int kA1 = kHas1 ? (kSp1 ? kSpTile : kCodesTile) : 0;
   static constexpr int kE1 = kHas1 && kSp1 ? kMetaTile : 0;
-  static constexpr int kS1 = kHas1 ? (kSp1 ? kSf32Tile : kSf16Tile) : 0;
+  static constexpr int kS1 = kHas1 ? (kSp1 ? kSfSp : kSfDn) : 0;
   static constexpr int kA2 = kHas2 ? (kSp2 ? kSpTile : kCodesTile) : 0;
   static constexpr int kE2 = kHas2 && kSp2 ? kMetaTile : 0;
-  static constexpr int kS2 = kHas2 ? (kSp2 ? kSf32Tile : kSf16Tile) : 0;
-  // stage layout (every size a multiple of 1 KB: swizzled tiles stay aligned)
+  static constexpr int kS2 = kHas2 ? (kSp2 ? kSfSp : kSfDn) : 0;
+  // stage layout: the swizzled code tiles first (1 KB multiples), then
+  // metadata and scales
   static constexpr int kOffB = 0;
   static constexpr int kOffA2 = kOffB + BN * 128;
   static constexpr int kOffA1 = kOffA2 + kA2;
@@ -785,8 +795,10 @@ struct PCfg {
   static constexpr int kOffS1 = kOffE2 + kE2;
   static constexpr int kOffS2 = kOffS1 + kS1;
   static constexpr int kOffSFB32 = kOffS2 + kS2;
-  static constexpr int kOffSFB16 = kOffSFB32 + (kB32 ? kHalves * kSf32Tile : 0);
-  static constexpr int kStageBytes = kOffSFB16 + (kB16 ? kHalves * kSf16Tile : 0);
+  static constexpr int kOffSFB16 = kOffSFB32 + (kB32 ? kHalves * kSfSp : 0);
+  // rounded to 1 KB so that every stage's swizzled code tiles (first in the
+  // stage) stay 1024-byte aligned; the scale regions need only 16 bytes
+  static constexpr int kStageBytes = (kOffSFB16 + (kB16 ? kHalves * kSfDn : 0) + 1023) / 1024 * 1024;
   static constexpr int kStages = (BN == 128 && 4 * kStageBytes + 1024 <= 232448) ? 4 : 3;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
   // TMEM: accumulator, then two scale regions (alternating by stage) of 32
@@ -800,7 +812,7 @@ struct PCfg {
   static constexpr uint32_t kTmemCols = BN + 2 * kSfRegion <= 256 ? 256 : 512;
   // transaction bytes per stage with `rows` valid activation rows
   __host__ __device__ static constexpr uint32_t tx(uint32_t rows) {
-    return BN * 128 + (kB32 ? kHalves * kSf32Tile : 0) + (kB16 ? kHalves * kSf16Tile : 0) +
+    return BN * 128 + (kB32 ? kHalves * kSfSp : 0) + (kB16 ? kHalves * kSfDn : 0) +
            rows * (uint32_t)(kA1 / 128 + kE1 / 128 + kA2 / 128 + kE2 / 128) + kS1 + kS2;
   }
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
@@ -890,8 +902,8 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
           for (int h = 0; h < C::kHalves; ++h) {
             const size_t bt = b_tile0 + (size_t)h * KS + i;
             bulk_g2s(st + C::kOffB + h * kCodesTile, args.w_codes + bt * kCodesTile, kCodesTile, fb);
-            if (C::kB16) bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bt * kSf16Tile, kSf16Tile, fb);
-            if (C::kB32) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bt * kSf32Tile, kSf32Tile, fb);
+            if (C::kB16) bulk_g2s(st + C::kOffSFB16 + h * C::kSfDn, args.w_sf16 + bt * C::kSfDn, C::kSfDn, fb);
+            if (C::kB32) bulk_g2s(st + C::kOffSFB32 + h * C::kSfSp, args.w_sf32 + bt * C::kSfSp, C::kSfSp, fb);
           }
           const size_t at = a_tile0 + i;
           if (C::kHas1) {
@@ -972,14 +984,59 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
               acc = true;
             }
           };
-          if (C::kHas1) {
-            if (C::kSp1) sparse_op(C::kOffA1, C::kOffE1, C::kOffS1, C::kSfE1, C::kSfS1, true);
-            else dense_op(C::kOffA1, C::kOffS1, C::kSfS1, true);
-          }
-          if (C::kHas2) {
-            // the weight view is already in TMEM when both operands share it
-            if (C::kSp2) sparse_op(C::kOffA2, C::kOffE2, C::kOffS2, C::kSfE2, C::kSfS2, !(C::kHas1 && C::kSp1));
-            else dense_op(C::kOffA2, C::kOffS2, C::kSfS2, !(C::kHas1 && !C::kSp1));
+          // MXFP4 (kind::mxf4, E8M0): one 512-byte atom holds 4 scales per row
+          // = two MMAs' worth; the scale-factor ID (byte 0 or 2 of the
+          // column) picks this MMA's pair, in the descriptor and in bits
+          // 30-31 of the TMEM scale address
+          auto sparse_op_mx = [&](uint32_t a_off, uint32_t e_off, uint32_t s_off, uint32_t e_col, uint32_t s_col) {
+            tc_cp_128x128b(sf + e_col, smem_desc(st + e_off, 0, 128, kSwNone));
+            tc_cp_32x128b_x4(sf + s_col, smem_desc(st + s_off, 0, 128, kSwNone));
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              tc_cp_32x128b_x4(sf + C::kSfB32 + 4 * h, smem_desc(st + C::kOffSFB32 + h * C::kSfSp, 0, 128, kSwNone));
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint32_t id = 2u * j;
+              mma_sp_mxf4(tmem + C::kColAcc, smem_desc(st + a_off + 32 * j, 16, 512, kSw64),
+                          smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + e_col + 2 * j,
+                          idesc_mxf4(128, BN, true, id, id), (sf + s_col) | (id << 30),
+                          (sf + C::kSfB32) | (id << 30), acc ? 1u : 0u);
+              acc = true;
+            }
+          };
+          auto dense_op_mx = [&](uint32_t a_off, uint32_t s_off, uint32_t s_col) {
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              tc_cp_32x128b_x4(sf + s_col + 4 * a, smem_desc(st + s_off + 512 * a, 0, 128, kSwNone));
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h)
+                tc_cp_32x128b_x4(sf + C::kSfB16 + a * C::kSfbCols + 4 * h,
+                                 smem_desc(st + C::kOffSFB16 + h * C::kSfDn + 512 * a, 0, 128, kSwNone));
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                const int j = 2 * a + q;
+                const uint32_t id = 2u * q;
+                mma_mxf4(tmem + C::kColAcc, smem_desc(st + a_off + 32 * j, 16, 1024, kSw128),
+                         smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_mxf4(128, BN, false, id, id),
+                         (sf + s_col + 4 * a) | (id << 30), (sf + C::kSfB16 + a * C::kSfbCols) | (id << 30),
+                         acc ? 1u : 0u);
+                acc = true;
+              }
+            }
+          };
+          if (C::kMx) {
+            if (C::kHas1) sparse_op_mx(C::kOffA1, C::kOffE1, C::kOffS1, C::kSfE1, C::kSfS1);
+            dense_op_mx(C::kOffA2, C::kOffS2, C::kSfS2);
+          } else {
+            if (C::kHas1) {
+              if (C::kSp1) sparse_op(C::kOffA1, C::kOffE1, C::kOffS1, C::kSfE1, C::kSfS1, true);
+              else dense_op(C::kOffA1, C::kOffS1, C::kSfS1, true);
+            }
+            if (C::kHas2) {
+              // the weight view is already in TMEM when both operands share it
+              if (C::kSp2) sparse_op(C::kOffA2, C::kOffE2, C::kOffS2, C::kSfE2, C::kSfS2, !(C::kHas1 && C::kSp1));
+              else dense_op(C::kOffA2, C::kOffS2, C::kSfS2, !(C::kHas1 && !C::kSp1));
+            }
           }
           tc_commit(&empty_bar[s]);
         }
@@ -1092,6 +1149,8 @@ cudaError_t launch_persistent_mode(const GemmArgs& a, int m_tiles, int gmode, cu
     case kGemmSparseOnly: return launch_persistent<BN, kGemmSparseOnly>(a, m_tiles, stream);
     case kGemmDenseDense: return launch_persistent<BN, kGemmDenseDense>(a, m_tiles, stream);
     case kGemmSparseSparse: return launch_persistent<BN, kGemmSparseSparse>(a, m_tiles, stream);
+    case kGemmSharqMx: return launch_persistent<BN, kGemmSharqMx>(a, m_tiles, stream);
+    case kGemmMxfp4: return launch_persistent<BN, kGemmMxfp4>(a, m_tiles, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -13,6 +13,7 @@
 // values, the layout the dense block16 MMA wants).
 //
 // Runs once per weight; two launches (device-wide amax, then quantization).
+// The MXFP4 payload (launch_pack_weight_mx) is one launch.
 #include "sharq_device.cuh"
 
 namespace sharq {
@@ -77,7 +78,57 @@ __global__ void __launch_bounds__(kThreads) weight_quant_kernel(
       (uint16_t)(bs.sb | (bs.sb << 8));
 }
 
+// MXFP4 payload (OCP Microscaling: E8M0 power-of-two scales, no tensor
+// scale): one thread per (expert, 64-K block, column d) -- 64 K is the scale
+// granularity of the sparse kind::mxf4 MMA, so the sparse view holds one byte
+// per 64 K and the dense view (32-K blocks) repeats it twice.  s_w = 1.
+__global__ void __launch_bounds__(kThreads) weight_quant_mx_kernel(
+    const __nv_bfloat16* __restrict__ W, int K, int D, float* __restrict__ s_w, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ sf64, uint8_t* __restrict__ sf32) {
+  const int e = blockIdx.z;
+  const int kb = blockIdx.y;  // 64-K block
+  const int d = blockIdx.x * kThreads + threadIdx.x;
+  if (d >= D) return;
+  if (kb == 0 && d == 0) s_w[e] = 1.0f;
+  const __nv_bfloat16* w = W + (size_t)e * K * D + (size_t)(64 * kb) * D + d;
+  float v[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __bfloat162float(w[(size_t)i * D]);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) a = fmaxf(a, fabsf(v[i]));
+  const BlockScale bs = mx_block_scale(a);
+  uint32_t word[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t wv = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = 8 * k + 2 * b;
+      wv |= cvt_e2m1x2(__fmul_rn(v[i], bs.inv), __fmul_rn(v[i + 1], bs.inv)) << (8 * b);
+    }
+    word[k] = wv;
+  }
+  const int KS = K >> 8, NB = D >> 7;
+  const int kt = kb >> 2, j = kb & 3, nb = d >> 7, r = d & 127;
+  const size_t tile = ((size_t)e * NB + nb) * KS + kt;
+  *reinterpret_cast<uint4*>(codes + tile * kCodesTile + codes_chunk_off(r, 2 * j)) =
+      make_uint4(word[0], word[1], word[2], word[3]);
+  *reinterpret_cast<uint4*>(codes + tile * kCodesTile + codes_chunk_off(r, 2 * j + 1)) =
+      make_uint4(word[4], word[5], word[6], word[7]);
+  sf64[tile * kSf64Tile + sf_off(r, 0, j)] = (uint8_t)bs.sb;
+  *reinterpret_cast<uint16_t*>(sf32 + tile * kSf32Tile + sf_off(r, j >> 1, (2 * j) & 3)) =
+      (uint16_t)(bs.sb | (bs.sb << 8));
+}
+
 }  // namespace
+
+cudaError_t launch_pack_weight_mx(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf64, uint8_t* sf32,
+                                  float* s_w, cudaStream_t stream) {
+  weight_quant_mx_kernel<<<dim3((D + kThreads - 1) / kThreads, K / 64, E), kThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(W), K, D, s_w, codes, sf64, sf32);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf32,
                                uint8_t* sf16, float* s_w, unsigned int* amax_bits, cudaStream_t stream) {

@@ -331,17 +331,22 @@ __global__ void __launch_bounds__(kRunsThreads) prep_runs_kernel(
   if (threadIdx.x == 0) gmax_sh = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
   __syncthreads();
   const float gmax = gmax_sh;
-  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
+  // MX formats have no tensor scale
+  const float s = kind_is_mx(kKind) ? 1.0f : (gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f);
   if (gid == 0) *s_g_out = s;
-  if (gid < (long long)T * segs) {
-    const int t = (int)(gid / segs);
-    const int c0 = (int)(gid - (long long)t * segs) * 4;
-    const int src = row_index ? row_index[t] : t;
-    float x[32];
-    load_runs<4>(x, X, src, K, c0);
-    if (gamma && src >= 0) normalise_runs<4>(x, gamma, c0, inv_rms[t]);
-    quant_runs<4, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out);
-  }
+  // Every lane of the warp runs the quantizer (an MXFP4 backbone block spans
+  // two lanes, reduced with warp shuffles); lanes past the end work on zeros
+  // and store nothing.  Active lanes come in groups of 8 (K / 32 is a
+  // multiple of 8), so a block never mixes active and idle lanes.
+  const bool active = gid < (long long)T * segs;
+  const long long g = active ? gid : 0;
+  const int t = (int)(g / segs);
+  const int c0 = (int)(g - (long long)t * segs) * 4;
+  const int src = active ? (row_index ? row_index[t] : t) : -1;
+  float x[32];
+  load_runs<4>(x, X, src, K, c0);
+  if (gamma && src >= 0) normalise_runs<4>(x, gamma, c0, inv_rms[t]);
+  quant_runs<4, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, active);
   if (threadIdx.x == 0) depart_and_reset(gmax_bits);
 }
 
@@ -459,7 +464,8 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   }
   __syncthreads();
   const float gmax = gmax_sh;
-  const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
+  // MX formats have no tensor scale
+  const float s = kind_is_mx(kKind) ? 1.0f : (gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
   // rows past T: whole warps (rows span whole warps), so they can skip
   if (live) quant_runs<NC, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
@@ -635,6 +641,14 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
         e = try_fused_any<kKindSparseSparse>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
                                              &launched);
         break;
+      case kKindSharqMx:
+        e = try_fused_any<kKindSharqMx>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+                                        &launched);
+        break;
+      case kKindMxfp4:
+        e = try_fused_any<kKindMxfp4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+                                      &launched);
+        break;
       default:
         return cudaErrorInvalidValue;
     }
@@ -662,15 +676,18 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
       prep_rowstats_kernel<false><<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms,
                                                                     gmax_bits);
   }
-  if (kind == kKindDenseDense || kind == kKindSparseSparse) {
+  if (kind != kKindSharq && kind != kKindNvfp4) {
     const long long n = (long long)T * (K >> 5);
     const unsigned grid = n > 0 ? (unsigned)((n + kRunsThreads - 1) / kRunsThreads) : 1u;
-    if (kind == kKindDenseDense)
-      prep_runs_kernel<kKindDenseDense><<<grid, kRunsThreads, 0, stream>>>(Xb, Gb, row_index, T, K, inv_rms,
-                                                                          gmax_bits, s_g, p);
-    else
-      prep_runs_kernel<kKindSparseSparse><<<grid, kRunsThreads, 0, stream>>>(Xb, Gb, row_index, T, K, inv_rms,
-                                                                            gmax_bits, s_g, p);
+#define SHARQ_RUNS(KIND) prep_runs_kernel<KIND><<<grid, kRunsThreads, 0, stream>>>(Xb, Gb, row_index, T, K, \
+                                                                                inv_rms, gmax_bits, s_g, p)
+    switch (kind) {
+      case kKindDenseDense: SHARQ_RUNS(kKindDenseDense); break;
+      case kKindSparseSparse: SHARQ_RUNS(kKindSparseSparse); break;
+      case kKindSharqMx: SHARQ_RUNS(kKindSharqMx); break;
+      default: SHARQ_RUNS(kKindMxfp4); break;
+    }
+#undef SHARQ_RUNS
     return cudaGetLastError();
   }
   const bool sharq_mode = kind == kKindSharq;

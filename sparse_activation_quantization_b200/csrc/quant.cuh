@@ -44,8 +44,11 @@ enum : int {
   kKindNvfp4 = 0,        // one dense operand: NVFP4 of Xn
   kKindSharq = 1,        // sparse backbone + dense residual (also Sparse only: the GEMM drops the residual)
   kKindDenseDense = 2,   // dense NVFP4 of Xn + dense NVFP4 of its residual
-  kKindSparseSparse = 3  // sparse backbone + sparse (4:8 in-pairs) residual
+  kKindSparseSparse = 3,  // sparse backbone + sparse (4:8 in-pairs) residual
+  kKindSharqMx = 4,       // SharQ in MXFP4: E8M0 scales, backbone per 64 logical K, residual per 32 K
+  kKindMxfp4 = 5          // plain MXFP4 of Xn (32-element blocks)
 };
+__host__ __device__ constexpr bool kind_is_mx(int kind) { return kind == kKindSharqMx || kind == kKindMxfp4; }
 
 // max over the `width` adjacent lanes of an aligned lane group
 __device__ __forceinline__ float group_max(float v, int width) {
@@ -80,8 +83,9 @@ __device__ __forceinline__ float2 e2m1x2_values(uint32_t byte) {
 // logical K, the metadata; out[] = v - f32(val * dec * s) at kept positions
 // and v elsewhere (exact).  Tiles: codes 8 KB (64-byte swizzle), metadata
 // 2 KB, scales 1 KB.  NC = 1, 2: the 32-K block spans 4 / NC adjacent lanes
-// (all 32 lanes of the warp must call it).
-template <int NC>
+// (all 32 lanes of the warp must call it).  kMx: one E8M0 scale per 64
+// logical K (8 runs; 512-byte scale tiles), s must be 1.
+template <int NC, bool kMx = false>
 __device__ __forceinline__ void sparse_operand(const float (&x)[8 * NC], float (&res)[8 * NC], int t, int c0, int K,
                                                float s, float six_s, uint8_t* codes_out, uint8_t* meta_out,
                                                uint8_t* sf_out, bool store) {
@@ -105,12 +109,13 @@ __device__ __forceinline__ void sparse_operand(const float (&x)[8 * NC], float (
     v[4 * c + 2] = k3 ? xc[6] : ((km[c] & 4u) ? xc[4] : xc[2]);
     v[4 * c + 3] = k3 ? xc[7] : ((km[c] & 4u) ? xc[5] : xc[3]);
   }
-  // one scale per 32 logical K (4 runs = 16 kept values)
+  // one scale per 32 logical K (4 runs = 16 kept values); MX: per 64 (8 runs)
+  constexpr int kBlockRuns = kMx ? 8 : 4;
   float am = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4 * NC; ++i) am = fmaxf(am, fabsf(v[i]));
-  if (NC < 4) am = group_max(am, 4 / NC);
-  const BlockScale bs = block_scale(am, six_s, s);
+  if (NC < kBlockRuns) am = group_max(am, kBlockRuns / NC);
+  const BlockScale bs = kMx ? mx_block_scale(am) : block_scale(am, six_s, s);
   uint32_t cb[2 * NC];  // code bytes: kept values (2i, 2i+1)
 #pragma unroll
   for (int i = 0; i < 2 * NC; ++i) cb[i] = cvt_e2m1x2(__fmul_rn(v[2 * i], bs.inv), __fmul_rn(v[2 * i + 1], bs.inv));
@@ -148,27 +153,34 @@ __device__ __forceinline__ void sparse_operand(const float (&x)[8 * NC], float (
       const uint32_t other = (uint32_t)((__ffs(m2) - 1) | ((31 - __clz(m2)) << 2));
       meta_out[tile * kMetaTile + r * 16 + (w >> 1)] = (uint8_t)(nib | (other << 4));
     }
-    if (store && (w & 3) == 0) sf_out[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
+    if (kMx) {
+      if (store && (w & 7) == 0) sf_out[tile * kSf64Tile + sf_off(r, 0, w >> 3)] = (uint8_t)bs.sb;
+    } else if (store && (w & 3) == 0) {
+      sf_out[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
+    }
   }
 }
 
 // Dense operand: NVFP4 of v in 16-element blocks; with kDeq, deq[] receives
 // f32(val * dec * s) of every element.  Tiles: codes 16 KB (128-byte
-// swizzle), scales 2 KB.  NC = 1: the 16-K block spans 2 adjacent lanes.
-template <int NC, bool kDeq>
+// swizzle), scales 2 KB.  kMx: MXFP4, one E8M0 scale per 32 K (1 KB scale
+// tiles), s must be 1.  A block spans 2 (MX: 4) runs; when a thread holds
+// fewer, it spans adjacent lanes (all 32 lanes of the warp must call it).
+template <int NC, bool kDeq, bool kMx = false>
 __device__ __forceinline__ void dense_operand(const float (&res)[8 * NC], float (&deq)[8 * NC], int t, int c0, int K,
                                               float s, float six_s, uint8_t* codes_out, uint8_t* sf_out, bool store) {
   const int KS = K >> 8;
   const int r = t & 127;
+  constexpr int kBlockRuns = kMx ? 4 : 2;
+  constexpr int nr = NC < kBlockRuns ? NC : kBlockRuns;  // runs of a block held by this thread
+  constexpr int lanes = kBlockRuns / nr;                  // lanes a block spans
 #pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    if (NC > 1 && (c & 1)) continue;  // the even run handles its block of two runs
-    const int nr = NC == 1 ? 1 : 2;   // runs of this block held by this thread
+  for (int c = 0; c < NC; c += nr) {
     float am = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8 * nr; ++i) am = fmaxf(am, fabsf(res[8 * c + i]));
-    if (NC == 1) am = group_max(am, 2);
-    const BlockScale bs = block_scale(am, six_s, s);
+    if (lanes > 1) am = group_max(am, lanes);
+    const BlockScale bs = kMx ? mx_block_scale(am) : block_scale(am, six_s, s);
 #pragma unroll
     for (int h = 0; h < nr; ++h) {
       uint32_t word = 0;
@@ -189,7 +201,11 @@ __device__ __forceinline__ void dense_operand(const float (&res)[8 * NC], float 
       if (store) {
         *reinterpret_cast<uint32_t*>(codes_out + tile * kCodesTile + codes_chunk_off(r, w >> 2) + 4 * (w & 3)) =
             word;
-        if ((w & 1) == 0) sf_out[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+        if (kMx) {
+          if ((w & 3) == 0) sf_out[tile * kSf32Tile + sf_off(r, w >> 4, (w >> 2) & 3)] = (uint8_t)bs.sb;
+        } else if ((w & 1) == 0) {
+          sf_out[tile * kSf16Tile + sf_off(r, w >> 3, (w >> 1) & 3)] = (uint8_t)bs.sb;
+        }
       }
     }
   }
@@ -213,10 +229,15 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
 #pragma unroll
     for (int i = 0; i < 8 * NC; ++i) res[i] = __fsub_rn(x[i], deq[i]);
     dense_operand<NC, false>(res, deq, t, c0, K, s, six_s, out.r_codes, out.r_sf, store);
-  } else {
+  } else if (kKind == kKindSparseSparse) {
     float res2[8 * NC];
     sparse_operand<NC>(x, res, t, c0, K, s, six_s, out.sp_codes, out.meta, out.sp_sf, store);
     sparse_operand<NC>(res, res2, t, c0, K, s, six_s, out.r_codes, out.r_meta, out.r_sf, store);
+  } else if (kKind == kKindSharqMx) {
+    sparse_operand<NC, true>(x, res, t, c0, K, 1.0f, 6.0f, out.sp_codes, out.meta, out.sp_sf, store);
+    dense_operand<NC, false, true>(res, res, t, c0, K, 1.0f, 6.0f, out.r_codes, out.r_sf, store);
+  } else {  // kKindMxfp4
+    dense_operand<NC, false, true>(x, res, t, c0, K, 1.0f, 6.0f, out.r_codes, out.r_sf, store);
   }
 }
 

@@ -21,6 +21,7 @@ constexpr int kCodesTile = 16384;   // 128 rows x 128 B, 128-byte swizzle
 constexpr int kSpTile = 8192;       // 128 rows x 64 B, 64-byte swizzle
 constexpr int kMetaTile = 2048;     // 128 rows x 16 B
 constexpr int kSf32Tile = 1024;     // 2 scale atoms
+constexpr int kSf64Tile = 512;      // 1 scale atom (MXFP4 backbone: one scale per 64 logical K)
 constexpr int kSf16Tile = 2048;     // 4 scale atoms
 constexpr float kGlobalDiv = 2688.0f;  // 6 (E2M1 max) * 448 (E4M3 max)
 
@@ -75,6 +76,23 @@ __device__ __forceinline__ BlockScale block_scale(float amax, float six_s, float
   r.dec = e4m3_value(r.sb);
   float S = __fmul_rn(r.dec, s);
   r.inv = S > 0.0f ? __frcp_rn(S) : 0.0f;
+  return r;
+}
+
+// MX block scale (OCP Microscaling Formats v1.0, E8M0): X = 2^e with
+// e = floor(log2 amax) - 2 (E2M1's largest exponent), clamped to [-127, 127];
+// -127 for an all-zero block.  floor(log2) is read off the float32 encoding.
+__device__ __forceinline__ float pow2f(int e) {  // exact 2^e for e in [-127, 127]
+  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+__device__ __forceinline__ BlockScale mx_block_scale(float amax) {
+  const uint32_t ef = __float_as_uint(amax) >> 23;  // amax >= 0
+  int e = ef > 0 ? (int)ef - 127 - 2 : -127;       // zero and subnormal blocks clamp to -127
+  e = e < -127 ? -127 : (e > 127 ? 127 : e);
+  BlockScale r;
+  r.sb = (uint32_t)(e + 127);
+  r.dec = pow2f(e);
+  r.inv = pow2f(-e);
   return r;
 }
 
@@ -256,6 +274,16 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N, bool sparse) {
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::mxf4 (E2M1 x E2M1 with E8M0 scales, one
+// per 32 stored elements -- 64 logical K in the sparse form -- FP32
+// accumulate): the fields of idesc_nvf4 plus the scale format (bit 23 = E8M0)
+// and the scale-factor IDs, A in bits 29-30 and B in bits 4-5: the byte of
+// the 32-bit TMEM scale column where this MMA's two scales per row start.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, bool sparse, uint32_t a_id, uint32_t b_id) {
+  return (sparse ? (1u << 2) : 0u) | (b_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         (1u << 23) | ((uint32_t)(M >> 4) << 24) | (a_id << 29);
+}
+
 // smem (described by desc) -> TMEM: 128 lanes x 16 bytes
 __device__ __forceinline__ void tc_cp_128x128b(uint32_t taddr, uint64_t desc) {
   asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
@@ -283,6 +311,28 @@ __device__ __forceinline__ void mma_sp_nvf4(uint32_t d, uint64_t adesc, uint64_t
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %5, 0;\n\t"
       "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%3], %4, [%6], [%7], "
+      "p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(e), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// MXFP4 forms: per-32 (sparse: per-64 logical) E8M0 scales from TMEM; the
+// scale addresses carry the scale-factor ID in bits 30-31 as well
+__device__ __forceinline__ void mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma_sp_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t e, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, [%3], %4, [%6], [%7], "
       "p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(e), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");

@@ -82,10 +82,11 @@ def untile_meta(buf, rows, K):
 
 
 def untile_sf(buf, rows, K, per):
-    """scale tiles -> bytes [rows_padded, K/per] (per = 16 or 32)."""
+    """scale tiles -> bytes [rows_padded, K/per] (per = 16, 32 or 64 logical
+    K per scale: 4, 2 or 1 atoms of 512 bytes per tile)."""
     RT, KS = (rows + 127) // 128, K // 256
     nb = 256 // per
-    size, perm = (SF16_TILE, SF16_PERM) if per == 16 else (SF32_TILE, SF8_PERM)
+    size, perm = nb // 4 * 512, _sf_perm(nb)
     t = _tiles(buf, RT, KS, size)
     return t[:, :, perm].transpose(0, 2, 1, 3).reshape(RT * 128, KS * nb)
 
@@ -122,7 +123,7 @@ def tile_sf(sf, per):
     R, nbk = sf.shape
     nb = 256 // per
     RT, KS = R // 128, nbk // nb
-    size, perm = (SF16_TILE, SF16_PERM) if per == 16 else (SF32_TILE, SF8_PERM)
+    size, perm = nb // 4 * 512, _sf_perm(nb)
     out = np.zeros((RT, KS, size), dtype=np.uint8)
     out[:, :, perm] = sf.reshape(RT, 128, KS, nb).transpose(0, 2, 1, 3)
     return out.reshape(-1)

@@ -54,7 +54,13 @@ def test_sizes(L):
     assert sq.sharq_act_bytes(16, 200, 0) == 0
     assert sq.sharq_weight_bytes(256, 100, 1) == 0
     assert sq.sharq_act_bytes(-1, 256, 0) == 0
-    assert sq.sharq_act_bytes(16, 256, 7) == 0
+    assert sq.sharq_act_bytes(16, 256, 99) == 0
+    # MXFP4: E8M0 scales per 64 K (sparse view) and per 32 K (dense view)
+    assert abs(sq.sharq_weight_bytes_fmt(4096, 4096, 1, sq.SHARQ_FMT_MXFP4) / (4096 * 4096) - 0.546875) < 1e-3
+    assert sq.sharq_weight_bytes_fmt(4096, 4096, 1, 7) == 0
+    mx = sq.sharq_act_bytes(T, K, sq.SHARQ_MODE_MXFP4)
+    assert mx >= tiles * (16384 + 1024 + 8192 + 2048 + 512) + Tp * 4 and mx < a
+    assert tiles * (16384 + 1024) + Tp * 4 <= sq.sharq_act_bytes(T, K, sq.SHARQ_MODE_MXFP4_PLAIN) < n
     assert sq.sharq_workspace_bytes(16, 256, 256, 1) > 0
 
 
