@@ -419,7 +419,9 @@ def run_gpu(args, world, rank, local):
     # same for every mode) on the first input copy
     MODES = {"sharq": sq.SHARQ_MODE_SHARQ, "nvfp4": sq.SHARQ_MODE_NVFP4, "sharq_per_token": sq.SHARQ_MODE_SHARQ_TOKEN,
              "sparse_only": sq.SHARQ_MODE_SPARSE_ONLY, "dense_dense": sq.SHARQ_MODE_DENSE_DENSE,
-             "sparse_sparse": sq.SHARQ_MODE_SPARSE_SPARSE}
+             "sparse_sparse": sq.SHARQ_MODE_SPARSE_SPARSE, "sharq_mxfp4": sq.SHARQ_MODE_MXFP4,
+             "mxfp4": sq.SHARQ_MODE_MXFP4_PLAIN}
+    MX_MODES = (sq.SHARQ_MODE_MXFP4, sq.SHARQ_MODE_MXFP4_PLAIN)
 
     def mode_table(L, li, src, W0):
         x0 = xs[src][0].float()
@@ -433,17 +435,28 @@ def run_gpu(args, world, rank, local):
         yref = xn @ W0.float()
         y32 = torch.empty((L.T, L.D), dtype=torch.float32, device=dev)
         out = {}
+        w_mx = None
         for name, mode in MODES.items():
             try:
                 a_m = sq.PreparedAct(L.T, L.K, mode=mode, device=dev)
             except Exception as e:  # a shape the mode does not support
                 out[name] = {"unsupported": str(e)}
                 continue
+            if mode in MX_MODES:  # the MXFP4 payloads of the same weights (same rotation)
+                if w_mx is None:
+                    w_mx = []
+                    for i in range(n_rot):
+                        Wi = torch.from_numpy(synthetic.weights(100 + 31 * li + i, L.K, L.D)).to(torch.bfloat16).to(dev)
+                        w_mx.append(sq.PackedWeight(Wi, stream=stream, fmt=sq.SHARQ_FMT_MXFP4))
+                        del Wi
+                wsel = lambda i: w_mx[i]
+            else:
+                wsel = lambda i: weights[L.name][i]
             us = kernel_us(lambda i: (a_m.prep(xs[src][i], gammas[src], EPS, stream=stream),
-                                      sq.linear(a_m, weights[L.name][i], out=outs[L.name], ws=wss[L.name],
+                                      sq.linear(a_m, wsel(i), out=outs[L.name], ws=wss[L.name],
                                                 stream=stream)), n_rot, stream)
             a_m.prep(xs[src][0], gammas[src], EPS, stream=stream)
-            sq.linear(a_m, weights[L.name][0], out_dtype=torch.float32, out=y32, ws=wss[L.name], stream=stream)
+            sq.linear(a_m, wsel(0), out_dtype=torch.float32, out=y32, ws=wss[L.name], stream=stream)
             torch.cuda.synchronize()
             err = (torch.linalg.norm(y32 - yref) / torch.linalg.norm(yref)).item()
             out[name] = {"layer_us": round(us, 3), "y_rel_err": round(err, 5)}
