@@ -126,6 +126,24 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max over all ranks of per-rank times (ms): with every rank
+    running its own replica (weak scaling), the job takes as long as its
+    slowest rank.  Identity with one process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(flops_per_rank, world, ms):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def init_dist(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -357,9 +375,7 @@ def run_gpu(args, world, rank, local):
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
     if world > 1:
-        t_ = torch.tensor([ms], device=dev)
-        dist.all_reduce(t_, op=dist.ReduceOp.MAX)
-        ms = t_.item()
+        ms = max_over_ranks([ms], dev)[0]
         dist.barrier()
     for L in layers:
         assert wss[L.name].check(stream) == 0, "device-side error"
@@ -409,9 +425,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
     if world > 1:
-        t_ = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t_, op=dist.ReduceOp.MAX)
-        e2e_ms = t_.item()
+        e2e_ms = max_over_ranks([e2e_ms], dev)[0]
 
     # --- every activation mode of the library on one layer: prep + GEMM time,
     # and the relative Frobenius error of Y (float32 output) against the
@@ -504,7 +518,7 @@ def run_gpu(args, world, rank, local):
     line = None
     if rank == 0:
         ms_step = ms / args.steps
-        value = flops_step * world / (ms_step * 1e-3) / 1e12
+        value = job_tflops(flops_step, world, ms_step)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -520,7 +534,7 @@ def run_gpu(args, world, rank, local):
                        for n, d in per.items()},
             "roofline": roof,
             "comparators": comparators,
-            "e2e": {"value": flops_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": job_tflops(flops_step, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
