@@ -453,6 +453,18 @@ def linear_mx(p, wq):
     return a_sp @ w64 + a_r @ w32
 
 
+def residual_add(x, res):
+    """The residual-stream update a pre-norm decoder layer performs before
+    the next RMSNorm, fused into the preparation step (the kasblo.com
+    explainer notes that RMSNorm and the preceding epilogues are fused into
+    the preparation kernel): h = bf16_rn(f32(x + res)) for bf16 x and res
+    (float32 [T, K] holding bf16 values) -- the float32 sum, rounded to
+    nearest even in bfloat16, as a bf16 framework computes it."""
+    x = np.asarray(x, dtype=np.float32)
+    r = np.asarray(res, dtype=np.float32)
+    return bf16_round((x + r).astype(np.float32))
+
+
 def prep_nvfp4(x, gamma=None, eps=1e-5):
     """Plain NVFP4 preparation, the comparator the SharQ evaluation reports
     as "NVFP4" (xllm-io review, Table 1; the kasblo.com explainer lists the
