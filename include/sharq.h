@@ -233,6 +233,29 @@ int sharq_prep(const void *d_X, const void *d_gamma, float eps, const int *d_row
                const sharq_act *a, sharq_stream_t stream);
 
 /*
+ * sharq_prep_residual - sharq_prep of the updated residual stream.
+ * A pre-norm decoder layer adds a sublayer's output to the residual stream
+ * and normalises the sum before the next linear layer; the kasblo.com
+ * explainer (section 4, on fusing the preparation) counts that epilogue
+ * among what the prep kernel takes in.  This call does both in the same
+ * kernels: the prep input is h = bf16_rn(f32(x) + f32(res)), element by
+ * element (a bf16 framework's x + res), and h is written out as the new
+ * residual stream.  Outputs in `a` are those of sharq_prep on h, bit for bit.
+ * d_X:       bf16 [a->T][K] row-major, the sublayer output.
+ * d_res:     bf16 [a->T][K] row-major, the residual stream.
+ * d_res_out: bf16 [a->T][K] that receives h, or NULL (h not stored).  It may
+ *            be d_res itself (in-place update: each element is read and then
+ *            written by the same thread); it must not overlap d_X, nor
+ *            overlap d_res other than exactly.
+ * d_gamma, eps, a: as for sharq_prep.  Row gathering is not offered.
+ * Errors: as sharq_prep; SHARQ_ERR_INVALID_ARG for a NULL or misaligned
+ * (16-byte) d_res or d_res_out, or d_res_out == d_X.  a->T == 0 touches
+ * none of the three arrays.
+ */
+int sharq_prep_residual(const void *d_X, const void *d_res, void *d_res_out, const void *d_gamma, float eps,
+                        const sharq_act *a, sharq_stream_t stream);
+
+/*
  * sharq_prep_noalloc - sharq_prep for callers that cannot allocate device
  * memory at run time: code inside a region being captured into a CUDA graph
  * (where cudaMalloc is not allowed), or a host framework whose memory

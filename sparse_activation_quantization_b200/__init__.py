@@ -23,6 +23,7 @@ __all__ = [
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
     "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc", "sharq_prep_linear", "prep_linear",
+    "sharq_prep_residual",
     "PackedWeight", "PreparedAct", "Workspace", "linear", "EXPORTED_SYMBOLS",
 ]
 
@@ -43,7 +44,7 @@ EXPORTED_SYMBOLS = (
     "sharq_weight_bytes", "sharq_act_bytes", "sharq_workspace_bytes", "sharq_weight_view",
     "sharq_act_view", "sharq_pack_weight", "sharq_prep", "sharq_linear", "sharq_linear_grouped",
     "sharq_check_status", "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
-    "sharq_prep_linear", "sharq_weight_bytes_fmt", "sharq_weight_view_fmt",
+    "sharq_prep_linear", "sharq_weight_bytes_fmt", "sharq_weight_view_fmt", "sharq_prep_residual",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -93,6 +94,7 @@ def lib():
             "sharq_pack_weight": (i, [vp, W, vp]),
             "sharq_prep": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
             "sharq_prep_noalloc": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
+            "sharq_prep_residual": (i, [vp, vp, vp, vp, ctypes.c_float, A, vp]),
             "sharq_linear": (i, [A, W, vp, i, vp, sz, vp]),
             "sharq_prep_linear": (i, [vp, vp, ctypes.c_float, i, A, W, vp, i, vp, sz, vp]),
             "sharq_linear_grouped": (i, [A, vp, W, vp, i, vp, sz, vp]),
@@ -168,6 +170,11 @@ def sharq_prep(d_X, d_gamma, eps, d_row_index, a, stream):
 def sharq_prep_noalloc(d_X, d_gamma, eps, d_row_index, a, stream):
     return _check(lib().sharq_prep_noalloc(d_X, d_gamma, eps, d_row_index, ctypes.byref(a), stream),
                   "sharq_prep_noalloc")
+
+
+def sharq_prep_residual(d_X, d_res, d_res_out, d_gamma, eps, a, stream):
+    return _check(lib().sharq_prep_residual(d_X, d_res, d_res_out, d_gamma, eps, ctypes.byref(a), stream),
+                  "sharq_prep_residual")
 
 
 def sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream):
@@ -258,6 +265,16 @@ class PreparedAct:
                    gamma.data_ptr() if gamma is not None else None, float(eps),
                    row_index.data_ptr() if row_index is not None else None,
                    self.view, _stream_ptr(stream))
+        return self
+
+    def prep_residual(self, X, res, res_out=None, gamma=None, eps=1e-5, stream=None):
+        """sharq_prep of h = bf16(X + res); h goes to res_out (which may be
+        res itself) when given."""
+        sharq_prep_residual(X.data_ptr() if X is not None else None,
+                            res.data_ptr() if res is not None else None,
+                            res_out.data_ptr() if res_out is not None else None,
+                            gamma.data_ptr() if gamma is not None else None, float(eps),
+                            self.view, _stream_ptr(stream))
         return self
 
     def region(self, name, nbytes):

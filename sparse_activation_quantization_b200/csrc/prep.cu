@@ -82,6 +82,22 @@ __device__ __forceinline__ double bf16_lo_x2p128(uint32_t w) {
   return __hiloint2double((int)(((w << 13) & 0x0FFFE000u) | 0x40000000u), 0);
 }
 
+// v[u] (vector c0 + 32 u of a row, zeros past its end) <- h = x + res, and
+// h stored to hr (the same vectors of the updated stream) when hr is given
+template <int N>
+__device__ __forceinline__ void add_row_residual(uint4 (&v)[N], const uint4* rr, uint4* hr, int c0, int nv) {
+  uint4 r[N];
+#pragma unroll
+  for (int u = 0; u < N; ++u) r[u] = c0 + 32 * u < nv ? rr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int u = 0; u < N; ++u) v[u] = add_bf16x8(v[u], r[u]);
+  if (hr) {
+#pragma unroll
+    for (int u = 0; u < N; ++u)
+      if (c0 + 32 * u < nv) hr[c0 + 32 * u] = v[u];
+  }
+}
+
 __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -93,6 +109,11 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 //   RMSNorm rows: float64 sum of squares -> 1/rms, then max |Xn| (Xn
 //   recomputed from L1/L2 as in the quantizer: bf16(f32(f32(x/rms) g))).
 //   Rows without RMSNorm: max |x| on packed bf16 bits.
+// With a residual stream (kResid) the rows are h = x + res: the first pass
+// forms h (4 vectors of x and 4 of res in flight per lane) and, when the
+// updated stream is wanted, stores it there; the second pass and the
+// quantizer launch then read h alone.  Each element of h is stored and
+// re-read by the lane that formed it.
 // The device-wide max goes to gmax_bits[0] with one atomicMax per CTA.
 // Sum of squares: each square of a bf16 value is exact in float64, and the
 // values enter scaled by 2^128 (bf16_*_x2p128, squares scaled by 2^256,
@@ -101,11 +122,12 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 // row -- far below one ulp of mean(x^2) + eps for any eps >= 2^-60, where
 // the result is that of an exact-input float64 sum in this lane order.  For
 // eps < 2^-60 (`exact`) the elements are converted exactly instead.
-template <bool kGamma>
+template <bool kGamma, bool kResid>
 __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int K, int exact, float* __restrict__ inv_rms,
-    unsigned int* __restrict__ gmax_bits) {
+    unsigned int* __restrict__ gmax_bits, Resid rs) {
+  constexpr int kC = kResid ? kRowChunk / 2 : kRowChunk;  // vectors of the row in flight per lane
   __shared__ uint32_t wmax[kRowThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = gridDim.x * (kRowThreads / 32);
@@ -118,15 +140,18 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
       continue;
     }
     const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K);
+    const uint4* rr = kResid ? reinterpret_cast<const uint4*>(rs.R + (size_t)src * K) : nullptr;
+    uint4* hr = kResid && rs.H ? reinterpret_cast<uint4*>(rs.H + (size_t)src * K) : nullptr;
     if (kGamma) {
       double acc0 = 0.0, acc1 = 0.0;
-      for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunk) {
-        uint4 v[kRowChunk];
+      for (int c0 = lane; c0 < nv; c0 += 32 * kC) {
+        uint4 v[kC];
 #pragma unroll
-        for (int u = 0; u < kRowChunk; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < kC; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+        if (kResid) add_row_residual<kC>(v, rr, hr, c0, nv);
         if (!exact) {
 #pragma unroll
-          for (int u = 0; u < kRowChunk; ++u) {
+          for (int u = 0; u < kC; ++u) {
             if (c0 + 32 * u < nv) {
               const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
@@ -139,7 +164,7 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
           }
         } else {
 #pragma unroll
-          for (int u = 0; u < kRowChunk; ++u) {
+          for (int u = 0; u < kC; ++u) {
             float f[8];
             bf16x8_to_float(v[u], f);  // zero-filled beyond the row: adds 0
 #pragma unroll
@@ -158,16 +183,18 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
       if (lane == 0) inv_rms[t] = inv;
       const f2_t inv2 = f2_make(inv, inv);
       const uint4* gr = reinterpret_cast<const uint4*>(gamma);
-      for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunk) {
-        uint4 v[kRowChunk], g[kRowChunk];
+      const uint4* sr = hr ? hr : xr;  // h, once stored
+      for (int c0 = lane; c0 < nv; c0 += 32 * kC) {
+        uint4 v[kC], g[kC];
 #pragma unroll
-        for (int u = 0; u < kRowChunk; ++u) {
+        for (int u = 0; u < kC; ++u) {
           const bool in = c0 + 32 * u < nv;
-          v[u] = in ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+          v[u] = in ? sr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
           g[u] = in ? gr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
         }
+        if (kResid && !hr) add_row_residual<kC>(v, rr, nullptr, c0, nv);
 #pragma unroll
-        for (int u = 0; u < kRowChunk; ++u) {
+        for (int u = 0; u < kC; ++u) {
           const uint32_t xw[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
           const uint32_t gw[4] = {g[u].x, g[u].y, g[u].z, g[u].w};
 #pragma unroll
@@ -179,12 +206,13 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
         }
       }
     } else {
-      for (int c0 = lane; c0 < nv; c0 += 32 * kRowChunk) {
-        uint4 v[kRowChunk];
+      for (int c0 = lane; c0 < nv; c0 += 32 * kC) {
+        uint4 v[kC];
 #pragma unroll
-        for (int u = 0; u < kRowChunk; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < kC; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
+        if (kResid) add_row_residual<kC>(v, rr, hr, c0, nv);
 #pragma unroll
-        for (int u = 0; u < kRowChunk; ++u) {
+        for (int u = 0; u < kC; ++u) {
           mx = vmax_u16x2(mx, v[u].x & 0x7FFF7FFFu);
           mx = vmax_u16x2(mx, v[u].y & 0x7FFF7FFFu);
           mx = vmax_u16x2(mx, v[u].z & 0x7FFF7FFFu);
@@ -237,7 +265,7 @@ template <bool kSharq, bool kGamma>
 __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
     const int* __restrict__ row_index, int T, int K, int nw, const float* __restrict__ inv_rms,
-    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
+    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out, Resid rs) {
   __shared__ float2 tab[128];
   __shared__ uint32_t msel[16];
   allow_dependents();
@@ -274,6 +302,7 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
 #pragma unroll
     for (int u = 0; u < 4; ++u)
       cur[u] = (active && src >= 0) ? reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * (size_t)j)[u] : z4;
+    if (rs.R && active && src >= 0) add_residual<4>(cur, (size_t)src * K + 32 * (size_t)j, rs);
     if (kGamma) inv = inv_rms[t];
     while (t < T) {
       // prefetch the next row of this warp
@@ -286,6 +315,7 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
         if (active && srcn >= 0) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) nxt[u] = reinterpret_cast<const uint4*>(X + (size_t)srcn * K + 32 * (size_t)j)[u];
+          if (rs.R) add_residual<4>(nxt, (size_t)srcn * K + 32 * (size_t)j, rs);
         }
         if (kGamma) invn = inv_rms[tn];
       }
@@ -323,7 +353,7 @@ template <int kKind>
 __global__ void __launch_bounds__(kRunsThreads) prep_runs_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
     const int* __restrict__ row_index, int T, int K, const float* __restrict__ inv_rms,
-    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out) {
+    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out, Resid rs) {
   __shared__ float gmax_sh;
   allow_dependents();
   const int segs = K >> 5;
@@ -344,7 +374,7 @@ __global__ void __launch_bounds__(kRunsThreads) prep_runs_kernel(
   const int c0 = (int)(g - (long long)t * segs) * 4;
   const int src = active ? (row_index ? row_index[t] : t) : -1;
   float x[32];
-  load_runs<4>(x, X, src, K, c0);
+  load_runs<4>(x, X, src, K, c0, rs);
   if (gamma && src >= 0) normalise_runs<4>(x, gamma, c0, inv_rms[t]);
   quant_runs<4, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, active);
   if (threadIdx.x == 0) depart_and_reset(gmax_bits);
@@ -362,7 +392,7 @@ template <int NC, int kKind, bool kPerToken = false>
 __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
-    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out) {
+    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out, Resid rs) {
   __shared__ double wsum[kFusedMaxThreads / 32];
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
@@ -385,7 +415,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   float x[8 * NC];
   int src = -1;
   if (live && has) src = row_index ? row_index[t] : t;
-  load_runs<NC>(x, X, src, K, c0);
+  load_runs<NC>(x, X, src, K, c0, rs);
   // gamma in flight together with X (not after the row reduction)
   uint4 graw[NC];
   if (gamma && src >= 0) {
@@ -516,7 +546,7 @@ int fused_max_ctas_t(int threads) {
 
 template <int NC, int kKind>
 cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
-                      int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
+                      int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p, Resid rs,
                       cudaStream_t stream, bool* launched) {
   *launched = false;
   const int tpr = (((K >> 3) / NC) + 31) & ~31;
@@ -536,7 +566,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   cfg.blockDim = dim3(threads);
   cfg.stream = stream;
   cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKind>, Xb, Gb, eps, row_index, T, Tp, K, rpc,
-                                     inv_rms, sync, s_g, p);
+                                     inv_rms, sync, s_g, p, rs);
   if (e == cudaSuccess) *launched = true;
   else cudaGetLastError();  // fall back to the two-launch form
   return cudaSuccess;
@@ -547,7 +577,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
 template <int NC>
 cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index,
                                 int T, int Tp, int K, float* inv_rms, unsigned int* sync, float* s_t, QuantPtrs p,
-                                cudaStream_t stream) {
+                                Resid rs, cudaStream_t stream) {
   const int tpr = (((K >> 3) / NC) + 31) & ~31;
   int rpc = 512 / tpr;
   rpc = rpc < 1 ? 1 : rpc;
@@ -556,17 +586,20 @@ cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb
   cfg.blockDim = dim3(rpc * tpr);
   cfg.stream = stream;
   return cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKindSharq, true>, Xb, Gb, eps, row_index, T, Tp, K, rpc, inv_rms,
-                            sync, s_t, p);
+                            sync, s_t, p, rs);
 }
 
 template <int kKind>
 cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
-                          int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p,
+                          int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p, Resid rs,
                           cudaStream_t stream, bool* launched) {
   switch (fused_runs_per_thread(K)) {
-    case 1: return try_fused<1, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
-    case 2: return try_fused<2, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
-    case 4: return try_fused<4, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, stream, launched);
+    case 1: return try_fused<1, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, rs, stream,
+                                          launched);
+    case 2: return try_fused<2, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, rs, stream,
+                                          launched);
+    case 4: return try_fused<4, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, rs, stream,
+                                          launched);
     default: *launched = false; return cudaSuccess;
   }
 }
@@ -607,19 +640,23 @@ bool prep_per_token_supported(int K) { return fused_runs_per_thread(K) != 0; }
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
                         int K, int kind, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
-                        uint8_t* r_meta, cudaStream_t stream) {
+                        uint8_t* r_meta, const void* res, void* res_out, cudaStream_t stream) {
   // gmax_bits[0..3]: device-wide max, barrier arrivals, departures, error
   // word; zero at rest (the kernels reset them), so no memset is needed
   cudaError_t e = cudaSuccess;
   QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf, r_meta};
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
+  const Resid rs{static_cast<const __nv_bfloat16*>(res), static_cast<__nv_bfloat16*>(res_out)};
   if (per_token) {  // s_g: Tp floats, one per row (SharQ mode only)
     if (T == 0) return cudaSuccess;
     switch (fused_runs_per_thread(K)) {
-      case 1: return launch_per_token_nc<1>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream);
-      case 2: return launch_per_token_nc<2>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream);
-      case 4: return launch_per_token_nc<4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream);
+      case 1: return launch_per_token_nc<1>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs,
+                                                stream);
+      case 2: return launch_per_token_nc<2>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs,
+                                                stream);
+      case 4: return launch_per_token_nc<4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs,
+                                                stream);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -628,25 +665,27 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
     bool launched = false;
     switch (kind) {
       case kKindNvfp4:
-        e = try_fused_any<kKindNvfp4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream, &launched);
+        e = try_fused_any<kKindNvfp4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs, stream,
+                               &launched);
         break;
       case kKindSharq:
-        e = try_fused_any<kKindSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream, &launched);
+        e = try_fused_any<kKindSharq>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs, stream,
+                               &launched);
         break;
       case kKindDenseDense:
-        e = try_fused_any<kKindDenseDense>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+        e = try_fused_any<kKindDenseDense>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs, stream,
                                            &launched);
         break;
       case kKindSparseSparse:
-        e = try_fused_any<kKindSparseSparse>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+        e = try_fused_any<kKindSparseSparse>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs, stream,
                                              &launched);
         break;
       case kKindSharqMx:
-        e = try_fused_any<kKindSharqMx>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+        e = try_fused_any<kKindSharqMx>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs, stream,
                                         &launched);
         break;
       case kKindMxfp4:
-        e = try_fused_any<kKindMxfp4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, stream,
+        e = try_fused_any<kKindMxfp4>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, gmax_bits, s_g, p, rs, stream,
                                       &launched);
         break;
       default:
@@ -664,23 +703,22 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   const bool g = Gb != nullptr;
   const int exact = eps < 0x1p-60f ? 1 : 0;
   if (T > 0) {
-    const int per_sm = g ? resident_ctas(prep_rowstats_kernel<true>, kRowThreads, dev)
-                         : resident_ctas(prep_rowstats_kernel<false>, kRowThreads, dev);
+    auto rowstats_fn = g ? (rs.R ? prep_rowstats_kernel<true, true> : prep_rowstats_kernel<true, false>)
+                         : (rs.R ? prep_rowstats_kernel<false, true> : prep_rowstats_kernel<false, false>);
+    const int per_sm = resident_ctas(rowstats_fn, kRowThreads, dev);
     const int rows_per_cta = kRowThreads / 32;
     int grid = (T + rows_per_cta - 1) / rows_per_cta;
     if (grid > sms * per_sm) grid = sms * per_sm;
-    if (g)
-      prep_rowstats_kernel<true><<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms,
-                                                                   gmax_bits);
-    else
-      prep_rowstats_kernel<false><<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms,
-                                                                    gmax_bits);
+    rowstats_fn<<<grid, kRowThreads, 0, stream>>>(Xb, Gb, eps, row_index, T, K, exact, inv_rms, gmax_bits, rs);
   }
+  // once the statistics launch has stored h, the quantizer reads h alone
+  const __nv_bfloat16* Xq = rs.H ? rs.H : Xb;
+  const Resid rq = rs.H ? Resid{} : rs;
   if (kind != kKindSharq && kind != kKindNvfp4) {
     const long long n = (long long)T * (K >> 5);
     const unsigned grid = n > 0 ? (unsigned)((n + kRunsThreads - 1) / kRunsThreads) : 1u;
-#define SHARQ_RUNS(KIND) prep_runs_kernel<KIND><<<grid, kRunsThreads, 0, stream>>>(Xb, Gb, row_index, T, K, \
-                                                                                inv_rms, gmax_bits, s_g, p)
+#define SHARQ_RUNS(KIND) prep_runs_kernel<KIND><<<grid, kRunsThreads, 0, stream>>>(Xq, Gb, row_index, T, K, \
+                                                                                inv_rms, gmax_bits, s_g, p, rq)
     switch (kind) {
       case kKindDenseDense: SHARQ_RUNS(kKindDenseDense); break;
       case kKindSparseSparse: SHARQ_RUNS(kKindSparseSparse); break;
@@ -700,7 +738,7 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   if (rows > T) rows = T;
   const int nw = (int)(rows * G);  // 0 when T == 0: one CTA still publishes s_g
   const int grid = nw > 0 ? (nw + kStripThreads / 32 - 1) / (kStripThreads / 32) : 1;
-  strip_fn<<<grid, kStripThreads, 0, stream>>>(Xb, Gb, row_index, T, K, nw, inv_rms, gmax_bits, s_g, p);
+  strip_fn<<<grid, kStripThreads, 0, stream>>>(Xq, Gb, row_index, T, K, nw, inv_rms, gmax_bits, s_g, p, rq);
   return cudaGetLastError();
 }
 
@@ -749,7 +787,7 @@ cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, con
   e = cudaMemsetAsync(sync, 0, 4 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
   e = launch_prep(X, gamma, eps, row_index, T, Tp, K, kind, per_token, inv, s_g, sync, sp_codes, meta, sp_sf,
-                  r_codes, r_sf, r_meta, stream);
+                  r_codes, r_sf, r_meta, nullptr, nullptr, stream);
   if (e != cudaSuccess) return e;
   // forward the error word to where sharq_linear looks for it
   if (err_out) e = cudaMemcpyAsync(err_out, sync + 3, sizeof(unsigned int), cudaMemcpyDeviceToDevice, stream);

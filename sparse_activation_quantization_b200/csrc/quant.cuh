@@ -241,14 +241,57 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
   }
 }
 
-// load NC runs of 8 (one 16-byte load each) and normalise them
+// The residual-stream update a pre-norm layer performs before its RMSNorm,
+// fused into the preparation (kasblo.com explainer, section 4 on fusing the
+// preparation: RMSNorm and the epilogues before it join the prep kernel):
+// h = bf16_rn(f32(x) + f32(res)), optionally written back as the new stream.
+struct Resid {
+  const __nv_bfloat16* R = nullptr;  // residual stream in, [T][K], or nullptr
+  __nv_bfloat16* H = nullptr;        // updated stream out (may alias R), or nullptr
+};
+
+__device__ __forceinline__ uint4 add_bf16x8(const uint4& a, const uint4& b) {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = __fadd_rn(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16));
+    const float hi = __fadd_rn(__uint_as_float(wa[i] & 0xFFFF0000u), __uint_as_float(wb[i] & 0xFFFF0000u));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[i]) : "f"(hi), "f"(lo));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// N consecutive vectors of 8 bf16 from element offset off, whose x values
+// are already in v: v <- h = x + res, and h written to the updated stream
+// when one is given (by the thread that read res there, so H may alias R).
+template <int N>
+__device__ __forceinline__ void add_residual(uint4 (&v)[N], size_t off, const Resid& rs) {
+  const uint4* rr = reinterpret_cast<const uint4*>(rs.R + off);
+  uint4 r[N];
+#pragma unroll
+  for (int c = 0; c < N; ++c) r[c] = rr[c];
+#pragma unroll
+  for (int c = 0; c < N; ++c) v[c] = add_bf16x8(v[c], r[c]);
+  if (rs.H) {
+    uint4* hh = reinterpret_cast<uint4*>(rs.H + off);
+#pragma unroll
+    for (int c = 0; c < N; ++c) hh[c] = v[c];
+  }
+}
+
+// load NC runs of 8 (one 16-byte load each) of row src (zeros when src < 0);
+// with a residual stream the runs are h = x + res (and h is stored)
 template <int NC>
-__device__ __forceinline__ void load_runs(float (&x)[8 * NC], const __nv_bfloat16* X, int src, int K, int c0) {
+__device__ __forceinline__ void load_runs(float (&x)[8 * NC], const __nv_bfloat16* X, int src, int K, int c0,
+                                          const Resid& rs = Resid{}) {
   if (src >= 0) {
-    const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K) + c0;
+    const size_t off = (size_t)src * K + 8 * (size_t)c0;
+    const uint4* xr = reinterpret_cast<const uint4*>(X + off);
     uint4 raw[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) raw[c] = xr[c];
+    if (rs.R) add_residual<NC>(raw, off, rs);
 #pragma unroll
     for (int c = 0; c < NC; ++c) bf16x8_to_float(raw[c], x + 8 * c);
   } else {
