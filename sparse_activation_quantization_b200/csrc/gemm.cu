@@ -12,24 +12,31 @@
 //               codes, their scales, the weight codes and both weight scale
 //               views -- into a STAGES-deep shared-memory ring, completion
 //               tracked by mbarrier transaction bytes.
-//   warp 1      TMEM allocation; one elected thread issues, per stage:
-//               tcgen05.cp of metadata and scale factors into TMEM, 2 sparse
-//               block-scaled FP4 MMAs (tcgen05.mma.sp kind::mxf4nvf4, K=128
-//               logical each, one scale per 32 logical K) and 4 dense ones
-//               (kind::mxf4nvf4 block16, K=64 each), all into ONE fp32 TMEM
-//               accumulator and all reading the SAME weight tile in shared
-//               memory; tcgen05.commit releases the stage.
+//   warp 1      TMEM allocation; one elected thread issues, per stage,
+//               2 sparse block-scaled FP4 MMAs (tcgen05.mma.sp
+//               kind::mxf4nvf4, K=128 logical each, one scale per 32 logical
+//               K) and 4 dense ones (kind::mxf4nvf4 block16, K=64 each), all
+//               into ONE fp32 TMEM accumulator and all reading the SAME
+//               weight tile in shared memory; tcgen05.commit releases the
+//               stage.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (one row per thread),
 //               y = f32(acc * f32(s_g * s_w)), bf16 or fp32 stores.
+//   warps 6-    copy warps: tcgen05.cp of the stage's metadata and scale
+//               factors into TMEM, spread over 2-4 warps.  A tcgen05.cp costs
+//               about as long as an MMA to issue from one thread, whatever
+//               its size, and copies from different warps proceed side by
+//               side, so the copies of stage i+1 run while the MMAs of stage
+//               i do (the scale region alternates by stage; each copy warp
+//               commits to the region's mbarrier, which the MMA thread waits
+//               on).
 // Split-K (decode shapes, where output tiles alone cannot fill 148 SMs):
 // the S CTAs that share an output tile form one thread-block cluster
-// (1 x 1 x S); each takes a contiguous range of K stages and parks its fp32
-// partial tile in its own (now idle) shared-memory ring.  CTA r of the
+// (1 x 1 x S); each takes a contiguous range of K stages.  CTA r of the
 // cluster owns 1/S of the tile's valid rows: every CTA pushes that slice of
-// its partial into the owner's shared memory with one bulk copy over
-// distributed shared memory (completion = transaction bytes on the owner's
-// mbarrier), and the owner sums the S slices in rank order -- deterministic,
-// no global scratch, no atomics, one bounded wait.
+// its fp32 partial, row by row from registers, into a receive buffer in the
+// owner's shared memory over distributed shared memory, and the owner sums
+// the S slices in rank order -- deterministic, no global scratch, no
+// atomics, one bounded wait.
 // Rows beyond the activation's valid rows are not copied into shared memory
 // (decode: T = 1 moves 1 row of codes, not 128) -- sharq_prep does not even
 // write them; their accumulator rows hold garbage that is never stored (MMA
@@ -43,7 +50,9 @@ namespace sharq {
 
 namespace {
 
-constexpr int kThreads = 192;
+// 6 warps (producer, MMA, 4 epilogue) + the copy warps
+constexpr int kBaseThreads = 192;
+__host__ __device__ constexpr int gemm_threads(int copy_warps) { return kBaseThreads + 32 * copy_warps; }
 
 // Optional phase timeline (compile with -DSHARQ_TRACE): 16 global-timer
 // stamps per CTA -- entry, set-up done, first stage issued, first stage
@@ -94,9 +103,13 @@ struct GemmArgs {
   float eps;
 };
 
-template <int BN, bool kSplit>
+template <int BN, bool kSplit, bool kFused = false>
 struct Cfg {
   static constexpr int kHalves = BN / 128;
+  // copy warps: 4 where registers allow (65536 / threads per thread), 2 for
+  // the register-heavy fused form
+  static constexpr int kCW = kFused ? 2 : 4;
+  static constexpr int kThreadsT = gemm_threads(kCW);
   // split-K CTAs do few stages and need room for the received partial rows
   static constexpr int kStages = (kSplit || BN == 256) ? 3 : 4;
   // shared-memory stage layout (bytes); 1024-aligned where a swizzle needs it
@@ -424,6 +437,43 @@ __device__ __forceinline__ bool fused_prep(const GemmArgs& args, uint8_t* smem, 
   return true;
 }
 
+// The stage's copies into the TMEM scale region sf, weight side then
+// activation side (copy number n is issued by copy warp n % kCW; the
+// counter n runs on across both calls).
+template <class C>
+__device__ __forceinline__ void copies_weight(uint32_t st, uint32_t sf, bool sharq, int cw, int& n) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int h = 0; h < C::kHalves; ++h)
+      if (n++ % C::kCW == cw)
+        tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
+                         smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
+  if (sharq) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h)
+        if (n++ % C::kCW == cw)
+          tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
+                           smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
+  }
+}
+template <class C>
+__device__ __forceinline__ void copies_act(uint32_t st, uint32_t sf, bool sharq, int cw, int& n) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (n++ % C::kCW == cw)
+      tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+  if (sharq) {
+    if (n++ % C::kCW == cw) tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (n++ % C::kCW == cw)
+        tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
+  }
+}
+
 // kFused: the decode form that prepares the activation itself.  The S CTAs
 // of a cluster split K between them: each reduces the row sums of squares and
 // the |Xn| max over its own K-slice and the partials are exchanged over
@@ -433,14 +483,16 @@ __device__ __forceinline__ bool fused_prep(const GemmArgs& args, uint8_t* smem, 
 // layout, while the producer streams the weight half.  No prepared activation
 // goes through HBM and no separate prep kernel runs.
 template <int BN, bool kSplit, bool kFused>
-__global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs args) {
-  using C = Cfg<BN, kSplit>;
+__global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_gemm_kernel(const GemmArgs args) {
+  using C = Cfg<BN, kSplit, kFused>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::kStages];
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ __align__(8) uint64_t recv_bar;
   __shared__ __align__(8) uint64_t afull_bar[kFused ? C::kStages : 1];
+  __shared__ __align__(8) uint64_t sf_full[2];       // scale region b holds stage i's copies (i & 1 == b)
+  __shared__ __align__(8) uint64_t cp_fin[C::kCW];   // each copy warp's last copies
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
   __shared__ int expert_sh;
@@ -470,6 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
+    mbar_init(&sf_full[0], C::kCW);
+    mbar_init(&sf_full[1], C::kCW);
+    for (int c = 0; c < C::kCW; ++c) mbar_init(&cp_fin[c], 1);
     if (kFused) {
       for (int st = 0; st < C::kStages; ++st) mbar_init(&afull_bar[st], 128);  // the epilogue threads
       // statistics exchange: every CTA of the cluster arrives once per row,
@@ -490,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
   if (args.sharq_mode && valid < 128) {
     // Rows past the activation's end are never copied in; give their
     // metadata a valid pattern (pairs 0 and 1) once, in every stage.
-    for (int idx = threadIdx.x; idx < C::kStages * (128 - valid); idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C::kStages * (128 - valid); idx += C::kThreadsT) {
       const int st = idx / (128 - valid), row = valid + idx % (128 - valid);
       *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE + row * 16) =
           make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
@@ -597,38 +652,21 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
         if (i == 0) TRACE_POINT(3);
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
         const uint32_t sf = tmem + C::kColSf0 + (uint32_t)(i & 1) * C::kSfRegion;
-        // scale factors (and metadata) shared memory -> TMEM; the weight side
-        // first (in the fused form it lands before the activation is ready)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int h = 0; h < C::kHalves; ++h)
-            tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
-                             smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
-        if (sharq) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int h = 0; h < C::kHalves; ++h)
-              tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
-                               smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
-        }
-        if (kFused) {
+        if (kFused) {  // the activation half, written by the epilogue warps
           if (!mbar_wait(&afull_bar[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
             record_error(args.err, kErrTimeout);
             abort_sh = 1;
             break;
           }
-          tc_fence_after();
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          tc_cp_32x128b_x4(sf + C::kSfAR + 4 * j, smem_desc(st + C::kOffSFAR + 512 * j, 0, 128, kSwNone));
+        // this stage's scale factors and metadata, copied by the copy warps
+        if (!mbar_wait(&sf_full[i & 1], (i >> 1) & 1, deadline, &abort_sh)) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        tc_fence_after();
         if (sharq) {
-          tc_cp_128x128b(sf + C::kSfE, smem_desc(st + C::kOffE, 0, 128, kSwNone));
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-            tc_cp_32x128b_x4(sf + C::kSfASP + 4 * j, smem_desc(st + C::kOffSFASP + 512 * j, 0, 128, kSwNone));
           // sparse backbone: 2 x (128 x BN x 128 logical K)
 #pragma unroll
           for (int j = 0; j < 2; ++j)
@@ -646,6 +684,43 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       }
       tc_commit(&acc_bar);  // accumulator complete (or everything issued so far, on abort)
       TRACE_POINT(4);
+    }
+  } else if (warp >= 6) {
+    // ---------------------------------------------------- copy warps ----
+    if (lane == 0) {
+      const int cw = warp - 6;
+      for (int i = 0; i < nks; ++i) {
+        const int s = i % C::kStages;
+        // the stage's data has landed, and the MMAs of stage i - 2 (the
+        // same scale region) have completed
+        if (!mbar_wait(&full_bar[s], (i / C::kStages) & 1, deadline, &abort_sh) ||
+            (i >= 2 &&
+             !mbar_wait(&empty_bar[(i - 2) % C::kStages], ((i - 2) / C::kStages) & 1, deadline, &abort_sh))) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t sf = tmem + C::kColSf0 + (uint32_t)(i & 1) * C::kSfRegion;
+        int n = 0;
+        copies_weight<C>(st, sf, sharq, cw, n);
+        if (kFused) {  // the activation half comes from the epilogue warps
+          if (!mbar_wait(&afull_bar[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
+        }
+        copies_act<C>(st, sf, sharq, cw, n);
+        tc_commit(&sf_full[i & 1]);
+      }
+      // every copy this warp issued has landed before the TMEM is freed
+      tc_commit(&cp_fin[cw]);
+      const uint64_t lim = globaltimer_ns() + kWaitLimitNs;
+      while (!mbar_try_wait(&cp_fin[cw], 0) && globaltimer_ns() < lim) {
+      }
     }
   } else {
     // ------------------------------------------------------- epilogue ----
@@ -715,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_kernel(const GemmArgs 
       const float sw = args.s_w[expert];
       const float* recv = reinterpret_cast<const float*>(smem + C::kRingBytes);
       constexpr int q4 = BN / 4;
-      for (int idx = threadIdx.x; idx < my_n * q4; idx += kThreads) {
+      for (int idx = threadIdx.x; idx < my_n * q4; idx += C::kThreadsT) {
         const int r = idx / q4, c4 = idx - r * q4;
         const float* p = recv + r * C::kRowFloats + 4 * c4;
         float4 acc = *reinterpret_cast<const float4*>(p);
@@ -768,6 +843,10 @@ enum : int {
 template <int BN, int kG>
 struct PCfg {
   static constexpr int kHalves = BN / 128;
+  // copy warps: 4 for 128-wide tiles; 2 for 256-wide ones, whose epilogue
+  // keeps a 256-column row in registers (65536 / 256 threads per thread)
+  static constexpr int kCW = BN == 256 ? 2 : 4;
+  static constexpr int kThreadsT = gemm_threads(kCW);
   static constexpr bool kMx = kG == kGemmSharqMx || kG == kGemmMxfp4;
   static constexpr bool kHas1 = kG != kGemmNvfp4 && kG != kGemmMxfp4;  // first operand (backbone)
   static constexpr bool kSp1 = kG != kGemmDenseDense;                 // ... sparse
@@ -820,14 +899,59 @@ struct PCfg {
   static_assert(BN + 2 * kSfRegion <= 512, "TMEM overflow");
 };
 
+// The scale-factor and metadata copies of one stage of the persistent
+// kernel (shared memory -> TMEM scale region sf): the weight views the
+// operand set needs, then each activation operand's metadata and scales.
+// Copy number n is issued by copy warp n % kCW.
+template <class C>
+__device__ __forceinline__ void stage_copies(uint32_t st, uint32_t sf, int cw) {
+  int n = 0;
+  auto cp4 = [&](uint32_t taddr, uint32_t saddr) {
+    if (n++ % C::kCW == cw) tc_cp_32x128b_x4(taddr, smem_desc(saddr, 0, 128, kSwNone));
+  };
+  auto cpm = [&](uint32_t taddr, uint32_t saddr) {
+    if (n++ % C::kCW == cw) tc_cp_128x128b(taddr, smem_desc(saddr, 0, 128, kSwNone));
+  };
+  // atoms (512 B, 4 TMEM columns) per 256-K stage: NVFP4 sparse 2 / dense 4,
+  // MXFP4 sparse 1 / dense 2
+  constexpr int kAtSp = C::kMx ? 1 : 2, kAtDn = C::kMx ? 2 : 4;
+  if (C::kB32) {
+#pragma unroll
+    for (int j = 0; j < kAtSp; ++j)
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h)
+        cp4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h, st + C::kOffSFB32 + h * C::kSfSp + 512 * j);
+  }
+  if (C::kB16) {
+#pragma unroll
+    for (int j = 0; j < kAtDn; ++j)
+#pragma unroll
+      for (int h = 0; h < C::kHalves; ++h)
+        cp4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h, st + C::kOffSFB16 + h * C::kSfDn + 512 * j);
+  }
+  if (C::kHas1) {
+    if (C::kSp1) cpm(sf + C::kSfE1, st + C::kOffE1);
+#pragma unroll
+    for (int j = 0; j < (C::kSp1 ? kAtSp : kAtDn); ++j) cp4(sf + C::kSfS1 + 4 * j, st + C::kOffS1 + 512 * j);
+  }
+  if (C::kHas2) {
+    if (C::kSp2) cpm(sf + C::kSfE2, st + C::kOffE2);
+#pragma unroll
+    for (int j = 0; j < (C::kSp2 ? kAtSp : kAtDn); ++j) cp4(sf + C::kSfS2 + 4 * j, st + C::kOffS2 + 512 * j);
+  }
+}
+
 template <int BN, int kG>
-__global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(const GemmArgs args, int m_tiles) {
+__global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
+    sharq_gemm_persistent_kernel(const GemmArgs args, int m_tiles) {
   using C = PCfg<BN, kG>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::kStages];
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
   __shared__ __align__(8) uint64_t acc_full;
   __shared__ __align__(8) uint64_t acc_empty;
+  __shared__ __align__(8) uint64_t sf_full[2];      // scale region b holds stage g's copies (g & 1 == b)
+  __shared__ __align__(8) uint64_t cp_fin[C::kCW];  // each copy warp's last copies
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
 
@@ -845,6 +969,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
     }
     mbar_init(&acc_full, 1);
     mbar_init(&acc_empty, 128);  // every epilogue thread, once per tile
+    mbar_init(&sf_full[0], C::kCW);
+    mbar_init(&sf_full[1], C::kCW);
+    for (int c = 0; c < C::kCW; ++c) mbar_init(&cp_fin[c], 1);
     fence_mbar_init();
     abort_sh = 0;
   }
@@ -856,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
     // Metadata rows past a partial tile's valid rows are never copied in: give
     // every row a valid pattern (pairs 0 and 1) once; later tiles leave
     // metadata written by sharq_prep there, which is valid as well.
-    for (int idx = threadIdx.x; idx < C::kStages * 128; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < C::kStages * 128; idx += C::kThreadsT) {
       const int st = idx >> 7, row = idx & 127;
       const uint4 v = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
       if (C::kE1) *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE1 + row * 16) = v;
@@ -943,24 +1070,20 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
             break;
           }
           tc_fence_after();
+          // this stage's scale factors and metadata, copied by the copy warps
+          if (!mbar_wait(&sf_full[g & 1u], (g >> 1) & 1u, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
           const uint32_t st = smem_u32(smem + s * C::kStageBytes);
           const uint32_t sf = tmem + C::kColSf0 + (g & 1u) * C::kSfRegion;
           bool acc = i > 0;  // the tile's first MMA overwrites the accumulator
-          // a sparse operand: 2 x (128 x BN x 128 logical K); its metadata
-          // and scales, and the weight's per-32 view (once per stage), right
-          // before each MMA so copies overlap the previous MMA
-          auto sparse_op = [&](uint32_t a_off, uint32_t e_off, uint32_t s_off, uint32_t e_col, uint32_t s_col,
-                               bool copy_b) {
-            tc_cp_128x128b(sf + e_col, smem_desc(st + e_off, 0, 128, kSwNone));
+          // a sparse operand: 2 x (128 x BN x 128 logical K), weight per-32 view
+          auto sparse_op = [&](uint32_t a_off, uint32_t e_col, uint32_t s_col) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-              tc_cp_32x128b_x4(sf + s_col + 4 * j, smem_desc(st + s_off + 512 * j, 0, 128, kSwNone));
-              if (copy_b) {
-#pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                  tc_cp_32x128b_x4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h,
-                                   smem_desc(st + C::kOffSFB32 + h * kSf32Tile + 512 * j, 0, 128, kSwNone));
-              }
               mma_sp_nvf4(tmem + C::kColAcc, smem_desc(st + a_off + 32 * j, 16, 512, kSw64),
                           smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + e_col + 2 * j, idesc_sp,
                           sf + s_col + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, acc ? 1u : 0u);
@@ -968,16 +1091,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
             }
           };
           // a dense operand: 4 x (128 x BN x 64 K), weight per-16 view
-          auto dense_op = [&](uint32_t a_off, uint32_t s_off, uint32_t s_col, bool copy_b) {
+          auto dense_op = [&](uint32_t a_off, uint32_t s_col) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              tc_cp_32x128b_x4(sf + s_col + 4 * j, smem_desc(st + s_off + 512 * j, 0, 128, kSwNone));
-              if (copy_b) {
-#pragma unroll
-                for (int h = 0; h < C::kHalves; ++h)
-                  tc_cp_32x128b_x4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h,
-                                   smem_desc(st + C::kOffSFB16 + h * kSf16Tile + 512 * j, 0, 128, kSwNone));
-              }
               mma_nvf4(tmem + C::kColAcc, smem_desc(st + a_off + 32 * j, 16, 1024, kSw128),
                        smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + s_col + 4 * j,
                        sf + C::kSfB16 + j * C::kSfbCols, acc ? 1u : 0u);
@@ -988,12 +1104,7 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
           // = two MMAs' worth; the scale-factor ID (byte 0 or 2 of the
           // column) picks this MMA's pair, in the descriptor and in bits
           // 30-31 of the TMEM scale address
-          auto sparse_op_mx = [&](uint32_t a_off, uint32_t e_off, uint32_t s_off, uint32_t e_col, uint32_t s_col) {
-            tc_cp_128x128b(sf + e_col, smem_desc(st + e_off, 0, 128, kSwNone));
-            tc_cp_32x128b_x4(sf + s_col, smem_desc(st + s_off, 0, 128, kSwNone));
-#pragma unroll
-            for (int h = 0; h < C::kHalves; ++h)
-              tc_cp_32x128b_x4(sf + C::kSfB32 + 4 * h, smem_desc(st + C::kOffSFB32 + h * C::kSfSp, 0, 128, kSwNone));
+          auto sparse_op_mx = [&](uint32_t a_off, uint32_t e_col, uint32_t s_col) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const uint32_t id = 2u * j;
@@ -1004,14 +1115,9 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
               acc = true;
             }
           };
-          auto dense_op_mx = [&](uint32_t a_off, uint32_t s_off, uint32_t s_col) {
+          auto dense_op_mx = [&](uint32_t a_off, uint32_t s_col) {
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
-              tc_cp_32x128b_x4(sf + s_col + 4 * a, smem_desc(st + s_off + 512 * a, 0, 128, kSwNone));
-#pragma unroll
-              for (int h = 0; h < C::kHalves; ++h)
-                tc_cp_32x128b_x4(sf + C::kSfB16 + a * C::kSfbCols + 4 * h,
-                                 smem_desc(st + C::kOffSFB16 + h * C::kSfDn + 512 * a, 0, 128, kSwNone));
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 const int j = 2 * a + q;
@@ -1025,23 +1131,52 @@ __global__ void __launch_bounds__(kThreads, 1) sharq_gemm_persistent_kernel(cons
             }
           };
           if (C::kMx) {
-            if (C::kHas1) sparse_op_mx(C::kOffA1, C::kOffE1, C::kOffS1, C::kSfE1, C::kSfS1);
-            dense_op_mx(C::kOffA2, C::kOffS2, C::kSfS2);
+            if (C::kHas1) sparse_op_mx(C::kOffA1, C::kSfE1, C::kSfS1);
+            dense_op_mx(C::kOffA2, C::kSfS2);
           } else {
             if (C::kHas1) {
-              if (C::kSp1) sparse_op(C::kOffA1, C::kOffE1, C::kOffS1, C::kSfE1, C::kSfS1, true);
-              else dense_op(C::kOffA1, C::kOffS1, C::kSfS1, true);
+              if (C::kSp1) sparse_op(C::kOffA1, C::kSfE1, C::kSfS1);
+              else dense_op(C::kOffA1, C::kSfS1);
             }
             if (C::kHas2) {
-              // the weight view is already in TMEM when both operands share it
-              if (C::kSp2) sparse_op(C::kOffA2, C::kOffE2, C::kOffS2, C::kSfE2, C::kSfS2, !(C::kHas1 && C::kSp1));
-              else dense_op(C::kOffA2, C::kOffS2, C::kSfS2, !(C::kHas1 && !C::kSp1));
+              if (C::kSp2) sparse_op(C::kOffA2, C::kSfE2, C::kSfS2);
+              else dense_op(C::kOffA2, C::kSfS2);
             }
           }
           tc_commit(&empty_bar[s]);
         }
         tc_commit(&acc_full);  // accumulator of this tile complete
         ++k;
+      }
+    }
+  } else if (warp >= 6) {
+    // ---------------------------------------------------- copy warps ----
+    if (lane == 0) {
+      const int cw = warp - 6;
+      uint32_t g = 0;  // stage counter across tiles, as the MMA warp's
+      for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
+        if (tile_expert(args, tile / n_tiles) < 0) continue;
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages;
+          // the stage's data has landed, and the MMAs of stage g - 2 (the
+          // same scale region) have completed
+          if (!mbar_wait(&full_bar[s], (g / C::kStages) & 1, deadline, &abort_sh) ||
+              (g >= 2 && !mbar_wait(&empty_bar[(g - 2) % C::kStages], ((g - 2) / C::kStages) & 1, deadline,
+                                    &abort_sh))) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
+          stage_copies<C>(smem_u32(smem + s * C::kStageBytes), tmem + C::kColSf0 + (g & 1u) * C::kSfRegion, cw);
+          tc_commit(&sf_full[g & 1u]);
+        }
+      }
+      // every copy this warp issued has landed before the TMEM is freed
+      tc_commit(&cp_fin[cw]);
+      const uint64_t lim = globaltimer_ns() + kWaitLimitNs;
+      while (!mbar_try_wait(&cp_fin[cw], 0) && globaltimer_ns() < lim) {
       }
     }
   } else {
@@ -1130,7 +1265,7 @@ cudaError_t launch_persistent(const GemmArgs& a, int m_tiles, cudaStream_t strea
   const long long ntiles = (long long)m_tiles * (a.D / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(ntiles < sms[dev] ? ntiles : sms[dev]));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(C::kThreadsT);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1157,7 +1292,7 @@ cudaError_t launch_persistent_mode(const GemmArgs& a, int m_tiles, int gmode, cu
 
 template <int BN, bool kSplit, bool kFused>
 cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
-  using C = Cfg<BN, kSplit>;
+  using C = Cfg<BN, kSplit, kFused>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1170,7 +1305,7 @@ cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.D / BN, m_tiles, kSplit ? a.splits : 1);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(C::kThreadsT);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
