@@ -58,14 +58,12 @@ def prep_alg_bytes(T, K):
     return T * K * 2 + Tp * K * 0.90625
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernel per launch, from the ncu capture summarised in
-# profiles/sharq_gemm_qproj_decode.md; reset to None whenever that kernel
-# changes until it is captured again.
-# DRAM bytes (read + write) per launch of the dominant GEMM, from ncu captures
-# of this script's workloads (profiles/sharq_gemm_qproj_decode.md,
-# profiles/sharq_gemm_persistent_mlp2048.md); None where none was taken.
-NCU_TRAFFIC = {"q_proj_T128": 10470912, "gate_T2048": 65486592, "up_T2048": 65486592}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
+# the dominant GEMM, from ncu captures of this script's workloads
+# (profiles/sharq_gemm_qproj_decode.md, profiles/sharq_gemm_persistent_mlp2048.md);
+# None where none was taken.  Reset an entry whenever its kernel changes,
+# until it is captured again.
+NCU_TRAFFIC = {"q_proj_T128": 10474752, "gate_T2048": 64406272, "up_T2048": 57812992}
 
 
 def read_peaks():
@@ -504,7 +502,7 @@ def run_gpu(args, world, rank, local):
     if args.workload == "mlp":
         from sparse_activation_quantization_b200 import peak
         pk = peak.fp4_peaks()
-        roof = {"kernel": f"sharq_gemm_kernel ({dom.name})", "bound": "tensor",
+        roof = {"kernel": f"sharq_gemm_persistent_kernel ({dom.name})", "bound": "tensor",
                 "achieved": per[dom.name]["gemm_tflops"], "peak": pk["effective_pflops"] * 1e3,
                 "unit": "TFLOP/s", "frac": per[dom.name]["gemm_tflops"] / (pk["effective_pflops"] * 1e3),
                 "peak_kind": "measured tcgen05 FP4 (dense %.2f, sparse %.2f PFLOP/s; dual-GEMM effective)"
