@@ -465,6 +465,84 @@ def residual_add(x, res):
     return bf16_round((x + r).astype(np.float32))
 
 
+def bf16_round_f64(x):
+    """Round float64 to the nearest bfloat16 (ties to even) in ONE rounding,
+    not through float32; returns float32.  bfloat16 keeps 8 significant bits
+    and float32's exponent range: the quantum of a value in [2^e, 2^(e+1)) is
+    2^(e-7), and 2^-133 below 2^-126.  Finite inputs; the sign of zero is
+    kept."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                     # x = m 2^e, 1/2 <= |m| < 1
+    q = np.maximum(e, -125) - 8            # log2 of the quantum
+    r = np.ldexp(np.round(np.ldexp(x, -q)), q)  # x / 2^q is exact; np.round ties to even
+    return np.copysign(r, x).astype(np.float32)
+
+
+def _bf16_midpoint(x):
+    """True where float64 x lies exactly halfway between two bfloat16s."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    q = np.maximum(e, -125) - 8
+    t = np.ldexp(x, -q)
+    return (t - np.floor(t)) == 0.5
+
+
+def silu_bf16(g):
+    """SiLU of bf16 values rounded once to bfloat16 (ties cannot occur: silu(g)
+    is transcendental for g != 0).  silu(g) = g / (1 + e^-g), evaluated in
+    float64 in three forms that avoid overflow and cancellation:
+      g >= 1:   g / (1 + e^-g)
+      g <= -1:  g e^g / (1 + e^g)
+      |g| < 1:  g/2 + d with d = (g/2) tanh(g/2) >= 0 (silu(g) - g/2 = d), kept
+                as the float64 pair hi + lo (Knuth's two-sum), so that a hi
+                lying exactly on a bf16 midpoint -- g/2 for tiny g -- rounds
+                in the direction of lo.
+    silu(+inf) = +inf, silu(-inf) = -0, NaN stays NaN.  Input: float32 holding
+    bf16 values; returns float32 holding bf16 values."""
+    with np.errstate(invalid="ignore"):  # signalling NaN patterns
+        g = np.asarray(g, dtype=np.float32).astype(np.float64)
+    fin = np.isfinite(g)
+    gf = np.where(fin, g, 0.0)
+    with np.errstate(over="ignore", under="ignore", invalid="ignore"):
+        e = np.exp(-np.abs(gf))                              # in (0, 1]
+        big = np.where(gf >= 0, gf / (1.0 + e), gf * e / (1.0 + e))
+        a = gf / 2.0                                         # exact
+        d = a * np.tanh(a)
+        hi = a + d
+        bb = hi - a
+        lo = (a - (hi - bb)) + (d - bb)                      # hi + lo = a + d exactly
+    small = np.abs(gf) < 1.0
+    hi = np.where(small, hi, big)
+    lo = np.where(small, lo, 0.0)
+    r = bf16_round_f64(hi).astype(np.float64)
+    # a hi exactly halfway between two bf16s goes to the neighbour on lo's side
+    # (half a quantum away; the quantum is that of the lower neighbour)
+    tie = _bf16_midpoint(hi) & (lo != 0.0)
+    _, ex = np.frexp(hi)
+    quantum = np.ldexp(1.0, np.maximum(ex, -125) - 8)
+    r = np.where(tie, hi + np.sign(lo) * quantum / 2.0, r)
+    # silu(g) has the sign of g (silu(g) / g = sigmoid(g) > 0), zeros included
+    out = np.copysign(r, gf).astype(np.float32)
+    out = np.where(fin, out, np.where(np.isnan(g), np.float32(np.nan),
+                                      np.where(g > 0, np.float32(np.inf), np.float32(-0.0))))
+    return out.astype(np.float32)
+
+
+def silu_mul(gate, up):
+    """The SwiGLU product the down projection of a Llama-style MLP takes,
+    fused into its preparation step (the kasblo.com explainer, section 4 on
+    fusing the preparation: the epilogues before it join the prep kernel):
+        h = bf16_rn(f32(silu_bf16(gate) * up))
+    for bf16 gate and up (float32 arrays holding bf16 values) -- the SiLU
+    rounded to bf16 as a bf16 framework stores it, then the bf16 product (two
+    bf16 values multiply exactly in float32 unless the product underflows;
+    the float32 product is rounded to bf16)."""
+    s = silu_bf16(gate)
+    u = np.asarray(up, dtype=np.float32)
+    with np.errstate(over="ignore", under="ignore"):
+        return bf16_round((s * u).astype(np.float32))
+
+
 def prep_nvfp4(x, gamma=None, eps=1e-5):
     """Plain NVFP4 preparation, the comparator the SharQ evaluation reports
     as "NVFP4" (xllm-io review, Table 1; the kasblo.com explainer lists the
