@@ -256,6 +256,27 @@ int sharq_prep_residual(const void *d_X, const void *d_res, void *d_res_out, con
                         const sharq_act *a, sharq_stream_t stream);
 
 /*
+ * sharq_prep_silu_mul - sharq_prep of the SwiGLU product a down projection
+ * takes.  In a Llama-style MLP the down projection's input is SiLU(gate) * up;
+ * the kasblo.com explainer (section 4, on fusing the preparation) counts the
+ * epilogues before the preparation among what the prep kernel takes in.  The
+ * prep input here is, element by element,
+ *     h = bf16_rn(f32(silu_bf16(gate)) * f32(up))
+ * where silu_bf16(g) is silu(g) = g / (1 + e^-g) correctly rounded to bf16
+ * (silu(+-0) = +-0, silu(+inf) = +inf, silu(-inf) = -0), as a bf16 framework
+ * stores SiLU(gate) before multiplying by up.  Outputs in `a` are those of
+ * sharq_prep on h, bit for bit.
+ * d_gate, d_up: bf16 [a->T][K] row-major.
+ * d_h:      bf16 [a->T][K] that receives h, or NULL.  It may be d_up itself;
+ *           it must not overlap d_gate, nor overlap d_up other than exactly.
+ * d_gamma, eps, a: as for sharq_prep (the down projection's input is not
+ *           normalised: pass NULL).  Row gathering is not offered.
+ * Errors: as sharq_prep_residual.
+ */
+int sharq_prep_silu_mul(const void *d_gate, const void *d_up, void *d_h, const void *d_gamma, float eps,
+                        const sharq_act *a, sharq_stream_t stream);
+
+/*
  * sharq_prep_noalloc - sharq_prep for callers that cannot allocate device
  * memory at run time: code inside a region being captured into a CUDA graph
  * (where cudaMalloc is not allowed), or a host framework whose memory

@@ -23,7 +23,7 @@ __all__ = [
     "sharq_weight_view", "sharq_act_view", "sharq_pack_weight", "sharq_prep",
     "sharq_linear", "sharq_linear_grouped", "sharq_check_status",
     "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc", "sharq_prep_linear", "prep_linear",
-    "sharq_prep_residual",
+    "sharq_prep_residual", "sharq_prep_silu_mul",
     "PackedWeight", "PreparedAct", "Workspace", "linear", "EXPORTED_SYMBOLS",
 ]
 
@@ -45,6 +45,7 @@ EXPORTED_SYMBOLS = (
     "sharq_act_view", "sharq_pack_weight", "sharq_prep", "sharq_linear", "sharq_linear_grouped",
     "sharq_check_status", "sharq_status_string", "sharq_abi_version", "sharq_prep_noalloc",
     "sharq_prep_linear", "sharq_weight_bytes_fmt", "sharq_weight_view_fmt", "sharq_prep_residual",
+    "sharq_prep_silu_mul",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +96,7 @@ def lib():
             "sharq_prep": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
             "sharq_prep_noalloc": (i, [vp, vp, ctypes.c_float, vp, A, vp]),
             "sharq_prep_residual": (i, [vp, vp, vp, vp, ctypes.c_float, A, vp]),
+            "sharq_prep_silu_mul": (i, [vp, vp, vp, vp, ctypes.c_float, A, vp]),
             "sharq_linear": (i, [A, W, vp, i, vp, sz, vp]),
             "sharq_prep_linear": (i, [vp, vp, ctypes.c_float, i, A, W, vp, i, vp, sz, vp]),
             "sharq_linear_grouped": (i, [A, vp, W, vp, i, vp, sz, vp]),
@@ -175,6 +177,11 @@ def sharq_prep_noalloc(d_X, d_gamma, eps, d_row_index, a, stream):
 def sharq_prep_residual(d_X, d_res, d_res_out, d_gamma, eps, a, stream):
     return _check(lib().sharq_prep_residual(d_X, d_res, d_res_out, d_gamma, eps, ctypes.byref(a), stream),
                   "sharq_prep_residual")
+
+
+def sharq_prep_silu_mul(d_gate, d_up, d_h, d_gamma, eps, a, stream):
+    return _check(lib().sharq_prep_silu_mul(d_gate, d_up, d_h, d_gamma, eps, ctypes.byref(a), stream),
+                  "sharq_prep_silu_mul")
 
 
 def sharq_linear(a, w, d_Y, out_dtype, d_ws, ws_bytes, stream):
@@ -273,6 +280,15 @@ class PreparedAct:
         sharq_prep_residual(X.data_ptr() if X is not None else None,
                             res.data_ptr() if res is not None else None,
                             res_out.data_ptr() if res_out is not None else None,
+                            gamma.data_ptr() if gamma is not None else None, float(eps),
+                            self.view, _stream_ptr(stream))
+        return self
+
+    def prep_silu_mul(self, gate, up, h_out=None, gamma=None, eps=1e-5, stream=None):
+        """sharq_prep of h = bf16(silu(gate) * up); h goes to h_out when given."""
+        sharq_prep_silu_mul(gate.data_ptr() if gate is not None else None,
+                            up.data_ptr() if up is not None else None,
+                            h_out.data_ptr() if h_out is not None else None,
                             gamma.data_ptr() if gamma is not None else None, float(eps),
                             self.view, _stream_ptr(stream))
         return self

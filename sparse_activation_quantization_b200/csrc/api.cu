@@ -13,7 +13,7 @@ namespace sharq {
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp, int K,
                         int kind, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
-                        uint8_t* r_meta, const void* res, void* res_out, cudaStream_t stream);
+                        uint8_t* r_meta, int epi_kind, const void* epi_b, void* epi_h, cudaStream_t stream);
 cudaError_t launch_pack_weight(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf32, uint8_t* sf16,
                                float* s_w, unsigned int* amax_bits, cudaStream_t stream);
 cudaError_t launch_pack_weight_mx(const void* W, int K, int D, int E, uint8_t* codes, uint8_t* sf64, uint8_t* sf32,
@@ -331,8 +331,9 @@ int sharq_pack_weight(const void* d_W, const sharq_weight* w, sharq_stream_t str
 }
 
 namespace {
+// epi_kind: 0 none, 1 residual add (h = x + b), 2 SwiGLU product (h = silu(x) * b)
 int prep_common(const void* d_X, const void* d_gamma, float eps, const int* d_row_index, const sharq_act* a,
-                const void* d_res, void* d_res_out, sharq_stream_t stream) {
+                int epi_kind, const void* d_b, void* d_h, sharq_stream_t stream) {
   int st = act_ok(a);
   if (st) return st;
   if (a->T > 0 && (!d_X || !aligned(d_X, 16))) return SHARQ_ERR_INVALID_ARG;
@@ -345,24 +346,36 @@ int prep_common(const void* d_X, const void* d_gamma, float eps, const int* d_ro
       d_X, d_gamma, eps, d_row_index, a->T, a->Tp, a->K, prep_kind(a->mode), per_token, a->inv_rms, a->s_g,
       a->gmax_bits, static_cast<uint8_t*>(a->sp_codes), static_cast<uint8_t*>(a->meta),
       static_cast<uint8_t*>(a->sp_sf), static_cast<uint8_t*>(a->r_codes), static_cast<uint8_t*>(a->r_sf),
-      static_cast<uint8_t*>(a->r_meta), d_res, d_res_out, reinterpret_cast<cudaStream_t>(stream));
+      static_cast<uint8_t*>(a->r_meta), epi_kind, d_b, d_h, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }
 }  // namespace
 
 int sharq_prep(const void* d_X, const void* d_gamma, float eps, const int* d_row_index, const sharq_act* a,
                sharq_stream_t stream) {
-  return prep_common(d_X, d_gamma, eps, d_row_index, a, nullptr, nullptr, stream);
+  return prep_common(d_X, d_gamma, eps, d_row_index, a, 0, nullptr, nullptr, stream);
 }
+
+namespace {
+int prep_epilogue(int kind, const void* d_A, const void* d_B, void* d_H, const void* d_gamma, float eps,
+                  const sharq_act* a, sharq_stream_t stream) {
+  if (!a) return SHARQ_ERR_INVALID_ARG;
+  if (a->T > 0 && (!d_B || !aligned(d_B, 16))) return SHARQ_ERR_INVALID_ARG;
+  if (d_H && !aligned(d_H, 16)) return SHARQ_ERR_INVALID_ARG;
+  if (a->T > 0 && d_H == d_A) return SHARQ_ERR_INVALID_ARG;  // may alias d_B, not d_A
+  if (a->T == 0) return prep_common(d_A, d_gamma, eps, nullptr, a, 0, nullptr, nullptr, stream);
+  return prep_common(d_A, d_gamma, eps, nullptr, a, kind, d_B, d_H, stream);
+}
+}  // namespace
 
 int sharq_prep_residual(const void* d_X, const void* d_res, void* d_res_out, const void* d_gamma, float eps,
                         const sharq_act* a, sharq_stream_t stream) {
-  if (!a) return SHARQ_ERR_INVALID_ARG;
-  if (a->T > 0 && (!d_res || !aligned(d_res, 16))) return SHARQ_ERR_INVALID_ARG;
-  if (d_res_out && !aligned(d_res_out, 16)) return SHARQ_ERR_INVALID_ARG;
-  if (a->T > 0 && d_res_out == d_X) return SHARQ_ERR_INVALID_ARG;  // may alias d_res, not d_X
-  return prep_common(d_X, d_gamma, eps, nullptr, a, a->T > 0 ? d_res : nullptr, a->T > 0 ? d_res_out : nullptr,
-                     stream);
+  return prep_epilogue(1, d_X, d_res, d_res_out, d_gamma, eps, a, stream);
+}
+
+int sharq_prep_silu_mul(const void* d_gate, const void* d_up, void* d_h, const void* d_gamma, float eps,
+                        const sharq_act* a, sharq_stream_t stream) {
+  return prep_epilogue(2, d_gate, d_up, d_h, d_gamma, eps, a, stream);
 }
 
 int sharq_prep_noalloc(const void* d_X, const void* d_gamma, float eps, const int* d_row_index,

@@ -82,15 +82,15 @@ __device__ __forceinline__ double bf16_lo_x2p128(uint32_t w) {
   return __hiloint2double((int)(((w << 13) & 0x0FFFE000u) | 0x40000000u), 0);
 }
 
-// v[u] (vector c0 + 32 u of a row, zeros past its end) <- h = x + res, and
-// h stored to hr (the same vectors of the updated stream) when hr is given
+// v[u] (vector c0 + 32 u of a row, zeros past its end) <- h, and h stored to
+// hr (the same vectors of the output) when hr is given
 template <int N>
-__device__ __forceinline__ void add_row_residual(uint4 (&v)[N], const uint4* rr, uint4* hr, int c0, int nv) {
+__device__ __forceinline__ void row_epi(uint4 (&v)[N], const uint4* rr, uint4* hr, int c0, int nv, int kind) {
   uint4 r[N];
 #pragma unroll
   for (int u = 0; u < N; ++u) r[u] = c0 + 32 * u < nv ? rr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
 #pragma unroll
-  for (int u = 0; u < N; ++u) v[u] = add_bf16x8(v[u], r[u]);
+  for (int u = 0; u < N; ++u) v[u] = epi8(v[u], r[u], kind);
   if (hr) {
 #pragma unroll
     for (int u = 0; u < N; ++u)
@@ -109,10 +109,10 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 //   RMSNorm rows: float64 sum of squares -> 1/rms, then max |Xn| (Xn
 //   recomputed from L1/L2 as in the quantizer: bf16(f32(f32(x/rms) g))).
 //   Rows without RMSNorm: max |x| on packed bf16 bits.
-// With a residual stream (kResid) the rows are h = x + res: the first pass
-// forms h (4 vectors of x and 4 of res in flight per lane) and, when the
-// updated stream is wanted, stores it there; the second pass and the
-// quantizer launch then read h alone.  Each element of h is stored and
+// With an epilogue (kEpi: the residual add or the SwiGLU product) the rows
+// are h: the first pass forms h (4 vectors of X and 4 of B in flight per
+// lane) and, when an output is given, stores it there; the second pass and
+// the quantizer launch then read h alone.  Each element of h is stored and
 // re-read by the lane that formed it.
 // The device-wide max goes to gmax_bits[0] with one atomicMax per CTA.
 // Sum of squares: each square of a bf16 value is exact in float64, and the
@@ -122,12 +122,12 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 // row -- far below one ulp of mean(x^2) + eps for any eps >= 2^-60, where
 // the result is that of an exact-input float64 sum in this lane order.  For
 // eps < 2^-60 (`exact`) the elements are converted exactly instead.
-template <bool kGamma, bool kResid>
+template <bool kGamma, bool kEpi>
 __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int K, int exact, float* __restrict__ inv_rms,
-    unsigned int* __restrict__ gmax_bits, Resid rs) {
-  constexpr int kC = kResid ? kRowChunk / 2 : kRowChunk;  // vectors of the row in flight per lane
+    unsigned int* __restrict__ gmax_bits, Epi rs) {
+  constexpr int kC = kEpi ? kRowChunk / 2 : kRowChunk;  // vectors of the row in flight per lane
   __shared__ uint32_t wmax[kRowThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = gridDim.x * (kRowThreads / 32);
@@ -140,15 +140,15 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
       continue;
     }
     const uint4* xr = reinterpret_cast<const uint4*>(X + (size_t)src * K);
-    const uint4* rr = kResid ? reinterpret_cast<const uint4*>(rs.R + (size_t)src * K) : nullptr;
-    uint4* hr = kResid && rs.H ? reinterpret_cast<uint4*>(rs.H + (size_t)src * K) : nullptr;
+    const uint4* rr = kEpi ? reinterpret_cast<const uint4*>(rs.B + (size_t)src * K) : nullptr;
+    uint4* hr = kEpi && rs.H ? reinterpret_cast<uint4*>(rs.H + (size_t)src * K) : nullptr;
     if (kGamma) {
       double acc0 = 0.0, acc1 = 0.0;
       for (int c0 = lane; c0 < nv; c0 += 32 * kC) {
         uint4 v[kC];
 #pragma unroll
         for (int u = 0; u < kC; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
-        if (kResid) add_row_residual<kC>(v, rr, hr, c0, nv);
+        if (kEpi) row_epi<kC>(v, rr, hr, c0, nv, rs.kind);
         if (!exact) {
 #pragma unroll
           for (int u = 0; u < kC; ++u) {
@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
           v[u] = in ? sr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
           g[u] = in ? gr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
         }
-        if (kResid && !hr) add_row_residual<kC>(v, rr, nullptr, c0, nv);
+        if (kEpi && !hr) row_epi<kC>(v, rr, nullptr, c0, nv, rs.kind);
 #pragma unroll
         for (int u = 0; u < kC; ++u) {
           const uint32_t xw[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
         uint4 v[kC];
 #pragma unroll
         for (int u = 0; u < kC; ++u) v[u] = c0 + 32 * u < nv ? xr[c0 + 32 * u] : make_uint4(0, 0, 0, 0);
-        if (kResid) add_row_residual<kC>(v, rr, hr, c0, nv);
+        if (kEpi) row_epi<kC>(v, rr, hr, c0, nv, rs.kind);
 #pragma unroll
         for (int u = 0; u < kC; ++u) {
           mx = vmax_u16x2(mx, v[u].x & 0x7FFF7FFFu);
@@ -265,7 +265,7 @@ template <bool kSharq, bool kGamma>
 __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
     const int* __restrict__ row_index, int T, int K, int nw, const float* __restrict__ inv_rms,
-    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out, Resid rs) {
+    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out, Epi rs) {
   __shared__ float2 tab[128];
   __shared__ uint32_t msel[16];
   allow_dependents();
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
 #pragma unroll
     for (int u = 0; u < 4; ++u)
       cur[u] = (active && src >= 0) ? reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * (size_t)j)[u] : z4;
-    if (rs.R && active && src >= 0) add_residual<4>(cur, (size_t)src * K + 32 * (size_t)j, rs);
+    if (rs.kind && active && src >= 0) apply_epi<4>(cur, (size_t)src * K + 32 * (size_t)j, rs);
     if (kGamma) inv = inv_rms[t];
     while (t < T) {
       // prefetch the next row of this warp
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
         if (active && srcn >= 0) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) nxt[u] = reinterpret_cast<const uint4*>(X + (size_t)srcn * K + 32 * (size_t)j)[u];
-          if (rs.R) add_residual<4>(nxt, (size_t)srcn * K + 32 * (size_t)j, rs);
+          if (rs.kind) apply_epi<4>(nxt, (size_t)srcn * K + 32 * (size_t)j, rs);
         }
         if (kGamma) invn = inv_rms[tn];
       }
@@ -353,7 +353,7 @@ template <int kKind>
 __global__ void __launch_bounds__(kRunsThreads) prep_runs_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma,
     const int* __restrict__ row_index, int T, int K, const float* __restrict__ inv_rms,
-    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out, Resid rs) {
+    unsigned int* __restrict__ gmax_bits, float* __restrict__ s_g_out, QuantPtrs out, Epi rs) {
   __shared__ float gmax_sh;
   allow_dependents();
   const int segs = K >> 5;
@@ -392,7 +392,7 @@ template <int NC, int kKind, bool kPerToken = false>
 __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
-    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out, Resid rs) {
+    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out, Epi rs) {
   __shared__ double wsum[kFusedMaxThreads / 32];
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
@@ -546,7 +546,7 @@ int fused_max_ctas_t(int threads) {
 
 template <int NC, int kKind>
 cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
-                      int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p, Resid rs,
+                      int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p, Epi rs,
                       cudaStream_t stream, bool* launched) {
   *launched = false;
   const int tpr = (((K >> 3) / NC) + 31) & ~31;
@@ -577,7 +577,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
 template <int NC>
 cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index,
                                 int T, int Tp, int K, float* inv_rms, unsigned int* sync, float* s_t, QuantPtrs p,
-                                Resid rs, cudaStream_t stream) {
+                                Epi rs, cudaStream_t stream) {
   const int tpr = (((K >> 3) / NC) + 31) & ~31;
   int rpc = 512 / tpr;
   rpc = rpc < 1 ? 1 : rpc;
@@ -591,7 +591,7 @@ cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb
 
 template <int kKind>
 cudaError_t try_fused_any(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float eps, const int* row_index, int T,
-                          int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p, Resid rs,
+                          int Tp, int K, float* inv_rms, unsigned int* sync, float* s_g, QuantPtrs p, Epi rs,
                           cudaStream_t stream, bool* launched) {
   switch (fused_runs_per_thread(K)) {
     case 1: return try_fused<1, kKind>(Xb, Gb, eps, row_index, T, Tp, K, inv_rms, sync, s_g, p, rs, stream,
@@ -640,14 +640,14 @@ bool prep_per_token_supported(int K) { return fused_runs_per_thread(K) != 0; }
 cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
                         int K, int kind, bool per_token, float* inv_rms, float* s_g, unsigned int* gmax_bits,
                         uint8_t* sp_codes, uint8_t* meta, uint8_t* sp_sf, uint8_t* r_codes, uint8_t* r_sf,
-                        uint8_t* r_meta, const void* res, void* res_out, cudaStream_t stream) {
+                        uint8_t* r_meta, int epi_kind, const void* epi_b, void* epi_h, cudaStream_t stream) {
   // gmax_bits[0..3]: device-wide max, barrier arrivals, departures, error
   // word; zero at rest (the kernels reset them), so no memset is needed
   cudaError_t e = cudaSuccess;
   QuantPtrs p{sp_codes, meta, sp_sf, r_codes, r_sf, r_meta};
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Gb = static_cast<const __nv_bfloat16*>(gamma);
-  const Resid rs{static_cast<const __nv_bfloat16*>(res), static_cast<__nv_bfloat16*>(res_out)};
+  const Epi rs{static_cast<const __nv_bfloat16*>(epi_b), static_cast<__nv_bfloat16*>(epi_h), epi_b ? epi_kind : kEpiNone};
   if (per_token) {  // s_g: Tp floats, one per row (SharQ mode only)
     if (T == 0) return cudaSuccess;
     switch (fused_runs_per_thread(K)) {
@@ -703,8 +703,8 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   const bool g = Gb != nullptr;
   const int exact = eps < 0x1p-60f ? 1 : 0;
   if (T > 0) {
-    auto rowstats_fn = g ? (rs.R ? prep_rowstats_kernel<true, true> : prep_rowstats_kernel<true, false>)
-                         : (rs.R ? prep_rowstats_kernel<false, true> : prep_rowstats_kernel<false, false>);
+    auto rowstats_fn = g ? (rs.kind ? prep_rowstats_kernel<true, true> : prep_rowstats_kernel<true, false>)
+                         : (rs.kind ? prep_rowstats_kernel<false, true> : prep_rowstats_kernel<false, false>);
     const int per_sm = resident_ctas(rowstats_fn, kRowThreads, dev);
     const int rows_per_cta = kRowThreads / 32;
     int grid = (T + rows_per_cta - 1) / rows_per_cta;
@@ -713,7 +713,7 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   }
   // once the statistics launch has stored h, the quantizer reads h alone
   const __nv_bfloat16* Xq = rs.H ? rs.H : Xb;
-  const Resid rq = rs.H ? Resid{} : rs;
+  const Epi rq = rs.H ? Epi{} : rs;
   if (kind != kKindSharq && kind != kKindNvfp4) {
     const long long n = (long long)T * (K >> 5);
     const unsigned grid = n > 0 ? (unsigned)((n + kRunsThreads - 1) / kRunsThreads) : 1u;
@@ -787,7 +787,7 @@ cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, con
   e = cudaMemsetAsync(sync, 0, 4 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
   e = launch_prep(X, gamma, eps, row_index, T, Tp, K, kind, per_token, inv, s_g, sync, sp_codes, meta, sp_sf,
-                  r_codes, r_sf, r_meta, nullptr, nullptr, stream);
+                  r_codes, r_sf, r_meta, 0, nullptr, nullptr, stream);
   if (e != cudaSuccess) return e;
   // forward the error word to where sharq_linear looks for it
   if (err_out) e = cudaMemcpyAsync(err_out, sync + 3, sizeof(unsigned int), cudaMemcpyDeviceToDevice, stream);

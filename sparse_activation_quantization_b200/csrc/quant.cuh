@@ -241,14 +241,89 @@ __device__ __forceinline__ void quant_runs(const float (&x)[8 * NC], int t, int 
   }
 }
 
-// The residual-stream update a pre-norm layer performs before its RMSNorm,
-// fused into the preparation (kasblo.com explainer, section 4 on fusing the
-// preparation: RMSNorm and the epilogues before it join the prep kernel):
-// h = bf16_rn(f32(x) + f32(res)), optionally written back as the new stream.
-struct Resid {
-  const __nv_bfloat16* R = nullptr;  // residual stream in, [T][K], or nullptr
-  __nv_bfloat16* H = nullptr;        // updated stream out (may alias R), or nullptr
+// Epilogues of the preceding operation, fused into the preparation
+// (kasblo.com explainer, section 4 on fusing the preparation: RMSNorm and the
+// epilogues before it join the prep kernel).  The prep input becomes h, formed
+// element by element from two bf16 tensors A (the prep's X) and B:
+//   kEpiAdd:     h = bf16_rn(f32(a) + f32(b))  -- the residual-stream update
+//                before a pre-norm layer's RMSNorm (a = sublayer output, b =
+//                residual stream);
+//   kEpiSiluMul: h = bf16_rn(silu_bf16(a) * f32(b))  -- the SwiGLU product a
+//                down projection takes (a = gate, b = up), with silu_bf16 the
+//                correctly rounded bf16 of silu(a) = a / (1 + e^-a).
+// h is optionally written out (H may alias B: each element is read and
+// written by the same thread).
+enum : int { kEpiNone = 0, kEpiAdd = 1, kEpiSiluMul = 2 };
+struct Epi {
+  const __nv_bfloat16* B = nullptr;  // second input, [T][K], or nullptr
+  __nv_bfloat16* H = nullptr;        // h out (may alias B), or nullptr
+  int kind = kEpiNone;
 };
+
+// silu(g) rounded to bf16 by way of float64 and round-to-odd (the slow path
+// of silu_bf16; out of line so that its registers stay out of the callers').
+//   |g| < 1:   g/2 + d with d = (g/2) tanh(g/2) >= 0, kept as the pair hi + lo
+//              (Knuth's two-sum), so that hi on a bf16 midpoint -- g/2 for
+//              tiny g -- rounds the way lo points;
+//   g >= 1:    g / (1 + e^-g);   g <= -1:  g e^g / (1 + e^g).
+// hi + lo goes to float32 rounded to odd (truncate, then set the last bit
+// when inexact), then to bf16 to nearest even: float32 keeps more than two
+// extra bits, so the two roundings give the correctly rounded bf16.
+static __device__ __noinline__ float silu_bf16_f64(float g) {
+  if (isinf(g)) return g > 0.0f ? g : -0.0f;  // silu(+inf) = +inf, silu(-inf) = -0
+  const double gd = g;
+  double hi, lo = 0.0;
+  if (fabs(gd) < 1.0) {
+    const double a = 0.5 * gd, d = a * tanh(a);
+    hi = a + d;
+    const double bb = hi - a;
+    lo = (a - (hi - bb)) + (d - bb);
+  } else if (gd >= 1.0) {
+    hi = gd / (1.0 + exp(-gd));
+  } else {
+    const double e = exp(gd);
+    hi = gd * e / (1.0 + e);
+  }
+  const double mag = fabs(hi);
+  const double b = hi < 0.0 ? -lo : lo;  // lo along the magnitude
+  uint32_t fb = __float_as_uint(__double2float_rz(mag));
+  if ((double)__uint_as_float(fb) != mag) fb |= 1u;  // strictly between two floats
+  else if (b > 0.0) fb |= 1u;
+  else if (b < 0.0 && fb != 0u) fb = (fb - 1u) | 1u;
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(__uint_as_float(fb)));
+  // silu(g) has the sign of g (silu(g) / g = sigmoid(g) > 0), zeros included
+  return __uint_as_float(((uint32_t)r << 16) | (__float_as_uint(g) & 0x80000000u));
+}
+
+// silu(g) correctly rounded to bf16, returned as a float32 holding it.  Fast
+// path in float32, branch-free: e = expf(-|g|) in (0, 1] (CUDA's expf, max
+// error 2 ulp), numerator g (g >= 0) or g e (g < 0), one __fdividef by 1 + e
+// (max error 2 ulp for divisors in [1, 2]): the result is within about 7
+// float32 ulps of silu(g), which fixes its bf16 rounding unless it lies within
+// 16 ulps of a bf16 rounding midpoint (low 16 bits near 0x8000).  Those
+// inputs, g < -80 (e near float32's subnormals), the infinities and NaN take
+// the float64 path.
+__device__ __forceinline__ float silu_bf16(float g) {
+  const float e = expf(-fabsf(g));
+  const float num = g >= 0.0f ? g : __fmul_rn(g, e);
+  const float s = __fdividef(num, __fadd_rn(1.0f, e));
+  const uint32_t low = __float_as_uint(s) & 0xFFFFu;
+  if (low + 16u - 0x8000u > 32u && g > -80.0f && g < INFINITY) {  // |low - 0x8000| > 16
+    // s is not near a midpoint, so rounding half up in magnitude is rounding
+    // to nearest
+    return __uint_as_float((__float_as_uint(s) + 0x8000u) & 0xFFFF0000u);
+  }
+  return silu_bf16_f64(g);
+}
+
+__device__ __forceinline__ uint32_t silu_mul_bf16x2(uint32_t g2, uint32_t u2) {
+  const float h_lo = __fmul_rn(silu_bf16(__uint_as_float(g2 << 16)), __uint_as_float(u2 << 16));
+  const float h_hi = __fmul_rn(silu_bf16(__uint_as_float(g2 & 0xFFFF0000u)), __uint_as_float(u2 & 0xFFFF0000u));
+  uint32_t o;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o) : "f"(h_hi), "f"(h_lo));
+  return o;
+}
 
 __device__ __forceinline__ uint4 add_bf16x8(const uint4& a, const uint4& b) {
   const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
@@ -262,36 +337,43 @@ __device__ __forceinline__ uint4 add_bf16x8(const uint4& a, const uint4& b) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// N consecutive vectors of 8 bf16 from element offset off, whose x values
-// are already in v: v <- h = x + res, and h written to the updated stream
-// when one is given (by the thread that read res there, so H may alias R).
+// h for 8 consecutive elements (a from X, b from B)
+__device__ __forceinline__ uint4 epi8(const uint4& a, const uint4& b, int kind) {
+  if (kind == kEpiAdd) return add_bf16x8(a, b);
+  return make_uint4(silu_mul_bf16x2(a.x, b.x), silu_mul_bf16x2(a.y, b.y), silu_mul_bf16x2(a.z, b.z),
+                    silu_mul_bf16x2(a.w, b.w));
+}
+
+// N consecutive vectors of 8 bf16 from element offset off, whose X values
+// are already in v: v <- h, and h written out when an output is given (by the
+// thread that read B there, so H may alias B).
 template <int N>
-__device__ __forceinline__ void add_residual(uint4 (&v)[N], size_t off, const Resid& rs) {
-  const uint4* rr = reinterpret_cast<const uint4*>(rs.R + off);
+__device__ __forceinline__ void apply_epi(uint4 (&v)[N], size_t off, const Epi& ep) {
+  const uint4* bp = reinterpret_cast<const uint4*>(ep.B + off);
   uint4 r[N];
 #pragma unroll
-  for (int c = 0; c < N; ++c) r[c] = rr[c];
+  for (int c = 0; c < N; ++c) r[c] = bp[c];
 #pragma unroll
-  for (int c = 0; c < N; ++c) v[c] = add_bf16x8(v[c], r[c]);
-  if (rs.H) {
-    uint4* hh = reinterpret_cast<uint4*>(rs.H + off);
+  for (int c = 0; c < N; ++c) v[c] = epi8(v[c], r[c], ep.kind);
+  if (ep.H) {
+    uint4* hh = reinterpret_cast<uint4*>(ep.H + off);
 #pragma unroll
     for (int c = 0; c < N; ++c) hh[c] = v[c];
   }
 }
 
 // load NC runs of 8 (one 16-byte load each) of row src (zeros when src < 0);
-// with a residual stream the runs are h = x + res (and h is stored)
+// with an epilogue the runs are h (and h is stored when an output is given)
 template <int NC>
 __device__ __forceinline__ void load_runs(float (&x)[8 * NC], const __nv_bfloat16* X, int src, int K, int c0,
-                                          const Resid& rs = Resid{}) {
+                                          const Epi& ep = Epi{}) {
   if (src >= 0) {
     const size_t off = (size_t)src * K + 8 * (size_t)c0;
     const uint4* xr = reinterpret_cast<const uint4*>(X + off);
     uint4 raw[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) raw[c] = xr[c];
-    if (rs.R) add_residual<NC>(raw, off, rs);
+    if (ep.kind) apply_epi<NC>(raw, off, ep);
 #pragma unroll
     for (int c = 0; c < NC; ++c) bf16x8_to_float(raw[c], x + 8 * c);
   } else {
