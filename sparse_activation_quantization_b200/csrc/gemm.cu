@@ -126,7 +126,9 @@ struct Cfg {
   // split-K receive buffer (outside the ring, so peers may write into it
   // while this CTA's own mainloop still runs): S slices of ceil(rows/S) rows
   static constexpr int kRowFloats = BN + 4;  // padded: conflict-free float4 access
-  static constexpr int kRecvRows = 136;      // >= 128 + S - 1 for S <= 8
+  // receive buffer: S slices of ceil(rows / S) + 1 rows x BN floats, at most
+  // (128 + 2 S - 1) x 512 bytes for S <= 4
+  static constexpr int kRecvRows = 136;
   static constexpr int kRecvBytes = kSplit ? kRecvRows * kRowFloats * 4 : 0;
   static constexpr int kSmemBytes = kRingBytes + kRecvBytes + 1024;
   // TMEM columns: the accumulator, then two buffers (alternating by stage)
@@ -148,6 +150,7 @@ struct Cfg {
   static_assert(kColsUsed <= 512, "TMEM overflow");
   static_assert(kSmemBytes <= 232448, "shared memory overflow");
   static_assert(!kSplit || BN == 128, "split-K uses 128-wide tiles");
+  static_assert(!kSplit || kRecvBytes >= (128 + 2 * 4 - 1) * (BN / 4) * 16, "split-K receive buffer");
 };
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -751,11 +754,14 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
       }
     } else {
       // push this split's partial row straight from registers into the
-      // owner CTA's receive buffer (slot [my rank][row within the slice])
+      // owner CTA's receive buffer, laid out [sender][column quad][row of the
+      // slice (+1 pad)][4 floats]: the lanes of a warp hold consecutive rows,
+      // so each of their stores is one contiguous 512-byte run
       const int owner = rl / max(rows_per, 1);
+      const int rp = rows_per + 1;  // padded: the owner's quad-major reads stay conflict-free
       const uint32_t dst =
           rl < valid ? mapa_shared(smem_u32(smem + C::kRingBytes) +
-                                       (uint32_t)((split * rows_per + (rl - owner * rows_per)) * C::kRowFloats * 4),
+                                       (uint32_t)((split * (BN / 4) * rp + (rl - owner * rows_per)) * 16),
                                    (uint32_t)owner)
                      : 0u;
 #pragma unroll 1
@@ -766,7 +772,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
         if (rl < valid) {
 #pragma unroll
           for (int q = 0; q < 32; q += 4)
-            st_cluster_f4(dst + (uint32_t)(c + q) * 4u, __uint_as_float(v[q]), __uint_as_float(v[q + 1]),
+            st_cluster_f4(dst + (uint32_t)((c + q) / 4 * rp) * 16u, __uint_as_float(v[q]), __uint_as_float(v[q + 1]),
                           __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
         }
       }
@@ -790,12 +796,13 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
       const float sw = args.s_w[expert];
       const float* recv = reinterpret_cast<const float*>(smem + C::kRingBytes);
       constexpr int q4 = BN / 4;
+      const int rp = rows_per + 1;
       for (int idx = threadIdx.x; idx < my_n * q4; idx += C::kThreadsT) {
-        const int r = idx / q4, c4 = idx - r * q4;
-        const float* p = recv + r * C::kRowFloats + 4 * c4;
+        const int r = idx / q4, c4 = idx - r * q4;  // consecutive threads: consecutive columns of a row
+        const float* p = recv + ((size_t)c4 * rp + r) * 4;
         float4 acc = *reinterpret_cast<const float4*>(p);
         for (int s2 = 1; s2 < S; ++s2) {
-          const float4 q = *reinterpret_cast<const float4*>(p + (size_t)s2 * rows_per * C::kRowFloats);
+          const float4 q = *reinterpret_cast<const float4*>(p + (size_t)s2 * q4 * rp * 4);
           acc.x = __fadd_rn(acc.x, q.x);
           acc.y = __fadd_rn(acc.y, q.y);
           acc.z = __fadd_rn(acc.z, q.z);
@@ -1368,14 +1375,14 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   if (X_fused) {  // fused decode form
     if (T > 32 || m_tiles != 1 || gmode != kGemmSharq || group_offsets || per_token) return cudaErrorInvalidValue;
     if (splits > 1) {
-      if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
+      if (bn != 128 || splits > 4) return cudaErrorInvalidValue;
       return launch_cfg<128, true, true>(a, m_tiles, stream);
     }
     return bn == 256 ? launch_cfg<256, false, true>(a, m_tiles, stream)
                      : launch_cfg<128, false, true>(a, m_tiles, stream);
   }
   if (splits > 1 && two_way) {
-    if (bn != 128 || splits > 8) return cudaErrorInvalidValue;
+    if (bn != 128 || splits > 4) return cudaErrorInvalidValue;
     return launch_cfg<128, true, false>(a, m_tiles, stream);
   }
   // the Table-5 modes run the persistent form at every size
