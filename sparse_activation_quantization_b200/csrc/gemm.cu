@@ -25,10 +25,12 @@
 //               factors into TMEM, spread over 2-4 warps.  A tcgen05.cp costs
 //               about as long as an MMA to issue from one thread, whatever
 //               its size, and copies from different warps proceed side by
-//               side, so the copies of stage i+1 run while the MMAs of stage
-//               i do (the scale region alternates by stage; each copy warp
-//               commits to the region's mbarrier, which the MMA thread waits
-//               on).
+//               side, so the copies of later stages run while the MMAs of
+//               stage i do.  Each ring slot has its own TMEM scale region, so
+//               a stage's copies start as soon as its data has landed (a
+//               copy's completion takes a good fraction of a microsecond);
+//               each copy warp commits to the slot's mbarrier, which the MMA
+//               thread waits on.
 // Split-K (decode shapes, where output tiles alone cannot fill 148 SMs):
 // the S CTAs that share an output tile form one thread-block cluster
 // (1 x 1 x S); each takes a contiguous range of K stages.  CTA r of the
@@ -131,15 +133,15 @@ struct Cfg {
   static constexpr int kRecvRows = 136;
   static constexpr int kRecvBytes = kSplit ? kRecvRows * kRowFloats * 4 : 0;
   static constexpr int kSmemBytes = kRingBytes + kRecvBytes + 1024;
-  // TMEM columns: the accumulator, then two buffers (alternating by stage)
-  // of metadata + scale factors, so the copies for stage i+1 never
-  // overwrite columns the MMAs of stage i still read.
+  // TMEM columns: the accumulator, then one region of metadata + scale
+  // factors per ring slot (a slot is refilled only after the MMAs that read
+  // its region have completed).
   static constexpr uint32_t kColAcc = 0;
   static constexpr uint32_t kSfbCols = BN / 32;  // per MMA: one column per 32 rows of B
   static constexpr uint32_t kSfE = 0, kSfASP = 8, kSfAR = 16, kSfB32 = 32, kSfB16 = 32 + 2 * kSfbCols;
   static constexpr uint32_t kSfRegion = 32 + 6 * kSfbCols;
   static constexpr uint32_t kColSf0 = BN;
-  static constexpr uint32_t kColsUsed = BN + 2 * kSfRegion;
+  static constexpr uint32_t kColsUsed = BN + kStages * kSfRegion;
   static constexpr uint32_t kTmemCols = kColsUsed <= 256 ? 256 : 512;
   // transaction bytes per stage (activation code copies trimmed to valid rows)
   static constexpr uint32_t kTxSharq = BN * 128 + kHalves * (kSf32Tile + kSf16Tile) + kCodesTile + kSpTile +
@@ -494,7 +496,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ __align__(8) uint64_t recv_bar;
   __shared__ __align__(8) uint64_t afull_bar[kFused ? C::kStages : 1];
-  __shared__ __align__(8) uint64_t sf_full[2];       // scale region b holds stage i's copies (i & 1 == b)
+  __shared__ __align__(8) uint64_t sf_full[C::kStages];  // ring slot s: its stage's copies have landed
   __shared__ __align__(8) uint64_t cp_fin[C::kCW];   // each copy warp's last copies
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
@@ -525,8 +527,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_bar, 1);
-    mbar_init(&sf_full[0], C::kCW);
-    mbar_init(&sf_full[1], C::kCW);
+    for (int st = 0; st < C::kStages; ++st) mbar_init(&sf_full[st], C::kCW);
     for (int c = 0; c < C::kCW; ++c) mbar_init(&cp_fin[c], 1);
     if (kFused) {
       for (int st = 0; st < C::kStages; ++st) mbar_init(&afull_bar[st], 128);  // the epilogue threads
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
         tc_fence_after();
         if (i == 0) TRACE_POINT(3);
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t sf = tmem + C::kColSf0 + (uint32_t)(i & 1) * C::kSfRegion;
+        const uint32_t sf = tmem + C::kColSf0 + (uint32_t)s * C::kSfRegion;
         if (kFused) {  // the activation half, written by the epilogue warps
           if (!mbar_wait(&afull_bar[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
             record_error(args.err, kErrTimeout);
@@ -663,7 +664,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
           }
         }
         // this stage's scale factors and metadata, copied by the copy warps
-        if (!mbar_wait(&sf_full[i & 1], (i >> 1) & 1, deadline, &abort_sh)) {
+        if (!mbar_wait(&sf_full[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
           record_error(args.err, kErrTimeout);
           abort_sh = 1;
           break;
@@ -694,18 +695,16 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
       const int cw = warp - 6;
       for (int i = 0; i < nks; ++i) {
         const int s = i % C::kStages;
-        // the stage's data has landed, and the MMAs of stage i - 2 (the
-        // same scale region) have completed
-        if (!mbar_wait(&full_bar[s], (i / C::kStages) & 1, deadline, &abort_sh) ||
-            (i >= 2 &&
-             !mbar_wait(&empty_bar[(i - 2) % C::kStages], ((i - 2) / C::kStages) & 1, deadline, &abort_sh))) {
+        // the stage's data has landed (the slot, and with it its scale
+        // region, is refilled only after the MMAs that read it completed)
+        if (!mbar_wait(&full_bar[s], (i / C::kStages) & 1, deadline, &abort_sh)) {
           record_error(args.err, kErrTimeout);
           abort_sh = 1;
           break;
         }
         tc_fence_after();
         const uint32_t st = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t sf = tmem + C::kColSf0 + (uint32_t)(i & 1) * C::kSfRegion;
+        const uint32_t sf = tmem + C::kColSf0 + (uint32_t)s * C::kSfRegion;
         int n = 0;
         copies_weight<C>(st, sf, sharq, cw, n);
         if (kFused) {  // the activation half comes from the epilogue warps
@@ -717,7 +716,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
           tc_fence_after();
         }
         copies_act<C>(st, sf, sharq, cw, n);
-        tc_commit(&sf_full[i & 1]);
+        tc_commit(&sf_full[s]);
       }
       // every copy this warp issued has landed before the TMEM is freed
       tc_commit(&cp_fin[cw]);
@@ -887,15 +886,15 @@ struct PCfg {
   static constexpr int kStageBytes = (kOffSFB16 + (kB16 ? kHalves * kSfDn : 0) + 1023) / 1024 * 1024;
   static constexpr int kStages = (BN == 128 && 4 * kStageBytes + 1024 <= 232448) ? 4 : 3;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-  // TMEM: accumulator, then two scale regions (alternating by stage) of 32
-  // activation columns + the weight scale columns
+  // TMEM: accumulator, then one scale region per ring slot: 32 activation
+  // columns + the weight scale columns
   static constexpr uint32_t kColAcc = 0;
   static constexpr uint32_t kSfbCols = BN / 32;
   static constexpr uint32_t kSfE1 = 0, kSfE2 = 4, kSfS1 = kSp1 ? 8 : 0, kSfS2 = 16;
   static constexpr uint32_t kSfB32 = 32, kSfB16 = 32 + 2 * kSfbCols;
   static constexpr uint32_t kSfRegion = 32 + 6 * kSfbCols;
   static constexpr uint32_t kColSf0 = BN;
-  static constexpr uint32_t kTmemCols = BN + 2 * kSfRegion <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = BN + kStages * kSfRegion <= 256 ? 256 : 512;
   // transaction bytes per stage with `rows` valid activation rows
   __host__ __device__ static constexpr uint32_t tx(uint32_t rows) {
     return BN * 128 + (kB32 ? kHalves * kSfSp : 0) + (kB16 ? kHalves * kSfDn : 0) +
@@ -903,7 +902,7 @@ struct PCfg {
   }
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory overflow");
-  static_assert(BN + 2 * kSfRegion <= 512, "TMEM overflow");
+  static_assert(BN + kStages * kSfRegion <= 512, "TMEM overflow");
 };
 
 // The scale-factor and metadata copies of one stage of the persistent
@@ -957,7 +956,7 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
   __shared__ __align__(8) uint64_t empty_bar[C::kStages];
   __shared__ __align__(8) uint64_t acc_full;
   __shared__ __align__(8) uint64_t acc_empty;
-  __shared__ __align__(8) uint64_t sf_full[2];      // scale region b holds stage g's copies (g & 1 == b)
+  __shared__ __align__(8) uint64_t sf_full[C::kStages];  // ring slot s: its stage's copies have landed
   __shared__ __align__(8) uint64_t cp_fin[C::kCW];  // each copy warp's last copies
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_sh;
@@ -976,8 +975,7 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
     }
     mbar_init(&acc_full, 1);
     mbar_init(&acc_empty, 128);  // every epilogue thread, once per tile
-    mbar_init(&sf_full[0], C::kCW);
-    mbar_init(&sf_full[1], C::kCW);
+    for (int st = 0; st < C::kStages; ++st) mbar_init(&sf_full[st], C::kCW);
     for (int c = 0; c < C::kCW; ++c) mbar_init(&cp_fin[c], 1);
     fence_mbar_init();
     abort_sh = 0;
@@ -1078,14 +1076,14 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
           }
           tc_fence_after();
           // this stage's scale factors and metadata, copied by the copy warps
-          if (!mbar_wait(&sf_full[g & 1u], (g >> 1) & 1u, deadline, &abort_sh)) {
+          if (!mbar_wait(&sf_full[s], (g / C::kStages) & 1, deadline, &abort_sh)) {
             record_error(args.err, kErrTimeout);
             abort_sh = 1;
             break;
           }
           tc_fence_after();
           const uint32_t st = smem_u32(smem + s * C::kStageBytes);
-          const uint32_t sf = tmem + C::kColSf0 + (g & 1u) * C::kSfRegion;
+          const uint32_t sf = tmem + C::kColSf0 + (uint32_t)s * C::kSfRegion;
           bool acc = i > 0;  // the tile's first MMA overwrites the accumulator
           // a sparse operand: 2 x (128 x BN x 128 logical K), weight per-32 view
           auto sparse_op = [&](uint32_t a_off, uint32_t e_col, uint32_t s_col) {
@@ -1166,18 +1164,16 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
         const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
         for (int i = 0; i < KS; ++i, ++g) {
           const int s = g % C::kStages;
-          // the stage's data has landed, and the MMAs of stage g - 2 (the
-          // same scale region) have completed
-          if (!mbar_wait(&full_bar[s], (g / C::kStages) & 1, deadline, &abort_sh) ||
-              (g >= 2 && !mbar_wait(&empty_bar[(g - 2) % C::kStages], ((g - 2) / C::kStages) & 1, deadline,
-                                    &abort_sh))) {
+          // the stage's data has landed (the slot, and with it its scale
+          // region, is refilled only after the MMAs that read it completed)
+          if (!mbar_wait(&full_bar[s], (g / C::kStages) & 1, deadline, &abort_sh)) {
             record_error(args.err, kErrTimeout);
             abort_sh = 1;
             break;
           }
           tc_fence_after();
-          stage_copies<C>(smem_u32(smem + s * C::kStageBytes), tmem + C::kColSf0 + (g & 1u) * C::kSfRegion, cw);
-          tc_commit(&sf_full[g & 1u]);
+          stage_copies<C>(smem_u32(smem + s * C::kStageBytes), tmem + C::kColSf0 + (uint32_t)s * C::kSfRegion, cw);
+          tc_commit(&sf_full[s]);
         }
       }
       // every copy this warp issued has landed before the TMEM is freed
