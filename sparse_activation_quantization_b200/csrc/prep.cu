@@ -383,6 +383,7 @@ __global__ void __launch_bounds__(kRunsThreads) prep_runs_kernel(
 // ---------------------------------------------------------------------------
 // Single-launch form (cooperative grid; whole rows inside a CTA).
 constexpr int kFusedMaxThreads = 1024;
+constexpr int kMaxClusterCtas = 16;  // cluster form: at most 16 CTAs (non-portable size above 8)
 constexpr uint64_t kBarrierLimitNs = 2000000000ull;
 
 template <int NC>
@@ -392,12 +393,16 @@ template <int NC, int kKind, bool kPerToken = false>
 __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ gamma, float eps,
     const int* __restrict__ row_index, int T, int Tp, int K, int rows_per_cta, float* __restrict__ inv_rms,
-    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out, Epi rs) {
+    unsigned int* sync, float* __restrict__ s_g_out, QuantPtrs out, Epi rs, int cluster) {
   __shared__ double wsum[kFusedMaxThreads / 32];
+  __shared__ float cmax[kMaxClusterCtas];  // cluster form: every CTA's max
   __shared__ float wmax[kFusedMaxThreads / 32];
   __shared__ float gmax_sh;
   PREP_TRACE(0);
   allow_dependents();
+  // cluster form: announce this CTA (its shared memory exists) before any
+  // peer stores into it; the matching wait comes just before those stores
+  if (cluster) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   if (blockIdx.x == 0 && threadIdx.x == 0) sync[3] = 0u;  // error word of the previous prep
   // threads per row, padded to whole warps (a warp never spans two rows);
   // the padding lanes hold zeros and store nothing
@@ -466,7 +471,28 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     if (live) quant_runs<NC, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
     return;
   }
-  if (threadIdx.x == 0) {
+  if (cluster) {
+    // The grid is one thread-block cluster: every CTA writes its max into
+    // every CTA's shared memory, and one hardware cluster barrier (release /
+    // acquire) replaces the global-memory grid barrier.
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every peer has started
+    if (threadIdx.x == 0) {
+      float m = 0.0f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+      const uint32_t dst = smem_u32(&cmax[blockIdx.x]);
+      for (uint32_t r = 0; r < gridDim.x; ++r) {
+        const uint32_t a = mapa_shared(dst, r);
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(m) : "memory");
+      }
+    }
+    cluster_sync_all();
+    if (threadIdx.x == 0) {
+      float m = 0.0f;
+      for (int r = 0; r < (int)gridDim.x; ++r) m = fmaxf(m, cmax[r]);
+      gmax_sh = m;
+      PREP_TRACE(2);
+    }
+  } else if (threadIdx.x == 0) {
     float m = 0.0f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
     if (gridDim.x == 1) {
@@ -499,7 +525,7 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;
   // rows past T: whole warps (rows span whole warps), so they can skip
   if (live) quant_runs<NC, kKind>(x, t, c0, K, s, __fmul_rn(6.0f, s), out, has);
-  if (threadIdx.x == 0 && gridDim.x > 1) depart_and_reset(sync);
+  if (threadIdx.x == 0 && gridDim.x > 1 && !cluster) depart_and_reset(sync);
 #ifdef SHARQ_TRACE
   __syncthreads();
   PREP_TRACE(3);
@@ -550,6 +576,44 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
                       cudaStream_t stream, bool* launched) {
   *launched = false;
   const int tpr = (((K >> 3) / NC) + 31) & ~31;
+  // Small tensors: CTAs of about 512 threads (larger ones would keep the
+  // GEMM launched as this grid's programmatic dependent off their SMs); a
+  // single CTA needs no barrier at all, and 2-16 CTAs run as one thread-block
+  // cluster whose hardware barrier replaces the global-memory grid barrier.
+  {
+    const int rpc = 512 / tpr > 0 ? 512 / tpr : 1;
+    const int ctas = rpc > 0 ? (T + rpc - 1) / rpc : 0;
+    if (ctas >= 1 && ctas <= kMaxClusterCtas) {
+      const int threads = (ctas == 1 ? T : rpc) * tpr;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(ctas);
+      cfg.blockDim = dim3(threads);
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[1];
+      if (ctas > 1) {
+        static bool nonportable[64] = {};
+        int dev = 0;
+        if (ctas > 8 && cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !nonportable[dev]) {
+          cudaFuncSetAttribute(prep_fused_kernel<NC, kKind>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+          cudaGetLastError();
+          nonportable[dev] = true;
+        }
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)ctas;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+      }
+      cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKind>, Xb, Gb, eps, row_index, T, Tp, K,
+                                         ctas == 1 ? T : rpc, inv_rms, sync, s_g, p, rs, ctas > 1 ? 1 : 0);
+      if (e == cudaSuccess) {
+        *launched = true;
+        return cudaSuccess;
+      }
+      cudaGetLastError();  // e.g. no GPC can host the cluster: the grid-barrier form below
+    }
+  }
   int rpc = 512 / tpr;
   rpc = rpc < 1 ? 1 : rpc;
   const int threads = rpc * tpr;
@@ -566,7 +630,7 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   cfg.blockDim = dim3(threads);
   cfg.stream = stream;
   cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKind>, Xb, Gb, eps, row_index, T, Tp, K, rpc,
-                                     inv_rms, sync, s_g, p, rs);
+                                     inv_rms, sync, s_g, p, rs, 0);
   if (e == cudaSuccess) *launched = true;
   else cudaGetLastError();  // fall back to the two-launch form
   return cudaSuccess;
@@ -586,7 +650,7 @@ cudaError_t launch_per_token_nc(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb
   cfg.blockDim = dim3(rpc * tpr);
   cfg.stream = stream;
   return cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKindSharq, true>, Xb, Gb, eps, row_index, T, Tp, K, rpc, inv_rms,
-                            sync, s_t, p, rs);
+                            sync, s_t, p, rs, 0);
 }
 
 template <int kKind>
