@@ -118,3 +118,20 @@ def test_linear_after_silu_prep():
     torch.cuda.synchronize()
     assert ws.check() == 0
     assert H.rel_fro(y.cpu().numpy(), ref) < 1e-5
+
+
+def test_silu_prep_with_rmsnorm_and_empty_batch():
+    """gamma applies to h like any prep input (bit-exact); T = 0 touches nothing."""
+    T, K = 24, 2048
+    g, u = _inputs(T, K, 3400)
+    gamma = synthetic.gamma(3401, K)
+    act = _act(T, K, sq.SHARQ_MODE_SHARQ)
+    act.prep_silu_mul(H.bf16_dev(g), H.bf16_dev(u), None, H.bf16_dev(gamma), 1e-5)
+    ref = _act(T, K, sq.SHARQ_MODE_SHARQ)
+    ref.prep(H.bf16_dev(O.silu_mul(g, u)), H.bf16_dev(gamma), 1e-5)
+    torch.cuda.synchronize()
+    assert torch.equal(act.buf, ref.buf)
+    empty = sq.PreparedAct(0, K, sq.SHARQ_MODE_SHARQ)
+    empty.prep_silu_mul(None, None, None, None, 1e-5)
+    empty.prep_residual(None, None, None, None, 1e-5)
+    torch.cuda.synchronize()
