@@ -224,8 +224,12 @@ __device__ __forceinline__ int tile_expert(const GemmArgs& args, int mt) {
 // has completed and its memory is visible (returns at once if there is none).
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+// 16-byte store into a peer CTA's shared memory that counts its bytes on the
+// peer's mbarrier (transaction bytes) when it lands: no release fence and no
+// separate arrival are needed for the peer to see it.
+__device__ __forceinline__ void st_async_f4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
                : "memory");
 }
 
@@ -536,9 +540,12 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
       mbar_init(&stat_bar[0], (uint32_t)(S * max(valid, 1)));
       mbar_init(&stat_bar[1], (uint32_t)S);
     }
-    // one arrival per received row: S senders x my_n rows
-    mbar_init(&recv_bar, kSplit && my_n > 0 ? (uint32_t)(S * my_n) : 1u);
+    mbar_init(&recv_bar, 1u);
     fence_mbar_init();
+    // the receive barrier completes when all S senders' rows have landed
+    // (transaction bytes of their st.async stores); set before the cluster
+    // sync below, so before any peer can store
+    if (kSplit && my_n > 0) mbar_arrive_expect_tx(&recv_bar, (uint32_t)(S * my_n * BN * 4));
     abort_sh = 0;
     expert_sh = tile_expert(args, mt);
   }
@@ -763,6 +770,7 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
                                        (uint32_t)((split * (BN / 4) * rp + (rl - owner * rows_per)) * 16),
                                    (uint32_t)owner)
                      : 0u;
+      const uint32_t rbar = rl < valid ? mapa_shared(smem_u32(&recv_bar), (uint32_t)owner) : 0u;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         uint32_t v[32];
@@ -771,12 +779,10 @@ __global__ void __launch_bounds__(Cfg<BN, kSplit, kFused>::kThreadsT, 1) sharq_g
         if (rl < valid) {
 #pragma unroll
           for (int q = 0; q < 32; q += 4)
-            st_cluster_f4(dst + (uint32_t)((c + q) / 4 * rp) * 16u, __uint_as_float(v[q]), __uint_as_float(v[q + 1]),
-                          __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
+            st_async_f4(dst + (uint32_t)((c + q) / 4 * rp) * 16u, __uint_as_float(v[q]), __uint_as_float(v[q + 1]),
+                        __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]), rbar);
         }
       }
-      // release: this thread's stores before its arrival at the owner
-      if (rl < valid) mbar_arrive_remote(mapa_shared(smem_u32(&recv_bar), (uint32_t)owner));
     }
   }
 
