@@ -64,7 +64,7 @@ def prep_alg_bytes(T, K):
 # (profiles/sharq_gemm_qproj_decode.md, profiles/sharq_gemm_persistent_mlp2048.md);
 # None where none was taken.  Reset an entry whenever its kernel changes,
 # until it is captured again.
-NCU_TRAFFIC = {"q_proj_T128": 10475008, "gate_T2048": 64077824, "up_T2048": 59511552}
+NCU_TRAFFIC = {"q_proj_T128": 10474752, "gate_T2048": 64077824, "up_T2048": 59511552}
 
 
 def read_peaks():
