@@ -36,9 +36,10 @@
 // (1 x 1 x S); each takes a contiguous range of K stages.  CTA r of the
 // cluster owns 1/S of the tile's valid rows: every CTA pushes that slice of
 // its fp32 partial, row by row from registers, into a receive buffer in the
-// owner's shared memory over distributed shared memory, and the owner sums
-// the S slices in rank order -- deterministic, no global scratch, no
-// atomics, one bounded wait.
+// owner's shared memory over distributed shared memory (st.async stores that
+// complete the owner's barrier by transaction bytes), and the owner sums the
+// S slices in rank order -- deterministic, no global scratch, no atomics,
+// one bounded wait.
 // Rows beyond the activation's valid rows are not copied into shared memory
 // (decode: T = 1 moves 1 row of codes, not 128) -- sharq_prep does not even
 // write them; their accumulator rows hold garbage that is never stored (MMA
