@@ -99,3 +99,16 @@ def test_product_matches_torch_bf16():
 def test_times_one_is_silu():
     g = synthetic.activations(33, 8, 256)
     assert np.array_equal(sharq.silu_mul(g, np.ones_like(g)), sharq.silu_bf16(g))
+
+
+def test_bf16_round_f64_matches_torch_conversion():
+    """One rounding from float64 to bf16 (not through float32): checked
+    against torch's float64 -> bfloat16 conversion on values spread over the
+    normal and subnormal range, including exact halfway cases."""
+    g = np.random.default_rng(9)
+    x = g.standard_normal(20000) * np.exp2(g.integers(-140, 120, 20000).astype(np.float64))
+    halfway = (np.arange(1, 200, dtype=np.float64) * 2 + 1) * 2.0 ** -9  # odd multiples of half a bf16 ulp at 1
+    x = np.concatenate([x, halfway, -halfway, [0.0, -0.0, 2.0 ** -134, 3 * 2.0 ** -134]])
+    want = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    got = sharq.bf16_round_f64(x)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
