@@ -91,6 +91,17 @@ def test_prep_bit_exact(name, T, K, kw, gam, eps):
     _check_sharq(x, gamma, eps)
 
 
+@pytest.mark.parametrize("T", [2, 9, 17])
+def test_prep_grid_forms_bit_exact(T):
+    """K = 4096 (one row per 512-thread CTA): T = 2 and 9 run as one
+    thread-block cluster (9 is above the portable cluster size), T = 17 as a
+    grid with the global-memory barrier."""
+    K = 4096
+    x = synthetic.activations(150 + T, T, K)
+    x[T - 1] *= 32.0  # the tensor max in the last CTA
+    _check_sharq(x, synthetic.gamma(151, K), 1e-5)
+
+
 @pytest.mark.parametrize("T,K", [(64, 14336), (32, 18944), (33, 3584)])
 def test_prep_long_rows_bit_exact(T, K):
     """Rows longer than 8192 give each thread 2 or 4 runs of 8 in the
