@@ -1,16 +1,21 @@
 """Benchmark of the SharQ hot path (sharq_prep + sharq_linear) on B200.
 
-Workload: the Llama-3.1-8B q_proj linear (K = D = 4096) at decode / small
-batch, T in {1, 16, 128}.  One step = one prep + one dual-path GEMM for each
-T (three layers).  Metric: effective TFLOP/s = sum(2 T K D) / time, whole job
-(all ranks); µs per layer per T is reported beside it.
+Default workload: the linear stack of one Qwen2.5-7B decoder layer -- qkv
+3584 -> 4608 and gate+up 3584 -> 37888 (both with the RMSNorm fused into
+sharq_prep), o 3584 -> 3584 and down 18944 -> 3584 (no norm; Student-t input)
+-- at T = 1, 64, 1024 and 8192 tokens, i.e. from decode to prefill, the
+largest single-GPU configuration.  One step = prep + dual-path GEMM of all 16
+layers (4 linears x 4 token counts).  Metric: effective TFLOP/s =
+sum(2 T K D) / time, whole job (all ranks); µs per layer, per kernel and per
+T are reported beside it.  Other workloads: --workload q_proj (Llama-3.1-8B
+q_proj decode, T in {1, 16, 128}) and --workload mlp (Llama-3.1-8B MLP
+prefill).
 
 Timing: CUDA events on the launching stream around exactly K steps, barrier
-+ synchronize on both sides, max over ranks.  L2 (126 MB) is defeated by
-rotating through 16 packed weight copies (160 MB) and 16 activation copies,
-so every step reads cold weights from HBM.  Each step is replayed from a CUDA
-graph (one per rotation slot) so launch latency does not dominate µs-sized
-kernels.
++ synchronize on both sides, max over ranks.  The step's working set (packed
+weights alone: 550 MB) is larger than the 126 MB L2, so every step reads its
+weights from HBM; smaller workloads rotate through up to 16 weight and
+activation copies to the same end.  Each step is replayed from a CUDA graph.
 
 --impl reference times the CPU oracle (the only reference this method has:
 the pages ship no code) on a bounded sample of the same workload.
@@ -28,21 +33,15 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-K_DIM, D_DIM = 4096, 4096
-T_LIST = (1, 16, 128)
-N_ROT = 16
 EPS = 1e-5
-WORKLOAD = "llama3.1-8b q_proj K=4096 D=4096, T in {1,16,128}, RMSNorm gamma~U(0.5,1.5)"
 WORKLOADS = {"q_proj": "llama3.1-8b q_proj K=4096 D=4096 (prep+linear per T), RMSNorm gamma~U(0.5,1.5)",
              "mlp": "llama3.1-8b MLP prefill: gate/up 4096->14336 (shared prep, RMSNorm), down 14336->4096 "
                     "(Student-t input)",
              "qwen_layer": "qwen2.5-7b decoder-layer linears: qkv 3584->4608 (RMSNorm), o 3584->3584, "
                            "gate+up 3584->37888 (RMSNorm), down 18944->3584 (Student-t input)"}
+DEFAULT_T = {"q_proj": [1, 16, 128], "mlp": [2048], "qwen_layer": [1, 64, 1024, 8192]}
 METRIC = "prep+dual-GEMM effective TFLOP/s (2TKD)"
-
-
-def flops_per_step():
-    return sum(2.0 * t * K_DIM * D_DIM for t in T_LIST)
+NOMINAL_FP4_DENSE_PFLOPS = 9.0   # B200 datasheet, dense; sparse 2x
 
 
 def gemm_alg_bytes(T, K, D):
@@ -59,12 +58,20 @@ def prep_alg_bytes(T, K):
     return T * K * 2 + Tp * K * 0.90625
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
-# the dominant GEMM, from ncu captures of this script's workloads
-# (profiles/sharq_gemm_qproj_decode.md, profiles/sharq_gemm_persistent_mlp2048.md);
+def gemm_split_k(L):
+    """Whether sharq_linear runs this layer as the split-K decode kernel (its
+    output tiles cannot fill the GPU) rather than the persistent one; mirrors
+    the library's launch rule, for naming the kernel in the report."""
+    m = -(-L.T // 128)
+    n = L.D // 256 if L.D % 256 == 0 else L.D // 128
+    return m * n < 74
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch,
+# from one ncu capture of this script's command, keyed by layer and kernel;
 # None where none was taken.  Reset an entry whenever its kernel changes,
 # until it is captured again.
-NCU_TRAFFIC = {"q_proj_T128": 10474752, "gate_T2048": 64077824, "up_T2048": 59511552}
+NCU_TRAFFIC = {}
 
 
 def read_peaks():
@@ -152,69 +159,89 @@ def init_dist(args):
 
 # ------------------------------------------------------------- CPU oracle ---
 
-def oracle_sample(seconds=10.0):
-    """Time the CPU oracle (prep + float64 dual GEMM) on the same workload:
-    whole layers (weights packed once, outside the timed loop), cycling
-    through T in {1, 16, 128} until about `seconds` of CPU work."""
+ORACLE_T = 64        # token rows of the oracle sample
+ORACLE_COLS = 1024   # output columns of each weight in the oracle sample
+
+
+def oracle_layers(workload):
+    """The oracle's bounded sample of a workload: each distinct linear of it
+    at T = 64 rows (the decode-batch point of the sweep), whole rows of K,
+    against the first 1024 output columns of its weight (packed once, outside
+    any timed region: weight packing is not part of a layer's work)."""
     import synthetic
     from oracle import sharq as O
-    w = synthetic.weights(11, K_DIM, D_DIM)
-    q = O.pack_weight(w)
-    gamma = synthetic.gamma(12, K_DIM)
-    xs = {t: synthetic.activations(13 + t, t, K_DIM) for t in T_LIST}
-    flops, layers = 0.0, 0
+    seen, out = set(), []
+    for L in workload_layers(workload, [ORACLE_T]):
+        if L.shares:
+            continue
+        key = (L.K, L.D, L.norm, L.base)
+        if key in seen:
+            continue
+        seen.add(key)
+        d = min(ORACLE_COLS, L.D)
+        w = synthetic.weights(11 + L.K + L.D, L.K, d)
+        out.append({"name": L.name, "K": L.K, "D": d, "q": O.pack_weight(w),
+                    "gamma": synthetic.gamma(12, L.K) if L.norm else None,
+                    "x": synthetic.activations(13 + L.K, ORACLE_T, L.K, base=L.base)})
+    return out
+
+
+def oracle_step(layers, k):
+    """One layer of the sample through the oracle (prep + float64 dual GEMM);
+    returns its 2TKD FLOPs."""
+    from oracle import sharq as O
+    L = layers[k % len(layers)]
+    O.linear(O.prep(L["x"], L["gamma"], EPS), L["q"])
+    return 2.0 * ORACLE_T * L["K"] * L["D"]
+
+
+def oracle_sample(workload, seconds=10.0):
+    """cpu_baseline: the oracle on the workload's bounded sample, layers in
+    turn, until about `seconds` of CPU work."""
+    layers = oracle_layers(workload)
+    flops, done = 0.0, 0
     t0 = time.perf_counter()
     while True:
-        for t in T_LIST:
-            p = O.prep(xs[t], gamma, EPS)
-            O.linear(p, q)
-            flops += 2.0 * t * K_DIM * D_DIM
-            layers += 1
+        flops += oracle_step(layers, done)
+        done += 1
         el = time.perf_counter() - t0
-        if el >= seconds:
+        if el >= seconds and done >= len(layers):
             break
     threads = os.environ.get("OMP_NUM_THREADS") or str(len(os.sched_getaffinity(0)))
+    names = ", ".join(f"{L['name']} K={L['K']}" for L in layers)
     return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
-            "sample": f"{layers} whole layers (T cycling 1,16,128; K=D=4096), {el:.1f} s, "
-                      f"numpy float32-emulated prep + float64 BLAS GEMM"}, el / layers
+            "sample": f"{done} layers ({names}; T={ORACLE_T} rows, first {ORACLE_COLS} output columns of each "
+                      f"weight, packed beforehand), {el:.1f} s, numpy float32-emulated prep + float64 BLAS GEMM"}
 
 
 def run_reference(args, world, rank, budget_s=120.0):
-    """Time the oracle as it stands.  One step = one whole layer, T cycling
-    through 1, 16, 128.  Steps stop early once `budget_s` seconds of timed
-    CPU work have passed so the run stays within a few minutes; the value is
-    the work done over the time taken."""
+    """Time the oracle as it stands.  One step = one layer of the workload's
+    bounded sample (oracle_layers), layers in turn.  Steps stop early once
+    `budget_s` seconds of timed CPU work have passed so the run stays within a
+    few minutes; the value is the work done over the time taken."""
     if rank != 0:
         return
-    import synthetic
-    from oracle import sharq as O
-    w = synthetic.weights(11, K_DIM, D_DIM)
-    q = O.pack_weight(w)
-    gamma = synthetic.gamma(12, K_DIM)
-    xs = {t: synthetic.activations(13 + t, t, K_DIM) for t in T_LIST}
-
-    def step(k):
-        t = T_LIST[k % len(T_LIST)]
-        O.linear(O.prep(xs[t], gamma, EPS), q)
-        return 2.0 * t * K_DIM * D_DIM
+    layers = oracle_layers(args.workload)
     for k in range(args.warmup):
-        step(k)
+        oracle_step(layers, k)
     flops, done = 0.0, 0
     t0 = time.perf_counter()
     for k in range(args.steps):
-        flops += step(k)
+        flops += oracle_step(layers, k)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     el = time.perf_counter() - t0
     v = flops / el / 1e12
     cores = len(os.sched_getaffinity(0))
+    sample = f"{done} layers of {', '.join(L['name'] for L in layers)} (T={ORACLE_T}, first {ORACLE_COLS} columns)"
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "steps_timed": done, "warmup": args.warmup, "ms_per_step": el / done * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "replicas"},
+            "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.workload] + f", T in {tuple(args.T)}", "parallelism": "replicas"},
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{done} whole layers (T cycling 1,16,128; K=D=4096), {el:.1f} s"},
+                             "sample": f"{sample}, {el:.1f} s"},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -235,7 +262,7 @@ class Layer:
 
 def workload_layers(name, t_list):
     if name == "q_proj":
-        return [Layer(f"q_proj_T{t}", t, K_DIM, D_DIM, True) for t in t_list]
+        return [Layer(f"q_proj_T{t}", t, 4096, 4096, True) for t in t_list]
     if name == "qwen_layer":   # Qwen2.5-7B decoder-layer linears
         out = []
         for t in t_list:
@@ -276,6 +303,29 @@ def kernel_us(fn, n_rot, stream, launches=96):
     b.record(stream)
     torch.cuda.synchronize()
     return a.elapsed_time(b) * 1e3 / (5 * reps * n_rot)
+
+
+def graph_kernel_launches(g):
+    """Number of kernel nodes in a captured graph (torch.cuda.CUDAGraph made
+    with keep_graph=True): the kernels one replay launches.  None if the
+    graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        count = 0
+        for node in nodes[:n]:
+            err, t = rt.cudaGraphNodeGetType(node)
+            if err == rt.cudaError_t.cudaSuccess and t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                count += 1
+        return count
+    except Exception:
+        return None
 
 
 def run_gpu(args, world, rank, local):
@@ -346,17 +396,20 @@ def run_gpu(args, world, rank, local):
         for L in layers:
             layer(L, i)
 
-    launches_per_step = sum(1 if (L.shares or fused(L)) else 2 for L in layers)
     for i in range(n_rot):
         step(i)
     torch.cuda.synchronize()
     graphs = []
     for i in range(n_rot):
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(g, stream=stream):
             step(i)
+        g.instantiate()
         graphs.append(g)
     torch.cuda.synchronize()
+    # kernels per step, counted in the captured graph (every one of them is
+    # this library's: the step issues nothing else)
+    launches_per_step = graph_kernel_launches(graphs[0])
 
     for k in range(args.warmup):
         graphs[k % n_rot].replay()
@@ -415,7 +468,7 @@ def run_gpu(args, world, rank, local):
     for i in range(3):
         e2e_step(i % n_rot)
     torch.cuda.synchronize()
-    e2e_steps = max(3, min(args.steps, 200))
+    e2e_steps = max(3, min(args.steps, 50))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for k in range(e2e_steps):
@@ -498,22 +551,37 @@ def run_gpu(args, world, rank, local):
             del Wb, act_n
 
     flops_step = sum(L.flops for L in layers)
-    # dominant kernel: the GEMM with the largest share of the step
+    peak_gbs, peak_kind = read_peaks()
+    from sparse_activation_quantization_b200 import peak
+    pk = peak.fp4_peaks()
+    eff_tflops = pk["effective_pflops"] * 1e3
+    nominal_eff = 1e3 / (1.0 / NOMINAL_FP4_DENSE_PFLOPS + 1.0 / (2 * NOMINAL_FP4_DENSE_PFLOPS))
+    # dominant kernel: the GEMM with the largest share of the step, against
+    # the roofline that bounds it (the slower of its tensor time at the
+    # combined FP4 peak and its HBM time at the copy bandwidth)
     dom = max(layers, key=lambda L: per[L.name]["gemm_us"])
-    if args.workload == "mlp":
-        from sparse_activation_quantization_b200 import peak
-        pk = peak.fp4_peaks()
-        roof = {"kernel": f"sharq_gemm_persistent_kernel ({dom.name})", "bound": "tensor",
-                "achieved": per[dom.name]["gemm_tflops"], "peak": pk["effective_pflops"] * 1e3,
-                "unit": "TFLOP/s", "frac": per[dom.name]["gemm_tflops"] / (pk["effective_pflops"] * 1e3),
-                "peak_kind": "measured tcgen05 FP4 (dense %.2f, sparse %.2f PFLOP/s; dual-GEMM effective)"
-                             % (pk["dense_pflops"], pk["sparse_pflops"]), "traffic": NCU_TRAFFIC.get(dom.name)}
+    t_tensor = dom.flops / (eff_tflops * 1e12)
+    t_hbm = gemm_alg_bytes(dom.T, dom.K, dom.D) / (peak_gbs * 1e9)
+    gemm_kernel = ("sharq_gemm_kernel (split-K)" if gemm_split_k(dom) else "sharq_gemm_persistent_kernel")
+    if t_tensor >= t_hbm:
+        ach = per[dom.name]["gemm_tflops"]
+        roof = {"kernel": f"{gemm_kernel} ({dom.name})", "bound": "tensor", "achieved": ach, "peak": eff_tflops,
+                "unit": "TFLOP/s", "frac": ach / eff_tflops,
+                "peak_kind": "measured tcgen05 FP4 dual-GEMM effective (dense %.2f, sparse %.2f PFLOP/s, best of "
+                             "1-CTA and 2-CTA forms)" % (pk["dense_pflops"], pk["sparse_pflops"]),
+                "frac_of_nominal": ach / nominal_eff,
+                "traffic": NCU_TRAFFIC.get(f"{dom.name}/gemm")}
     else:
-        peak_gbs, peak_kind = read_peaks()
         ach = per[dom.name]["gemm_gbs"]
-        roof = {"kernel": f"sharq_gemm_kernel ({dom.name})", "bound": "hbm", "achieved": ach, "peak": peak_gbs,
+        roof = {"kernel": f"{gemm_kernel} ({dom.name})", "bound": "hbm", "achieved": ach, "peak": peak_gbs,
                 "unit": "GB/s", "frac": ach / peak_gbs, "peak_kind": peak_kind + " burst copy",
-                "traffic": NCU_TRAFFIC.get(dom.name)}
+                "traffic": NCU_TRAFFIC.get(f"{dom.name}/gemm")}
+    # the prep with the largest share, against HBM
+    pdom = max((L for L in layers if per[L.name]["prep_us"] is not None), key=lambda L: per[L.name]["prep_us"])
+    pach = per[pdom.name]["prep_gbs"]
+    roof_prep = {"kernel": f"sharq_prep ({pdom.name})", "bound": "hbm", "achieved": pach, "peak": peak_gbs,
+                 "unit": "GB/s", "frac": pach / peak_gbs, "peak_kind": peak_kind + " burst copy",
+                 "traffic": NCU_TRAFFIC.get(f"{pdom.name}/prep")}
     line = None
     if rank == 0:
         ms_step = ms / args.steps
@@ -532,10 +600,12 @@ def run_gpu(args, world, rank, local):
             "layers": {n: {k: (round(v, 3) if isinstance(v, float) else v) for k, v in d.items()}
                        for n, d in per.items()},
             "roofline": roof,
+            "roofline_prep": roof_prep,
             "comparators": comparators,
             "e2e": {"value": job_tflops(flops_step, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
+            "gpu_launches_per_step": launches_per_step,
             "clocks": clk,
         }
     if world > 1:
@@ -552,7 +622,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="sharq", choices=["sharq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--workload", default="q_proj", choices=["q_proj", "mlp", "qwen_layer"])
+    ap.add_argument("--workload", default="qwen_layer", choices=["q_proj", "mlp", "qwen_layer"])
     ap.add_argument("--compare", action="store_true",
                     help="also time plain NVFP4 and bf16 cuBLAS on the same layers")
     ap.add_argument("--T", type=int, nargs="+", default=None)
@@ -561,14 +631,14 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.T is None:
-        args.T = {"q_proj": list(T_LIST), "mlp": [2048], "qwen_layer": [1, 64, 1024, 8192]}[args.workload]
+        args.T = DEFAULT_T[args.workload]
     world, rank, local = init_dist(args)
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
     cpu = None
-    if rank == 0 and world == 1 and args.workload == "q_proj":
-        cpu, _ = oracle_sample(args.cpu_seconds)   # before any CUDA work
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        cpu = oracle_sample(args.workload, args.cpu_seconds)   # before any CUDA work
     line = run_gpu(args, world, rank, local)
     if rank == 0 and line is not None:
         line["cpu_baseline"] = cpu

@@ -159,14 +159,20 @@ typedef struct {
  *   inv_rms: Tp floats (1/rms per row; 1 when RMSNorm is off).
  *   s_g:     the per-tensor global scale gmax / (6*448) (1 if gmax == 0);
  *            SHARQ_TOKEN: Tp floats, s_t of row t (rows >= T unused).
- *   gmax_bits: 16 bytes of scratch: device-wide amax, grid-barrier count,
- *            departure count, and an error word that sharq_linear forwards
- *            to its workspace (a prep whose grid barrier timed out).
+ *   gmax_bits: 24 bytes of scratch, six 32-bit words: device-wide amax,
+ *            grid-barrier count, departure count, the error word of the last
+ *            sharq_prep (SHARQ_ERR_TIMEOUT when its grid barrier timed out;
+ *            sharq_linear forwards it to its workspace), the error of the
+ *            prep in flight, and a fault-injection word that must stay zero
+ *            (a test writes k + 1 there to make CTA k of the grid-barrier form
+ *            skip its arrival, so that the bounded wait runs out).
  *   The 256-byte scalar block that holds gmax_bits (and s_g outside
  *   SHARQ_TOKEN)
  *   must be zero before the first sharq_prep on a buffer (zero the whole
- *   buffer once after allocation); sharq_prep leaves gmax_bits[0..2] zero
- *   again, so no per-call memset is needed.
+ *   buffer once after allocation); sharq_prep leaves gmax_bits[0..2] and
+ *   gmax_bits[4] zero again, so no per-call memset is needed.
+ *   sharq_linear reads only the operands, s_g and (when it is not NULL)
+ *   gmax_bits[3]; it does not need inv_rms.
  */
 typedef struct {
   void *sp_codes;
@@ -288,9 +294,10 @@ int sharq_prep_silu_mul(const void *d_gate, const void *d_up, void *d_h, const v
  *    error word, per-row 1/rms) lives in a fixed array inside the library
  *    (256 bytes + 4 bytes per row, up to 16384 rows, about 64 KB, held by
  *    every GPU that loads the library until the process exits).  a->inv_rms
- *    is not written and a->gmax_bits[0..2] are not used; a->gmax_bits may be
- *    NULL.  If it is not, the error word is copied to a->gmax_bits[3], where
- *    sharq_linear looks for it.
+ *    is not written (it may be NULL) and a->gmax_bits[0..2] are not used;
+ *    a->gmax_bits may be NULL.  If it is not, the error word is copied to
+ *    a->gmax_bits[3], where sharq_linear looks for it; if it is, sharq_linear
+ *    on that view has no prep error word to forward.
  *  - a->T > 16384 returns SHARQ_ERR_UNSUPPORTED_SHAPE.
  *  - The first call on each device looks the array's address up
  *    (cudaGetSymbolAddress); make that first call before any stream capture.

@@ -5,6 +5,7 @@ Run ``python -m sparse_activation_quantization_b200.build`` (or call
 it travels with the source tree.  No fast-math flags: the quantizer's float32
 steps must round exactly as IEEE single precision.
 """
+import hashlib
 import os
 import shutil
 import subprocess
@@ -25,41 +26,65 @@ def nvcc():
     raise RuntimeError("nvcc not found")
 
 
-def _stale(objs):
-    if not os.path.exists(LIB):
+STAMP = LIB + ".sha256"
+PEAK_SRC = os.path.join(HERE, "peak", "fp4_peak.cu")
+PEAK_LIB = os.path.join(HERE, "peak", "libsharq_peak.so")
+
+
+def source_hash(extra=()):
+    """sha256 over every input of the build: the CUDA sources and headers,
+    the public header, the peak microbenchmark, this file and the compiler
+    flags.  A library whose recorded hash differs is rebuilt, whatever the
+    files' times say (a prebuilt library copied in beside newer sources is
+    never reused)."""
+    h = hashlib.sha256()
+    deps = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h")))
+    deps += [PEAK_SRC, os.path.join(HERE, "..", "include", "sharq.h"), os.path.abspath(__file__)]
+    for d in deps:
+        h.update(os.path.basename(d).encode())
+        with open(d, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join([*ARCH, *FLAGS, *extra]).encode())
+    return h.hexdigest()
+
+
+def _stale(digest):
+    if not (os.path.exists(LIB) and os.path.exists(PEAK_LIB) and os.path.exists(STAMP)):
         return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
-    deps.append(os.path.join(HERE, "peak", "fp4_peak.cu"))
-    deps.append(os.path.join(HERE, "..", "include", "sharq.h"))
-    deps.append(os.path.abspath(__file__))
-    return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
+    with open(STAMP) as f:
+        return f.read().strip() != digest
 
 
 def build(force=False, verbose=False, extra=()):
-    """Compile every source for sm_100a and link libsharq.so; returns its path."""
-    if not force and not _stale(None):
+    """Compile every source for sm_100a and link libsharq.so; returns its path.
+    Skipped when the library was built from exactly these sources and flags."""
+    digest = source_hash(extra)
+    if not force and not _stale(digest):
         return LIB
     out_dir = os.path.join(HERE, "_build")
     os.makedirs(out_dir, exist_ok=True)
-    objs = []
-    for src in SOURCES:
+    objs, procs = [], []
+    for src in SOURCES:  # the translation units compile side by side
         obj = os.path.join(out_dir, src.replace(".cu", ".o"))
         cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
+        procs.append((cmd, subprocess.Popen(cmd)))
         objs.append(obj)
+    failed = [cmd for cmd, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
     tmp = LIB + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     # the FP4 peak microbenchmark (roofline denominators), a separate library
-    peak_src = os.path.join(HERE, "peak", "fp4_peak.cu")
-    peak_lib = os.path.join(HERE, "peak", "libsharq_peak.so")
-    subprocess.run([nvcc(), *ARCH, *FLAGS, "-shared", "-cudart", "static", peak_src, "-o", peak_lib + ".tmp"],
+    subprocess.run([nvcc(), *ARCH, *FLAGS, "-shared", "-cudart", "static", PEAK_SRC, "-o", PEAK_LIB + ".tmp"],
                    check=True)
-    os.replace(peak_lib + ".tmp", peak_lib)
+    os.replace(PEAK_LIB + ".tmp", PEAK_LIB)
+    with open(STAMP + ".tmp", "w") as f:
+        f.write(digest + "\n")
+    os.replace(STAMP + ".tmp", STAMP)
     return LIB
 
 

@@ -176,12 +176,15 @@ int check_device() {
   return ok ? SHARQ_OK : SHARQ_ERR_ARCH;
 }
 
-int act_ok(const sharq_act* a) {
+// for_prep: sharq_prep writes inv_rms and uses gmax_bits; sharq_linear reads
+// neither (a NULL gmax_bits only means no prep error word to forward)
+int act_ok(const sharq_act* a, bool for_prep = true) {
   if (!a) return SHARQ_ERR_INVALID_ARG;
   if (!shape_ok_t(a->T) || !shape_ok_k(a->K)) return SHARQ_ERR_UNSUPPORTED_SHAPE;
   if (!mode_ok(a->mode)) return SHARQ_ERR_INVALID_ARG;
   if (a->Tp != (int)round_up((size_t)a->T, 128)) return SHARQ_ERR_INVALID_ARG;
-  if (!a->r_codes || !a->r_sf || !a->inv_rms || !a->s_g || !a->gmax_bits) return SHARQ_ERR_INVALID_ARG;
+  if (!a->r_codes || !a->r_sf || !a->s_g) return SHARQ_ERR_INVALID_ARG;
+  if (for_prep && (!a->inv_rms || !a->gmax_bits)) return SHARQ_ERR_INVALID_ARG;
   if (has_first(a->mode) && (!a->sp_codes || !a->sp_sf)) return SHARQ_ERR_INVALID_ARG;
   if (first_sparse(a->mode) && !a->meta) return SHARQ_ERR_INVALID_ARG;
   if (second_sparse(a->mode) && !a->r_meta) return SHARQ_ERR_INVALID_ARG;
@@ -202,7 +205,7 @@ int weight_ok(const sharq_weight* w) {
 
 int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* w, void* d_Y, int out_dtype,
                   void* d_ws, size_t ws_bytes, sharq_stream_t stream, bool grouped) {
-  int st = act_ok(a);
+  int st = act_ok(a, false);
   if (st) return st;
   if ((st = weight_ok(w))) return st;
   if (a->K != w->K) return SHARQ_ERR_UNSUPPORTED_SHAPE;
@@ -223,7 +226,8 @@ int linear_common(const sharq_act* a, const int* d_offsets, const sharq_weight* 
       static_cast<const uint8_t*>(w->codes), static_cast<const uint8_t*>(w->sf32),
       static_cast<const uint8_t*>(w->sf16), w->s_w, w->D, w->E, grouped ? d_offsets : nullptr, d_Y,
       out_dtype == SHARQ_OUT_F32 ? 1 : 0, g.bn, g.splits, static_cast<int*>(d_ws),
-      reinterpret_cast<const int*>(a->gmax_bits + 3), reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr,
+      a->gmax_bits ? reinterpret_cast<const int*>(a->gmax_bits + 3) : nullptr, reinterpret_cast<cudaStream_t>(stream),
+      nullptr, nullptr,
       0.0f, a->mode == SHARQ_MODE_SHARQ_TOKEN);
   return e == cudaSuccess ? SHARQ_OK : SHARQ_ERR_CUDA;
 }

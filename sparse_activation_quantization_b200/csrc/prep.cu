@@ -241,15 +241,27 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
 // grid's completion (griddepcontrol.wait) before reading our outputs.
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Last CTA out resets the device-wide max and the counters (sync words
-// 0..2 of the act scalar block), so the next sharq_prep on this buffer
-// starts from zero without a memset.  Called by thread 0 of every CTA at its
-// end, after the CTA has read the max (so the reset cannot race a reader).
+// Words of the act scalar block (gmax_bits) that the prep kernels use:
+//   0  device-wide max |Xn| (float bits)    1  grid-barrier arrivals
+//   2  departures                           3  error word of the last call
+//                                              (read by sharq_linear)
+//   4  error of the call in flight          5  fault-injection word (tests)
+// Words 0..2 and 4 are zero at rest.  A CTA whose bounded barrier wait runs
+// out records into word 4; only the last CTA out moves word 4 into word 3,
+// so a CTA that starts late can neither erase nor miss this call's error.
+enum : int { kSyncMax = 0, kSyncArrive = 1, kSyncDepart = 2, kSyncErr = 3, kSyncPending = 4, kSyncInject = 5 };
+
+// Last CTA out publishes this call's error word and resets the device-wide
+// max and the counters, so the next sharq_prep on this buffer starts from
+// zero without a memset.  Called by thread 0 of every CTA at its end, after
+// the CTA has read the max (so the reset cannot race a reader) and after any
+// error it recorded (atomics, complete before the departure is counted).
 __device__ __forceinline__ void depart_and_reset(unsigned int* sync) {
-  if (atomicAdd(sync + 2, 1u) == gridDim.x - 1) {
-    sync[0] = 0u;
-    sync[1] = 0u;
-    sync[2] = 0u;
+  if (atomicAdd(sync + kSyncDepart, 1u) == gridDim.x - 1) {
+    sync[kSyncErr] = atomicExch(sync + kSyncPending, 0u);
+    sync[kSyncMax] = 0u;
+    sync[kSyncArrive] = 0u;
+    sync[kSyncDepart] = 0u;
     __threadfence();
   }
 }
@@ -403,7 +415,8 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
   // cluster form: announce this CTA (its shared memory exists) before any
   // peer stores into it; the matching wait comes just before those stores
   if (cluster) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  if (blockIdx.x == 0 && threadIdx.x == 0) sync[3] = 0u;  // error word of the previous prep
+  // forms without a grid barrier cannot time out: this call's error word is 0
+  if ((kPerToken || cluster || gridDim.x == 1) && blockIdx.x == 0 && threadIdx.x == 0) sync[kSyncErr] = 0u;
   // threads per row, padded to whole warps (a warp never spans two rows);
   // the padding lanes hold zeros and store nothing
   const int used = (K >> 3) / NC;
@@ -498,23 +511,28 @@ __global__ void __launch_bounds__(fused_max_threads<NC>()) prep_fused_kernel(
     if (gridDim.x == 1) {
       gmax_sh = m;  // one CTA holds the whole tensor: no grid barrier
     } else {
-      atomicMax(sync, __float_as_uint(m));
-      // arrival with release semantics: our max is visible before the count
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(sync + 1) : "memory");
+      // a test can name one CTA (index + 1) that never arrives, so that every
+      // CTA's bounded wait runs out; zero in normal use
+      const unsigned skip = *(volatile unsigned int*)(sync + kSyncInject);
+      if (skip != blockIdx.x + 1u) {
+        atomicMax(sync + kSyncMax, __float_as_uint(m));
+        // arrival with release semantics: our max is visible before the count
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(sync + kSyncArrive) : "memory");
+      }
       PREP_TRACE(1);
       // grid barrier: every CTA has published its max (bounded spin)
       const uint64_t deadline = globaltimer_ns() + kBarrierLimitNs;
       unsigned seen = 0;
       do {
-        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(sync + 1) : "memory");
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(sync + kSyncArrive) : "memory");
         if (seen >= gridDim.x) break;
         if (globaltimer_ns() > deadline) {
-          atomicCAS(reinterpret_cast<int*>(sync + 3), 0, -5);  // SHARQ_ERR_TIMEOUT
+          atomicCAS(reinterpret_cast<int*>(sync + kSyncPending), 0, -5);  // SHARQ_ERR_TIMEOUT
           break;
         }
       } while (true);
       asm volatile("fence.acq_rel.gpu;" ::: "memory");
-      gmax_sh = __uint_as_float(*(volatile unsigned int*)sync);
+      gmax_sh = __uint_as_float(*(volatile unsigned int*)(sync + kSyncMax));
     }
     PREP_TRACE(2);
   }
@@ -619,16 +637,22 @@ cudaError_t try_fused(const __nv_bfloat16* Xb, const __nv_bfloat16* Gb, float ep
   const int threads = rpc * tpr;
   const int ctas = (T + rpc - 1) / rpc;
   if (ctas > fused_max_ctas_t<NC, kKind>(threads)) return cudaSuccess;
-  // A plain launch: the grid fits the GPU at once (checked above), so all
-  // CTAs are resident together when the stream reaches this kernel; the
+  // A cooperative launch: the CTAs wait for one another at the grid barrier,
+  // so they must all be resident at once, which a cooperative launch
+  // guarantees (or refuses, and the two-launch form below runs instead).  The
   // GEMM that follows as a programmatic dependent can start only after every
-  // CTA of this grid has started (each triggers at entry), so it cannot
-  // crowd out a CTA that has not arrived at the grid barrier.  The barrier's
-  // spin is bounded all the same.
+  // CTA of this grid has started (each triggers at entry), so it cannot crowd
+  // out a CTA that has not arrived at the barrier.  The barrier's spin is
+  // bounded all the same.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(threads);
   cfg.stream = stream;
+  cudaLaunchAttribute coop[1];
+  coop[0].id = cudaLaunchAttributeCooperative;
+  coop[0].val.cooperative = 1;
+  cfg.attrs = coop;
+  cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, prep_fused_kernel<NC, kKind>, Xb, Gb, eps, row_index, T, Tp, K, rpc,
                                      inv_rms, sync, s_g, p, rs, 0);
   if (e == cudaSuccess) *launched = true;
@@ -848,7 +872,8 @@ cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, con
   unsigned int* sync = reinterpret_cast<unsigned int*>(scr);
   float* inv = reinterpret_cast<float*>(scr + kNoAllocSyncBytes);
   // the array keeps the last call's contents: start every call from zero
-  e = cudaMemsetAsync(sync, 0, 4 * sizeof(unsigned int), stream);
+  // (the max, the counters, both error words and the injection word)
+  e = cudaMemsetAsync(sync, 0, 8 * sizeof(unsigned int), stream);
   if (e != cudaSuccess) return e;
   e = launch_prep(X, gamma, eps, row_index, T, Tp, K, kind, per_token, inv, s_g, sync, sp_codes, meta, sp_sf,
                   r_codes, r_sf, r_meta, 0, nullptr, nullptr, stream);

@@ -1,11 +1,9 @@
-"""Measured FP4 tensor-core peaks of the current GPU (roofline denominators)
-and the issue cost of a GEMM stage's tensor-core work.
+"""Measured FP4 tensor-core peaks of the current GPU (roofline denominators).
 
-Runs the tcgen05 microbenchmarks in ``fp4_peak.cu`` (built next to it as
+Runs the tcgen05 microbenchmark in ``fp4_peak.cu`` (built next to it as
 ``libsharq_peak.so`` by the package build) on every SM: back-to-back dense
 ``kind::mxf4nvf4`` block16 MMAs, or 4:8-sparse ones, 128 x N from shared
-memory into TMEM; and one 256-K stage's MMAs and scale copies issued from one
-thread or from several warps.
+memory into TMEM.
 """
 import ctypes
 import os
@@ -33,28 +31,4 @@ def fp4_peaks(n256=True, iters=400):
     # (2TKD over the time of both) is the harmonic combination
     out["effective_pflops"] = 1.0 / (1.0 / out["dense_pflops"] + 1.0 / out["sparse_pflops"])
     out["n"] = 256 if n256 else 128
-    return out
-
-
-TC_ISSUE_MODES = {
-    0: "6 MMAs (2 sparse + 4 dense, N=128), one thread",
-    1: "13 tcgen05.cp (32x128b.warpx4), one thread",
-    2: "6 MMAs + 13 copies, the same thread",
-    3: "6 MMAs (warp 1) + 13 copies over warps 0, 2, 3",
-    4: "13 copies over warps 0-3",
-}
-
-
-def tc_issue_costs(iters=400):
-    """ns per 256-K stage for each issue layout of TC_ISSUE_MODES."""
-    L = ctypes.CDLL(LIB)
-    f = L.sharq_tc_issue_ns
-    f.restype = ctypes.c_int
-    f.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
-    out = {}
-    for mode, name in TC_ISSUE_MODES.items():
-        r = ctypes.c_double()
-        if f(mode, iters, ctypes.byref(r)) != 0:
-            raise RuntimeError("tcgen05 issue microbenchmark failed")
-        out[name] = round(r.value, 1)
     return out

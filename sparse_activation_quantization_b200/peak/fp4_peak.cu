@@ -13,7 +13,6 @@ using namespace sharq;
 namespace {
 
 constexpr int kSmem = 64 * 1024;
-constexpr int kIssueSmem = 120 * 1024;  // one CTA per SM (its first 64 KB are used)
 
 __global__ void __launch_bounds__(128, 1) fp4_peak_kernel(int sparse, int n256, int iters,
                                                           unsigned long long* ns) {
@@ -72,126 +71,7 @@ __global__ void __launch_bounds__(128, 1) fp4_peak_kernel(int sparse, int n256, 
   }
 }
 
-// Issue cost of a GEMM stage's tensor-core work (the copy-warp layout of the
-// SharQ GEMM follows from it): per iteration, the 6 MMAs of one 256-K stage
-// at N = 128 (2 sparse + 4 dense) and/or its 13 tcgen05.cp scale/metadata
-// copies (32x128b.warpx4, 512 B each), issued by
-//   mode 0: the MMAs alone (warp 1)
-//   mode 1: the copies alone, from one thread (warp 1)
-//   mode 2: MMAs and copies from the same thread (warp 1)
-//   mode 3: the MMAs from warp 1 and the copies spread over warps 0, 2, 3
-//   mode 4: the copies alone, spread over warps 0-3
-// Every issuing thread commits once at the end; the CTA's time is the
-// slowest thread's.  Copies go to columns no MMA reads (values do not matter).
-__global__ void __launch_bounds__(128, 1) tc_issue_kernel(int mode, int iters, unsigned long long* ns) {
-  extern __shared__ __align__(1024) uint8_t sm_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint32_t tbase;
-  __shared__ __align__(8) uint64_t setup_bar, bar[4];
-  __shared__ unsigned long long tend[4];
-  for (int i = threadIdx.x; i < (kSmem - 1024) / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(sm)[i] = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(sm + 56 * 1024)[i] = 0x44444444u;
-  if (threadIdx.x == 0) {
-    mbar_init(&setup_bar, 1);
-    for (int w = 0; w < 4; ++w) {
-      mbar_init(&bar[w], 1);
-      tend[w] = 0;
-    }
-    fence_mbar_init();
-  }
-  fence_proxy_async_smem();
-  if (threadIdx.x < 32) {
-    tmem_alloc(&tbase, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tm = tbase, s0 = smem_u32(sm);
-  const uint32_t B = s0, A = s0 + 32768, E = s0 + 56 * 1024, SF = s0 + 48 * 1024, CP = s0 + 60 * 1024;
-  if (threadIdx.x == 32) {  // metadata and scales the MMAs read
-    tc_cp_128x128b(tm + 256 + 48, smem_desc(E, 0, 128, kSwNone));
-    for (int j = 0; j < 8; ++j) tc_cp_32x128b_x4(tm + 256 + 4 * j, smem_desc(SF, 0, 128, kSwNone));
-    tc_commit(&setup_bar);
-    const unsigned long long lim = globaltimer_ns() + 2000000000ull;
-    while (!mbar_try_wait(&setup_bar, 0) && globaltimer_ns() < lim) {
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const int warp = threadIdx.x >> 5;
-  int ncp = 0;
-  bool mma = false;
-  if (mode == 0) mma = warp == 1;
-  if (mode == 1) ncp = warp == 1 ? 13 : 0;
-  if (mode == 2) { ncp = warp == 1 ? 13 : 0; mma = warp == 1; }
-  if (mode == 3) { ncp = warp == 0 ? 5 : (warp == 1 ? 0 : 4); mma = warp == 1; }
-  if (mode == 4) ncp = warp == 0 ? 4 : 3;
-  const unsigned long long t0 = globaltimer_ns();
-  if ((threadIdx.x & 31) == 0 && (ncp || mma)) {
-    const uint32_t idn = idesc_nvf4(128, 128, false), isp = idesc_nvf4(128, 128, true);
-    const uint32_t col = 320 + 48 * warp;  // this warp's copy columns: 320 + 48 w + [0, 48) < 512
-    for (int it = 0; it < iters; ++it) {
-      for (int j = 0; j < ncp; ++j) tc_cp_32x128b_x4(tm + col + 4 * (j % 12), smem_desc(CP, 0, 128, kSwNone));
-      if (mma) {
-        for (int j = 0; j < 2; ++j)
-          mma_sp_nvf4(tm, smem_desc(A + 32 * j, 16, 512, kSw64), smem_desc(B + 64 * j, 16, 1024, kSw128),
-                      tm + 256 + 48 + 2 * j, isp, tm + 256, tm + 256 + 8, 1u);
-        for (int j = 0; j < 4; ++j)
-          mma_nvf4(tm, smem_desc(A + 32 * j, 16, 1024, kSw128), smem_desc(B + 32 * j, 16, 1024, kSw128), idn,
-                   tm + 256, tm + 256 + 8, 1u);
-      }
-    }
-    tc_commit(&bar[warp]);
-    const unsigned long long lim = globaltimer_ns() + 2000000000ull;
-    while (!mbar_try_wait(&bar[warp], 0) && globaltimer_ns() < lim) {
-    }
-    tend[warp] = globaltimer_ns() - t0;
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long m = 0;
-    for (int w = 0; w < 4; ++w) m = tend[w] > m ? tend[w] : m;
-    ns[blockIdx.x] = m;
-  }
-  if (threadIdx.x < 32) {
-    tc_fence_after();
-    tmem_dealloc(tm, 512);
-  }
-}
-
 }  // namespace
-
-// Mean time per iteration (ns, over every SM) of tc_issue_kernel's mode.
-// Returns 0 on success.
-extern "C" int sharq_tc_issue_ns(int mode, int iters, double* ns_per_iter) {
-  int sms = 0, dev = 0;
-  if (mode < 0 || mode > 4 || iters < 1) return -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))
-    return -4;
-  unsigned long long* d = nullptr;
-  if (cudaMalloc(&d, sizeof(unsigned long long) * sms) != cudaSuccess) return -4;
-  cudaFuncSetAttribute(tc_issue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIssueSmem);
-  for (int rep = 0; rep < 2; ++rep) {  // first launch warms up
-    tc_issue_kernel<<<sms, 128, kIssueSmem>>>(mode, iters, d);
-    if (cudaDeviceSynchronize() != cudaSuccess) {
-      cudaFree(d);
-      return -4;
-    }
-  }
-  unsigned long long* h = new unsigned long long[sms];
-  cudaMemcpy(h, d, sizeof(unsigned long long) * sms, cudaMemcpyDeviceToHost);
-  double mean = 0.0;
-  for (int i = 0; i < sms; ++i) mean += (double)h[i];
-  delete[] h;
-  cudaFree(d);
-  *ns_per_iter = mean / sms / iters;
-  return 0;
-}
 
 // Measured FP4 peak in FLOP/s (logical FLOPs for the sparse form), N = 256
 // or 128, over every SM.  Returns 0 on success.

@@ -3,9 +3,11 @@
 For callers that cannot allocate device memory at run time (graph-capture
 regions, runtimes whose memory planner owns the GPU), sharq_prep_noalloc keeps
 the prep's working memory in a fixed array inside the library.  Called through
-the C ABI, it must give exactly sharq_prep's outputs, and keep doing so on the
-next call (the array keeps the previous call's contents).  This file is
-collected last so that a failure here comes after every other test has run.
+the C ABI, it must give exactly sharq_prep's outputs -- and the oracle's, bit
+for bit on every row -- and keep doing so on the next call (the array keeps
+the previous call's contents).  The cases cover the single-launch form and the
+wide two-launch form, which keeps each row's 1/rms in the array.  This file
+is collected last so that a failure here comes after every other test has run.
 """
 import numpy as np
 import pytest
@@ -13,6 +15,8 @@ import torch
 
 import sparse_activation_quantization_b200 as sq
 import synthetic
+from oracle import sharq as O
+from tests import _layout
 from tests import gpu_helpers as H
 
 pytestmark = pytest.mark.gpu
@@ -35,13 +39,29 @@ def _outputs(act, T, K):
     return out
 
 
-@pytest.mark.parametrize("T,K,D", [(16, 4096, 1024), (300, 1024, 512)])
+def _check_oracle(out, x, gamma, T, K):
+    """every row of the prepared operands against the oracle, bit for bit"""
+    p = O.prep(x, gamma, 1e-5)
+    assert out["s_g"] == float(p["s_g"])
+    Tp = -(-T // 128) * 128
+    flat = lambda name: out[name].reshape(-1)
+    assert np.array_equal(_layout.untile_meta(flat("meta"), Tp, K)[:T], p["meta"])
+    assert np.array_equal(_layout.untile_sp_codes(flat("sp_codes"), Tp, K)[:T], p["sp_codes"])
+    assert np.array_equal(_layout.untile_sf(flat("sp_sf"), Tp, K, 32)[:T], p["sp_sf"])
+    assert np.array_equal(_layout.untile_codes(flat("r_codes"), Tp, K)[:T], p["r_codes"])
+    assert np.array_equal(_layout.untile_sf(flat("r_sf"), Tp, K, 16)[:T], p["r_sf"])
+
+
+# (16, 4096): one thread-block cluster; (300, 1024): the grid-barrier form;
+# (400, 14336): the wide two-launch form (per-row 1/rms kept in the array)
+@pytest.mark.parametrize("T,K,D", [(16, 4096, 1024), (300, 1024, 512), (400, 14336, 256)])
 def test_noalloc_prep_matches_prep_on_consecutive_calls(T, K, D):
     stream = torch.cuda.current_stream().cuda_stream
     gamma = H.bf16_dev(synthetic.gamma(5, K))
     pw = sq.PackedWeight(torch.from_numpy(synthetic.weights(6, K, D)).to(torch.bfloat16).cuda())
     for call, seed in enumerate((11, 12)):      # two calls in a row, different inputs
-        x = H.bf16_dev(synthetic.activations(seed, T, K))
+        xh = synthetic.activations(seed, T, K)
+        x = H.bf16_dev(xh)
         ref = sq.PreparedAct(T, K)
         ref.buf.zero_()
         ref.prep(x, gamma, 1e-5)
@@ -53,6 +73,7 @@ def test_noalloc_prep_matches_prep_on_consecutive_calls(T, K, D):
         assert a["s_g"] == b["s_g"], call
         for name in ("r_codes", "r_sf", "sp_codes", "meta", "sp_sf"):
             assert np.array_equal(a[name], b[name]), (call, name)
+        _check_oracle(b, xh, synthetic.gamma(5, K), T, K)
         ya = sq.linear(ref, pw, out_dtype=torch.float32)
         yb = sq.linear(got, pw, out_dtype=torch.float32)
         torch.cuda.synchronize()
