@@ -47,6 +47,8 @@
 // shared memory once at start-up.
 // Every wait is bounded by the global timer; on timeout the CTA records
 // SHARQ_ERR_TIMEOUT in the workspace error word and leaves.
+#include <stdlib.h>
+
 #include "quant.cuh"
 
 namespace sharq {
@@ -981,7 +983,7 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
       mbar_init(&empty_bar[s], 1);
     }
     mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, 128);  // every epilogue thread, once per tile
+    mbar_init(&acc_empty, 4);  // each epilogue warp, once per tile
     for (int st = 0; st < C::kStages; ++st) mbar_init(&sf_full[st], C::kCW);
     for (int c = 0; c < C::kCW; ++c) mbar_init(&cp_fin[c], 1);
     fence_mbar_init();
@@ -1226,7 +1228,8 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive_local(&acc_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(&acc_empty);  // the warp's rows are in registers
         if (rl < valid) {
           uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off);
 #pragma unroll
@@ -1241,7 +1244,8 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
           if (rl < valid) store_row32(args.Y, 1, off + c, v, scale);
         }
         tc_fence_before();
-        mbar_arrive_local(&acc_empty);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_local(&acc_empty);
       }
       ++k;
     }
@@ -1253,6 +1257,456 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Pair form (prefill): two CTAs of a cluster run each 256 x 256 output tile
+// as one tensor-core unit (tcgen05 cta_group::2, M = 256).  CTA r of the pair
+// holds the tile's rows 128 r .. 128 r + 127 of the activation operands and
+// weight rows (output columns) 128 r .. 128 r + 127 of the shared FP4 weight
+// payload; the MMA reads B from both CTAs' shared memory, so each weight byte
+// crosses from L2 once per 256 activation rows instead of once per 128.  Per
+// CTA and 256-K stage that is 51 KB of operands (backbone, metadata, residual,
+// their scales, half the weight codes and both weight scale views) against
+// 67 KB in the one-CTA form, for the same tensor-core work.
+//   both CTAs  producer (warp 0): its own operand copies into its own ring of
+//              four stages;
+//              epilogue (warps 4-7): its own 128 accumulator rows.
+//   even CTA   MMA issuer (warp 1): both operands' MMAs with cta_group::2,
+//              committed to the ring slots of both CTAs at once (multicast)
+//              and to the stage's TMEM scale region;
+//              copy warps (2-3, 8-15): the stage's 19 scale and metadata
+//              copies into both CTAs' TMEM (each from its own shared memory)
+//              with cta_group::2.  Measured on B200 beside the MMAs, one warp
+//              issues a copy every ~75 ns, so a stage's copies keep pace with
+//              its six MMAs (~440 ns) only when spread over ten warps.
+//   odd CTA    warp 1 forwards "stage landed" to the even CTA: plain bulk
+//              copies complete only their own CTA's barrier, so it waits on
+//              its barrier and arrives on the even CTA's.
+// TMEM holds the 256-column accumulator and three scale regions (80 columns
+// each), so the shared-memory ring (four slots) runs one stage deeper than
+// the regions: the copies of stage g go to region g % 3 once the MMAs of
+// stage g - 3 have completed.  Both CTAs' epilogue threads release the
+// accumulator on the even CTA's barrier once the tile is in registers, before
+// their global stores, so the stores overlap the next tile's MMAs.  The
+// epilogue warpgroup takes 224 registers per thread (setmaxnreg), the other
+// three give theirs down to 96 (4 x 128 threads x their shares = the launch's
+// 65536).  Used for ungrouped SharQ and plain-NVFP4
+// GEMMs with at least two 128-row tiles; a pair's second m-tile may lie past
+// the activation's end (an odd tile count), in which case that CTA copies no
+// activation bytes and stores nothing.
+template <int kG>
+struct PairCfg {
+  static constexpr bool kHas1 = kG == kGemmSharq;  // the sparse backbone operand
+  static constexpr int BN = 256;                   // output columns per tile (both CTAs)
+  static constexpr int kWarps = 16;
+  static constexpr int kThreadsT = 32 * kWarps;
+  static constexpr int kCW = 10;                   // copy warps: 2, 3, 8..15
+  static constexpr int kEpiWarp0 = 4;              // epilogue warps 4..7 (TMEM lane quarters 0..3)
+  static constexpr int kRegsEpi = 224, kRegsOther = 96;  // setmaxnreg shares (x 128 threads each)
+  static constexpr int kOffB = 0;                         // this CTA's 128 weight rows
+  static constexpr int kOffA2 = kOffB + kCodesTile;       // residual (NVFP4: Xn) codes
+  static constexpr int kOffA1 = kOffA2 + kCodesTile;      // backbone codes
+  static constexpr int kOffE1 = kOffA1 + (kHas1 ? kSpTile : 0);
+  static constexpr int kOffS1 = kOffE1 + (kHas1 ? kMetaTile : 0);
+  static constexpr int kOffS2 = kOffS1 + (kHas1 ? kSf32Tile : 0);
+  static constexpr int kOffSFB32 = kOffS2 + kSf16Tile;    // both weight halves' views
+  static constexpr int kOffSFB16 = kOffSFB32 + (kHas1 ? 2 * kSf32Tile : 0);
+  static constexpr int kStageBytes = (kOffSFB16 + 2 * kSf16Tile + 1023) / 1024 * 1024;
+  static constexpr int kStages = 4;  // shared-memory ring slots
+  static constexpr int kRegions = 3;  // TMEM scale regions
+  // TMEM: the 256-column accumulator and the scale regions
+  static constexpr uint32_t kSfbCols = BN / 32;
+  static constexpr uint32_t kSfE1 = 0, kSfS1 = 8, kSfS2 = 16, kSfB32 = 32, kSfB16 = 32 + 2 * kSfbCols;
+  static constexpr uint32_t kSfRegion = 32 + 6 * kSfbCols;
+  static constexpr uint32_t kColAcc = 0, kColSf0 = BN;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  // transaction bytes of one CTA's stage with `rows` valid activation rows
+  __host__ __device__ static constexpr uint32_t tx(uint32_t rows) {
+    return kCodesTile + (kHas1 ? 2 * kSf32Tile : 0) + 2 * kSf16Tile +
+           (rows ? rows * (128u + (kHas1 ? 64u + 16u : 0u)) + (kHas1 ? kSf32Tile : 0) + kSf16Tile : 0u);
+  }
+  static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory overflow");
+  static_assert(BN + kRegions * kSfRegion <= kTmemCols, "TMEM overflow");
+  static_assert(kRegsEpi + 3 * kRegsOther <= 65536 / kThreadsT * 4, "register split above the launch's share");
+};
+
+// the pair kernel's register split (per thread; each warpgroup executes one)
+__device__ __forceinline__ void regs_inc_epi() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory"); }
+__device__ __forceinline__ void regs_dec_other() { asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory"); }
+
+template <int kG>
+__global__ void __launch_bounds__(PairCfg<kG>::kThreadsT, 1)
+    sharq_gemm_pair_kernel(const GemmArgs args, int m_tiles) {
+  using C = PairCfg<kG>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[C::kStages];
+  __shared__ __align__(8) uint64_t empty_bar[C::kStages];
+  __shared__ __align__(8) uint64_t peer_full[C::kStages];     // even CTA: the odd CTA's stage has landed
+  __shared__ __align__(8) uint64_t sf_full[C::kRegions];      // even CTA: a region's copies have landed
+  __shared__ __align__(8) uint64_t region_free[C::kRegions];  // even CTA: the MMAs reading a region are done
+  __shared__ __align__(8) uint64_t acc_full;
+  __shared__ __align__(8) uint64_t acc_empty;                 // even CTA: both epilogues took the accumulator
+  __shared__ __align__(8) uint64_t cp_fin[C::kCW];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_sh;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int KS = args.K >> 8;
+  const int n_tiles = args.D / C::BN;
+  const int m2_tiles = (m_tiles + 1) >> 1;
+  const int ntiles = m2_tiles * n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&peer_full[s], 1);
+    }
+    for (int r = 0; r < C::kRegions; ++r) {
+      mbar_init(&sf_full[r], C::kCW);
+      mbar_init(&region_free[r], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, 8);  // the 4 epilogue warps of each CTA, once per tile
+    for (int c = 0; c < C::kCW; ++c) mbar_init(&cp_fin[c], 1);
+    fence_mbar_init();
+    abort_sh = 0;
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tmem_base_sh, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (C::kHas1) {
+    // metadata of rows past a tile's valid rows is never copied in: a valid
+    // pattern (pairs 0 and 1) everywhere once; later tiles leave metadata
+    // written by sharq_prep there, which is valid as well
+    for (int idx = threadIdx.x; idx < C::kStages * 128; idx += C::kThreadsT) {
+      const int st = idx >> 7, row = idx & 127;
+      *reinterpret_cast<uint4*>(smem + st * C::kStageBytes + C::kOffE1 + row * 16) =
+          make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers and TMEM exist before any pair traffic
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t peer_full_lead = mapa_shared(smem_u32(&peer_full[0]), 0);
+  const uint32_t acc_empty_lead = mapa_shared(smem_u32(&acc_empty), 0);
+  const int cw = warp == 2 || warp == 3 ? warp - 2 : (warp >= 8 ? warp - 6 : -1);  // copy warp index
+  const bool epi_wg = warp >= C::kEpiWarp0 && warp < C::kEpiWarp0 + 4;
+
+  if (!epi_wg) {
+  regs_dec_other();  // warpgroups 0, 2 and 3 give registers to the epilogue
+  if (warp == 0) {
+    // ------------------------------------------------- producer (both) ----
+    if (lane == 0) {
+      grid_dependency_wait();  // the activation comes from the preceding sharq_prep
+      if (blockIdx.x == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
+      uint32_t g = 0;
+      for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
+        const int m2 = tile / n_tiles, nt = tile - m2 * n_tiles;
+        const int mt = 2 * m2 + (int)rank;
+        const uint32_t rows = (uint32_t)max(0, min(128, args.T - mt * 128));
+        const uint32_t tx = C::tx(rows);
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        const size_t a_tile0 = (size_t)mt * KS;
+        const size_t b_tile0 = (size_t)nt * 2 * KS;  // this column tile's first weight half
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages;
+          if (g >= (uint32_t)C::kStages &&
+              !mbar_wait(&empty_bar[s], ((g / C::kStages) & 1) ^ 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          uint8_t* st = smem + s * C::kStageBytes;
+          uint64_t* fb = &full_bar[s];
+          mbar_arrive_expect_tx(fb, tx);
+          // scales first: the copy warps need only those
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const size_t bh = b_tile0 + (size_t)h * KS + i;
+            bulk_g2s(st + C::kOffSFB16 + h * kSf16Tile, args.w_sf16 + bh * kSf16Tile, kSf16Tile, fb);
+            if (C::kHas1) bulk_g2s(st + C::kOffSFB32 + h * kSf32Tile, args.w_sf32 + bh * kSf32Tile, kSf32Tile, fb);
+          }
+          const size_t at = a_tile0 + i;
+          if (rows) {
+            bulk_g2s(st + C::kOffS2, args.a_rsf + at * kSf16Tile, kSf16Tile, fb);
+            if (C::kHas1) {
+              bulk_g2s(st + C::kOffE1, args.a_meta + at * kMetaTile, rows * 16u, fb);
+              bulk_g2s(st + C::kOffS1, args.a_spsf + at * kSf32Tile, kSf32Tile, fb);
+            }
+          }
+          const size_t bt = b_tile0 + (size_t)rank * KS + i;
+          bulk_g2s(st + C::kOffB, args.w_codes + bt * kCodesTile, kCodesTile, fb);
+          if (rows) {
+            bulk_g2s(st + C::kOffA2, args.a_r + at * kCodesTile, rows * 128u, fb);
+            if (C::kHas1) bulk_g2s(st + C::kOffA1, args.a_sp + at * kSpTile, rows * 64u, fb);
+          }
+        }
+      }
+      // every slot's last use has been released by the MMAs (their
+      // completion arrives on this CTA's barriers) before the CTA may leave
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+      for (int j = 0; j < C::kStages && !abort_sh; ++j, ++g)
+        if (g >= (uint32_t)C::kStages && !mbar_wait(&empty_bar[g % C::kStages], ((g / C::kStages) & 1) ^ 1,
+                                                   deadline, &abort_sh)) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------------------------------------- MMA (even CTA) ----
+      constexpr uint32_t idesc_dn = idesc_nvf4(256, C::BN, false);
+      constexpr uint32_t idesc_sp = idesc_nvf4(256, C::BN, true);
+      uint32_t g = 0, k = 0;
+      for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        if (k > 0 && !mbar_wait_cluster(&acc_empty, (k - 1) & 1, deadline, &abort_sh)) {
+          record_error(args.err, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        tc_fence_after();
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages, r = g % C::kRegions;
+          const uint32_t ph = (g / C::kStages) & 1;
+          if (!mbar_wait(&full_bar[s], ph, deadline, &abort_sh) ||
+              !mbar_wait_cluster(&peer_full[s], ph, deadline, &abort_sh) ||
+              !mbar_wait(&sf_full[r], (g / C::kRegions) & 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t sf = tmem + C::kColSf0 + (uint32_t)r * C::kSfRegion;
+          if (C::kHas1) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              mma_pair_sp_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffA1 + 32 * j, 16, 512, kSw64),
+                               smem_desc(st + C::kOffB + 64 * j, 16, 1024, kSw128), sf + C::kSfE1 + 2 * j, idesc_sp,
+                               sf + C::kSfS1 + 4 * j, sf + C::kSfB32 + j * C::kSfbCols, (i > 0 || j > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_pair_nvf4(tmem + C::kColAcc, smem_desc(st + C::kOffA2 + 32 * j, 16, 1024, kSw128),
+                          smem_desc(st + C::kOffB + 32 * j, 16, 1024, kSw128), idesc_dn, sf + C::kSfS2 + 4 * j,
+                          sf + C::kSfB16 + j * C::kSfbCols, (C::kHas1 || i > 0 || j > 0) ? 1u : 0u);
+          tc_commit_pair_mc(&empty_bar[s], 0x3);  // both CTAs' ring slot s
+          tc_commit_pair(&region_free[r]);        // the scale region, for the copy warps
+        }
+        tc_commit_pair_mc(&acc_full, 0x3);        // both CTAs' accumulator rows
+        ++k;
+      }
+    } else if (lane == 0) {
+      // ------------------------- odd CTA: forward "stage landed" ----
+      uint32_t g = 0;
+      for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages;
+          if (!mbar_wait(&full_bar[s], (g / C::kStages) & 1, deadline, &abort_sh)) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          // the stage's bytes are in this CTA's shared memory (its barrier
+          // completed); the even CTA's copies and MMAs read them after its
+          // wait on peer_full, so the arrival need not order anything
+          mbar_arrive_remote_relaxed(peer_full_lead + (uint32_t)(s * sizeof(uint64_t)));
+        }
+      }
+    }
+  } else if (cw >= 0) {
+    if (lane == 0 && leader) {
+      // ----------------------------------------- copy warps (even CTA) ----
+      uint32_t g = 0;
+      for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        for (int i = 0; i < KS; ++i, ++g) {
+          const int s = g % C::kStages, r = g % C::kRegions;
+          const uint32_t ph = (g / C::kStages) & 1;
+          // both CTAs' stage data has landed, and the MMAs of stage g - 3
+          // (the region's previous user) have completed
+          if (!mbar_wait(&full_bar[s], ph, deadline, &abort_sh) ||
+              !mbar_wait_cluster(&peer_full[s], ph, deadline, &abort_sh) ||
+              (g >= (uint32_t)C::kRegions &&
+               !mbar_wait(&region_free[r], ((g / C::kRegions) & 1) ^ 1, deadline, &abort_sh))) {
+            record_error(args.err, kErrTimeout);
+            abort_sh = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t sf = tmem + C::kColSf0 + (uint32_t)r * C::kSfRegion;
+          int n = 0;
+          auto cp4 = [&](uint32_t taddr, uint32_t saddr) {
+            if (n++ % C::kCW == cw) tc_cp_pair_32x128b_x4(taddr, smem_desc(saddr, 0, 128, kSwNone));
+          };
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) cp4(sf + C::kSfB16 + j * C::kSfbCols + 4 * h, st + C::kOffSFB16 + h * kSf16Tile + 512 * j);
+          if (C::kHas1) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                cp4(sf + C::kSfB32 + j * C::kSfbCols + 4 * h, st + C::kOffSFB32 + h * kSf32Tile + 512 * j);
+            if (n++ % C::kCW == cw) tc_cp_pair_128x128b(sf + C::kSfE1, smem_desc(st + C::kOffE1, 0, 128, kSwNone));
+#pragma unroll
+            for (int j = 0; j < 2; ++j) cp4(sf + C::kSfS1 + 4 * j, st + C::kOffS1 + 512 * j);
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) cp4(sf + C::kSfS2 + 4 * j, st + C::kOffS2 + 512 * j);
+          tc_commit_pair(&sf_full[r]);
+        }
+      }
+      tc_commit_pair(&cp_fin[cw]);
+      const uint64_t lim = globaltimer_ns() + kWaitLimitNs;
+      while (!mbar_try_wait(&cp_fin[cw], 0) && globaltimer_ns() < lim) {
+      }
+    }
+  }
+  } else {
+    // ---------------------------------------------- epilogue (both) ----
+    regs_inc_epi();  // the epilogue warpgroup holds a 256-column row
+    const int sp = warp & 3;  // TMEM lane quarter this warp may access
+    const int rl = sp * 32 + lane;
+    grid_dependency_wait();  // s_g is written by the preceding sharq_prep
+    const float s_tensor = args.per_token ? 0.0f : *args.s_g;
+    const float s_w = args.s_w[0];
+    uint32_t k = 0;
+    for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
+      const int m2 = tile / n_tiles, nt = tile - m2 * n_tiles;
+      const int mt = 2 * m2 + (int)rank;
+      const int valid = max(0, min(128, args.T - mt * 128));
+      const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+      if (!mbar_wait_cluster(&acc_full, k & 1, deadline, &abort_sh)) {
+        record_error(args.err, kErrTimeout);
+        abort_sh = 1;
+        break;
+      }
+      tc_fence_after();
+      const int row = mt * 128 + rl;
+      const float scale = __fmul_rn(args.per_token ? (rl < valid ? args.s_g[row] : 0.0f) : s_tensor, s_w);
+      const size_t off = (size_t)row * args.D + (size_t)nt * C::BN;
+      if (!args.out_f32) {
+        uint32_t pk[C::BN / 2];  // the row as packed bf16, then the accumulator is free
+#pragma unroll
+        for (int c = 0; c < C::BN; c += 64) {  // two loads in flight per wait
+          uint32_t v[2][32];
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v[0]);
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c + 32, v[1]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[q >> 4][2 * (q & 15)]), scale),
+                                                      __fmul_rn(__uint_as_float(v[q >> 4][2 * (q & 15) + 1]), scale));
+            pk[c / 2 + q] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_lead);  // loads done: one arrival per warp, 8 per tile
+        if (rl < valid) {
+          uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off);
+#pragma unroll
+          for (int q = 0; q < C::BN / 8; ++q) y[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < C::BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + ((uint32_t)(sp * 32) << 16) + C::kColAcc + c, v);
+          tmem_ld_wait();
+          if (rl < valid) store_row32(args.Y, 1, off + c, v, scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_lead);
+      }
+      ++k;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA frees its TMEM or leaves while the pair's work may touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::kTmemCols);
+  }
+}
+
+// The pair kernel's register split (setmaxnreg) needs the launch to hold the
+// full 65536 registers / 512 threads; a build whose kernel was allotted fewer
+// would make the epilogue's increase wait for registers that never come, so
+// the launcher checks and otherwise uses the one-CTA kernel.
+template <int kG>
+bool pair_regs_ok() {
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, sharq_gemm_pair_kernel<kG>) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  using C = PairCfg<kG>;
+  return fa.numRegs * C::kThreadsT >= 128 * (C::kRegsEpi + 3 * C::kRegsOther);
+}
+
+template <int kG>
+cudaError_t launch_pair(const GemmArgs& a, int m_tiles, cudaStream_t stream, bool* launched) {
+  using C = PairCfg<kG>;
+  static int sms[64] = {};  // SM count, or -1 if this device cannot run the pair form
+  *launched = false;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (sms[dev] == 0) {
+    if (!pair_regs_ok<kG>()) {
+      sms[dev] = -1;
+    } else {
+      e = cudaFuncSetAttribute(sharq_gemm_pair_kernel<kG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      int n = 0;
+      e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      sms[dev] = n;
+    }
+  }
+  if (sms[dev] < 2) return cudaSuccess;
+  const long long ntiles = (long long)((m_tiles + 1) / 2) * (a.D / C::BN);
+  const long long pairs = ntiles < sms[dev] / 2 ? ntiles : sms[dev] / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(C::kThreadsT);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, sharq_gemm_pair_kernel<kG>, a, m_tiles);
+  *launched = e == cudaSuccess;
+  return e;
 }
 
 template <int BN, int kG>
@@ -1332,6 +1786,17 @@ cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
 
 }  // namespace
 
+// The CTA-pair prefill form is on unless the environment sets
+// SHARQ_GEMM_PAIR=0 (read once per process), which runs those shapes on the
+// one-CTA persistent kernel instead -- the same result, for comparing the two.
+bool pair_form_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("SHARQ_GEMM_PAIR");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 #ifdef SHARQ_TRACE
 extern "C" int sharq_debug_set_trace(void* p) {
   return cudaMemcpyToSymbol(g_trace, &p, sizeof(p)) == cudaSuccess ? 0 : -4;
@@ -1387,6 +1852,14 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   if (splits > 1 && two_way) {
     if (bn != 128 || splits > 4) return cudaErrorInvalidValue;
     return launch_cfg<128, true, false>(a, m_tiles, stream);
+  }
+  // prefill SharQ / plain-NVFP4 GEMMs with two or more 128-row tiles and
+  // 256-column tiles: the CTA-pair form
+  if (two_way && !group_offsets && E == 1 && m_tiles >= 2 && bn == 256 && a.D % 256 == 0 && pair_form_enabled()) {
+    bool launched = false;
+    const cudaError_t e = gmode == kGemmSharq ? launch_pair<kGemmSharq>(a, m_tiles, stream, &launched)
+                                              : launch_pair<kGemmNvfp4>(a, m_tiles, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
   }
   // the Table-5 modes run the persistent form at every size
   const int pbn = (a.D % 256 == 0) ? 256 : 128;

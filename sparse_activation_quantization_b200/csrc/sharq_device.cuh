@@ -179,6 +179,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
+// relaxed arrive on an mbarrier of another CTA: orders none of this thread's
+// earlier memory operations (a release at cluster scope costs ~0.7 us on
+// B200).  For signals whose data is not written by this thread: TMA bytes
+// that already completed this CTA's own barrier, or TMEM loads already waited
+// for with tcgen05.wait::ld.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -189,6 +197,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+// Bounded wait with cluster-scope acquire, for barriers that peers arrive on
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t deadline,
+                                                  volatile int* abort) {
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() > deadline) return false;
+  }
+  return true;
 }
 __device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr) {
   float4 v;
@@ -333,6 +350,67 @@ __device__ __forceinline__ void mma_sp_mxf4(uint32_t d, uint64_t adesc, uint64_t
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %5, 0;\n\t"
       "tcgen05.mma.sp.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, [%3], %4, [%6], [%7], "
+      "p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(e), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// ---------------------------------------------- tcgen05, CTA pairs ----
+// The cta_group::2 forms: two CTAs of a cluster (ranks 2i, 2i+1) act as one
+// MMA unit.  One thread of the even CTA issues the MMAs and copies for both;
+// each CTA keeps its own rows of A, its half of B's rows and its own rows of
+// the accumulator, at the same shared-memory and TMEM addresses in both.  A
+// kernel uses one cta_group throughout.
+
+// collective over the pair: the same warp of both CTAs allocates the same
+// columns in both TMEMs, each writing the address to its own shared memory
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// arrive on `bar` of this CTA once the pair ops this thread issued finish
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// ... on the barrier at the same offset in every CTA of cta_mask
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                   "r"(smem_u32(bar)),
+               "h"(cta_mask)
+               : "memory");
+}
+// each CTA's shared memory (same offset) -> its own TMEM, as the 1-CTA forms
+__device__ __forceinline__ void tc_cp_pair_128x128b(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+__device__ __forceinline__ void tc_cp_pair_32x128b_x4(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+// D (M = 256 over the pair) (+)= A x B, per-16 E4M3 block scales from TMEM
+__device__ __forceinline__ void mma_pair_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma_pair_sp_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t e,
+                                                 uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%3], %4, [%6], [%7], "
       "p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(e), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
