@@ -67,6 +67,18 @@ def gemm_split_k(L):
     return m * n < 74
 
 
+def gemm_kernel_name(L):
+    """The kernel sharq_linear runs for this layer (SharQ mode, ungrouped),
+    by the library's launch rule: split-K decode kernel, CTA-pair prefill
+    kernel (two or more 128-row tiles, 256-column tiles), or the one-CTA
+    persistent kernel."""
+    if gemm_split_k(L):
+        return "sharq_gemm_kernel (split-K)"
+    if -(-L.T // 128) >= 2 and L.D % 256 == 0:
+        return "sharq_gemm_pair_kernel"
+    return "sharq_gemm_persistent_kernel"
+
+
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch,
 # from one ncu capture of this script's command, keyed by layer and kernel;
 # None where none was taken.  Reset an entry whenever its kernel changes,
@@ -562,7 +574,7 @@ def run_gpu(args, world, rank, local):
     dom = max(layers, key=lambda L: per[L.name]["gemm_us"])
     t_tensor = dom.flops / (eff_tflops * 1e12)
     t_hbm = gemm_alg_bytes(dom.T, dom.K, dom.D) / (peak_gbs * 1e9)
-    gemm_kernel = ("sharq_gemm_kernel (split-K)" if gemm_split_k(dom) else "sharq_gemm_persistent_kernel")
+    gemm_kernel = gemm_kernel_name(dom)
     if t_tensor >= t_hbm:
         ach = per[dom.name]["gemm_tflops"]
         roof = {"kernel": f"{gemm_kernel} ({dom.name})", "bound": "tensor", "achieved": ach, "peak": eff_tflops,

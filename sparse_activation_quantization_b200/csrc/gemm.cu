@@ -202,6 +202,36 @@ __device__ __forceinline__ void store4(void* Y, int out_f32, size_t off, float4 
   }
 }
 
+// Global stores of a warp's 32 output rows (row = lane, kCols bf16 columns
+// held as packed pairs pk) through the warp's 4 KB of shared memory, 64
+// columns (128 bytes of each row) at a time: stored straight from registers a
+// warp instruction would touch 32 rows' lines, here it writes 4 whole 128-byte
+// lines.  Chunk q of row r sits at q ^ (r % 8) so both the writes and the
+// reads spread over all banks.  y0: row 0 of the warp, first column; ld: the
+// row stride (elements); rows: the warp's valid rows (the others are not
+// stored).
+template <int kCols>
+__device__ __forceinline__ void store_rows_bf16_staged(const uint32_t (&pk)[kCols / 2], uint8_t* wst,
+                                                       __nv_bfloat16* y0, size_t ld, int rows, int lane) {
+  const int rsub = lane >> 3, q = lane & 7;  // store phase: row within a group of 4, 16-byte chunk
+#pragma unroll
+  for (int c = 0; c < kCols / 64; ++c) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint4*>(wst + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+          make_uint4(pk[32 * c + 4 * j], pk[32 * c + 4 * j + 1], pk[32 * c + 4 * j + 2], pk[32 * c + 4 * j + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int r = 4 * it + rsub;
+      if (r < rows)
+        *reinterpret_cast<uint4*>(y0 + (size_t)r * ld + 64 * c + 8 * q) =
+            *reinterpret_cast<const uint4*>(wst + r * 128 + ((q ^ (r & 7)) << 4));
+    }
+    __syncwarp();
+  }
+}
+
 // Expert that owns m-tile mt in the grouped form (offsets are 128-row
 // aligned), 0 without groups, -1 if the offsets do not cover the tile.
 __device__ __forceinline__ int tile_expert(const GemmArgs& args, int mt) {
@@ -893,8 +923,12 @@ struct PCfg {
   // rounded to 1 KB so that every stage's swizzled code tiles (first in the
   // stage) stay 1024-byte aligned; the scale regions need only 16 bytes
   static constexpr int kStageBytes = (kOffSFB16 + (kB16 ? kHalves * kSfDn : 0) + 1023) / 1024 * 1024;
-  static constexpr int kStages = (BN == 128 && 4 * kStageBytes + 1024 <= 232448) ? 4 : 3;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  static constexpr int kStages = (BN == 128 && 4 * kStageBytes + 4 * 4096 + 1024 <= 232448) ? 4 : 3;
+  // bf16 output staging after the ring, 4 KB per epilogue warp, where it fits
+  // (not beside the three 72 KB stages of the Dense+Dense operand set)
+  static constexpr bool kStaged = kStages * kStageBytes + 4 * 4096 + 1024 <= 232448;
+  static constexpr int kOffStage = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kOffStage + (kStaged ? 4 * 4096 : 0) + 1024;
   // TMEM: accumulator, then one scale region per ring slot: 32 activation
   // columns + the weight scale columns
   static constexpr uint32_t kColAcc = 0;
@@ -1230,7 +1264,12 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_local(&acc_empty);  // the warp's rows are in registers
-        if (rl < valid) {
+        if constexpr (C::kStaged) {
+          store_rows_bf16_staged<BN>(pk, smem + C::kOffStage + (size_t)sp * 4096,
+                                     static_cast<__nv_bfloat16*>(args.Y) + (size_t)(mt * 128 + sp * 32) * args.D +
+                                         (size_t)nt * BN,
+                                     (size_t)args.D, valid - sp * 32, lane);
+        } else if (rl < valid) {
           uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off);
 #pragma unroll
           for (int q = 0; q < BN / 8; ++q) y[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -1321,7 +1360,9 @@ struct PairCfg {
   static constexpr uint32_t kSfRegion = 32 + 6 * kSfbCols;
   static constexpr uint32_t kColAcc = 0, kColSf0 = BN;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  // bf16 output staging: 4 KB per epilogue warp (32 rows x 64 columns)
+  static constexpr int kOffStage = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kOffStage + 4 * 4096 + 1024;
   // transaction bytes of one CTA's stage with `rows` valid activation rows
   __host__ __device__ static constexpr uint32_t tx(uint32_t rows) {
     return kCodesTile + (kHas1 ? 2 * kSf32Tile : 0) + 2 * kSf16Tile +
@@ -1620,11 +1661,10 @@ __global__ void __launch_bounds__(PairCfg<kG>::kThreadsT, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote_relaxed(acc_empty_lead);  // loads done: one arrival per warp, 8 per tile
-        if (rl < valid) {
-          uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + off);
-#pragma unroll
-          for (int q = 0; q < C::BN / 8; ++q) y[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        store_rows_bf16_staged<C::BN>(pk, smem + C::kOffStage + (size_t)sp * 4096,
+                                      static_cast<__nv_bfloat16*>(args.Y) + (size_t)(mt * 128 + sp * 32) * args.D +
+                                          (size_t)nt * C::BN,
+                                      (size_t)args.D, valid - sp * 32, lane);
       } else {
 #pragma unroll 1
         for (int c = 0; c < C::BN; c += 32) {
