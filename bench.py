@@ -80,10 +80,14 @@ def gemm_kernel_name(L):
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch,
-# from one ncu capture of this script's command, keyed by layer and kernel;
-# None where none was taken.  Reset an entry whenever its kernel changes,
-# until it is captured again.
-NCU_TRAFFIC = {}
+# from one ncu capture of this script's default command (the eager step's
+# launch), keyed by layer and kernel;
+# a prep entry sums its two launches (row statistics + strip quantizer).
+# Reset an entry whenever its kernel changes, until it is captured again.
+NCU_TRAFFIC = {
+    "gate_up_T8192/gemm": 138069504 + 577048832,
+    "down_T8192/prep": (310391552 + 4768768) + (310826496 + 108708864),
+}
 
 
 def read_peaks():

@@ -102,6 +102,10 @@ struct GemmArgs {
   int sharq_mode;
   int splits;
   int per_token;  // s_g holds one scale per activation row
+  // persistent / pair tile order: 0 = row-tile major (consecutive tiles share
+  // activation rows), 1 = column-tile major (consecutive tiles share weight
+  // columns); the launcher picks the order that keeps the smaller operand in L2
+  int n_major;
   // fused decode form: raw activations are prepared inside the GEMM
   const __nv_bfloat16* X;      // [T][K] bf16
   const __nv_bfloat16* gamma;  // [K] bf16 or nullptr
@@ -251,6 +255,22 @@ __device__ __forceinline__ int tile_expert(const GemmArgs& args, int mt) {
   while (e >= 0 && e < args.E && args.group_offsets[e + 1] <= row0) ++e;
   if (e < 0 || e >= args.E || args.group_offsets[e] > row0 || args.group_offsets[e + 1] <= row0) e = -1;
   return e;
+}
+
+// (row tile, column tile) of persistent tile index `tile` over m_tiles x
+// n_tiles tiles.  Row-major order suits operands whose activation side is the
+// larger (each weight column tile is revisited while the whole weight stays in
+// L2); column-major order suits a weight larger than the activation, e.g. a
+// wide gate+up projection whose 80 MB weight would otherwise be evicted by the
+// output stream before the next row tile comes back to it.
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int n_major, int& mt, int& nt) {
+  if (n_major) {
+    nt = tile / m_tiles;
+    mt = tile - nt * m_tiles;
+  } else {
+    mt = tile / n_tiles;
+    nt = tile - mt * n_tiles;
+  }
 }
 
 // Programmatic dependent launch: wait until the preceding grid in the stream
@@ -1051,7 +1071,8 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
       if (blockIdx.x == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
       uint32_t g = 0;  // stage counter across tiles
       for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
-        const int mt = tile / n_tiles, nt = tile - mt * n_tiles;
+        int mt, nt;
+        tile_coords(tile, m_tiles, n_tiles, args.n_major, mt, nt);
         const int expert = tile_expert(args, mt);
         if (expert < 0) {
           if (nt == 0) record_error(args.err, kErrInvalid);
@@ -1101,7 +1122,9 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
       constexpr uint32_t idesc_sp = idesc_nvf4(128, BN, true);
       uint32_t g = 0, k = 0;  // stage counter, tiles done
       for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
-        if (tile_expert(args, tile / n_tiles) < 0) continue;
+        int tmt, tnt;
+        tile_coords(tile, m_tiles, n_tiles, args.n_major, tmt, tnt);
+        if (tile_expert(args, tmt) < 0) continue;
         const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
         // the epilogue has taken the previous tile's accumulator
         if (k > 0 && !mbar_wait(&acc_empty, (k - 1) & 1, deadline, &abort_sh)) {
@@ -1203,7 +1226,9 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
       const int cw = warp - 6;
       uint32_t g = 0;  // stage counter across tiles, as the MMA warp's
       for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
-        if (tile_expert(args, tile / n_tiles) < 0) continue;
+        int tmt, tnt;
+        tile_coords(tile, m_tiles, n_tiles, args.n_major, tmt, tnt);
+        if (tile_expert(args, tmt) < 0) continue;
         const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
         for (int i = 0; i < KS; ++i, ++g) {
           const int s = g % C::kStages;
@@ -1233,7 +1258,8 @@ __global__ void __launch_bounds__(PCfg<BN, kG>::kThreadsT, 1)
     const float s_tensor = args.per_token ? 0.0f : *args.s_g;
     uint32_t k = 0;
     for (int tile = blockIdx.x; tile < ntiles && !abort_sh; tile += gridDim.x) {
-      const int mt = tile / n_tiles, nt = tile - mt * n_tiles;
+      int mt, nt;
+      tile_coords(tile, m_tiles, n_tiles, args.n_major, mt, nt);
       const int expert = tile_expert(args, mt);
       if (expert < 0) continue;
       const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
@@ -1454,7 +1480,8 @@ __global__ void __launch_bounds__(PairCfg<kG>::kThreadsT, 1)
       if (blockIdx.x == 0 && args.act_err && *args.act_err) record_error(args.err, *args.act_err);
       uint32_t g = 0;
       for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
-        const int m2 = tile / n_tiles, nt = tile - m2 * n_tiles;
+        int m2, nt;
+        tile_coords(tile, m2_tiles, n_tiles, args.n_major, m2, nt);
         const int mt = 2 * m2 + (int)rank;
         const uint32_t rows = (uint32_t)max(0, min(128, args.T - mt * 128));
         const uint32_t tx = C::tx(rows);
@@ -1630,7 +1657,8 @@ __global__ void __launch_bounds__(PairCfg<kG>::kThreadsT, 1)
     const float s_w = args.s_w[0];
     uint32_t k = 0;
     for (int tile = pair; tile < ntiles && !abort_sh; tile += npairs) {
-      const int m2 = tile / n_tiles, nt = tile - m2 * n_tiles;
+      int m2, nt;
+      tile_coords(tile, m2_tiles, n_tiles, args.n_major, m2, nt);
       const int mt = 2 * m2 + (int)rank;
       const int valid = max(0, min(128, args.T - mt * 128));
       const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
@@ -1880,6 +1908,11 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
   a.eps = eps_fused;
   const int m_tiles = Tp / 128;
   if (m_tiles == 0) return cudaSuccess;
+  // keep the smaller operand resident in L2: column-tile major order when the
+  // packed weight (0.59375 B per element) outweighs the prepared activation
+  // (0.90625 B per element of the padded rows).  Grouped experts keep row
+  // order: consecutive row tiles of one expert share its (small) weight.
+  a.n_major = (!group_offsets && (double)D * 0.59375 > (double)Tp * 0.90625) ? 1 : 0;
   if (X_fused) {  // fused decode form
     if (T > 32 || m_tiles != 1 || gmode != kGemmSharq || group_offsets || per_token) return cudaErrorInvalidValue;
     if (splits > 1) {
