@@ -631,6 +631,45 @@ def run_gpu(args, world, rank, local):
     return line
 
 
+def run_epilogues(args):
+    """Fused preceding-op epilogues against the unfused framework ops, per call
+    (CUDA events over graph-replayed back-to-back calls): the SwiGLU product of
+    a down projection's input (K = 14336, no RMSNorm, h written out) and the
+    residual-stream add before an RMSNorm prep (K = 4096, h written out)."""
+    import torch
+    import sparse_activation_quantization_b200 as sq
+    import synthetic
+    from sparse_activation_quantization_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    out = {}
+    for T in args.T:
+        K = 14336
+        g = torch.from_numpy(synthetic.activations(1, T, K) * np.float32(0.5)).to(torch.bfloat16).to(dev)
+        u = torch.from_numpy(synthetic.activations(2, T, K, base="student_t")).to(torch.bfloat16).to(dev)
+        h = torch.empty_like(u)
+        act = sq.PreparedAct(T, K, device=dev)
+        fused = kernel_us(lambda i: act.prep_silu_mul(g, u, h, None, EPS, stream=stream), 1, stream, launches=32)
+        unfused = kernel_us(lambda i: act.prep(torch.mul(torch.nn.functional.silu(g), u, out=h), None, EPS,
+                                               stream=stream), 1, stream, launches=32)
+        prep_h = kernel_us(lambda i: act.prep(h, None, EPS, stream=stream), 1, stream, launches=32)
+        K2 = 4096
+        x = torch.from_numpy(synthetic.activations(3, T, K2)).to(torch.bfloat16).to(dev)
+        res = torch.from_numpy(synthetic.activations(4, T, K2)).to(torch.bfloat16).to(dev)
+        gam = torch.from_numpy(synthetic.gamma(5, K2)).to(torch.bfloat16).to(dev)
+        hr = torch.empty_like(res)
+        act2 = sq.PreparedAct(T, K2, device=dev)
+        rfused = kernel_us(lambda i: act2.prep_residual(x, res, hr, gam, EPS, stream=stream), 1, stream, launches=32)
+        runfused = kernel_us(lambda i: act2.prep(torch.add(x, res, out=hr), gam, EPS, stream=stream), 1, stream,
+                             launches=32)
+        out[f"T{T}"] = {"silu_mul_fused_us": round(fused, 2), "silu_mul_torch_plus_prep_us": round(unfused, 2),
+                        "prep_of_h_us": round(prep_h, 2), "residual_fused_us": round(rfused, 2),
+                        "residual_torch_plus_prep_us": round(runfused, 2)}
+    print(json.dumps({"epilogues": out, "K_silu": 14336, "K_residual": 4096}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -642,6 +681,8 @@ def main():
     ap.add_argument("--compare", action="store_true",
                     help="also time plain NVFP4 and bf16 cuBLAS on the same layers")
     ap.add_argument("--T", type=int, nargs="+", default=None)
+    ap.add_argument("--epilogues", action="store_true",
+                    help="time the fused SwiGLU / residual-add preps against the unfused framework ops")
     ap.add_argument("--decode-form", default="two", choices=["two", "fused"],
                     help="T <= 32 layers: sharq_prep + sharq_linear (two) or sharq_prep_linear's single kernel")
     args = ap.parse_args()
@@ -649,6 +690,11 @@ def main():
     if args.T is None:
         args.T = DEFAULT_T[args.workload]
     world, rank, local = init_dist(args)
+    if args.epilogues:
+        if args.T == DEFAULT_T[args.workload]:
+            args.T = [1, 16, 128, 2048, 8192]
+        run_epilogues(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

@@ -236,6 +236,59 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
   }
 }
 
+// Wide form of the SwiGLU prep without RMSNorm when h is written out: one
+// elementwise pass over the whole tensor forms h = bf16(silu_bf16(gate) * up),
+// stores it and takes the device-wide max |h|; the strip quantizer then reads
+// h alone (from L2 when it fits).  Every thread works on independent 16-byte
+// vectors, two in flight, where the statistics kernel's row loop keeps too few
+// loads in flight to cover the SiLU's extra work.  h may alias up: each
+// element is read and then written by the same thread.
+constexpr int kEwThreads = 256;
+__global__ void __launch_bounds__(kEwThreads) prep_swiglu_h_kernel(
+    const __nv_bfloat16* __restrict__ G, const __nv_bfloat16* U, __nv_bfloat16* H, size_t n_vec, int T,
+    float* __restrict__ inv_rms, unsigned int* __restrict__ gmax_bits, int stats) {
+  __shared__ uint32_t wmax[kEwThreads / 32];
+  const uint4* g = reinterpret_cast<const uint4*>(G);
+  const uint4* u = reinterpret_cast<const uint4*>(U);
+  uint4* h = reinterpret_cast<uint4*>(H);
+  const size_t stride = (size_t)gridDim.x * kEwThreads;
+  size_t i = (size_t)blockIdx.x * kEwThreads + threadIdx.x;
+  uint32_t mx = 0;  // max |h| so far: bf16 bit patterns, one per half
+  auto fold = [&](const uint4& v) {
+    mx = vmax_u16x2(mx, v.x & 0x7FFF7FFFu);
+    mx = vmax_u16x2(mx, v.y & 0x7FFF7FFFu);
+    mx = vmax_u16x2(mx, v.z & 0x7FFF7FFFu);
+    mx = vmax_u16x2(mx, v.w & 0x7FFF7FFFu);
+  };
+  for (; i + stride < n_vec; i += 2 * stride) {
+    const uint4 a0 = g[i], b0 = u[i], a1 = g[i + stride], b1 = u[i + stride];
+    const uint4 h0 = epi8(a0, b0, kEpiSiluMul), h1 = epi8(a1, b1, kEpiSiluMul);
+    h[i] = h0;
+    h[i + stride] = h1;
+    fold(h0);
+    fold(h1);
+  }
+  if (i < n_vec) {
+    const uint4 h0 = epi8(g[i], u[i], kEpiSiluMul);
+    h[i] = h0;
+    fold(h0);
+  }
+  if (!stats) return;  // h only: the prep that follows takes its own statistics
+  for (size_t t = (size_t)blockIdx.x * kEwThreads + threadIdx.x; t < (size_t)T; t += stride) inv_rms[t] = 1.0f;
+  // CTA max -> device-wide max (non-negative floats order as their bits)
+  uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t cm = 0;
+#pragma unroll
+    for (int w = 0; w < kEwThreads / 32; ++w) cm = max(cm, wmax[w]);
+    if (cm) atomicMax(gmax_bits, cm << 16);
+  }
+}
+
 // Allow the next kernel in the stream (the GEMM, launched as a programmatic
 // dependent) to start its set-up and weight loads now; it waits for this
 // grid's completion (griddepcontrol.wait) before reading our outputs.
@@ -749,6 +802,24 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
     }
   }
 
+  // SwiGLU without RMSNorm, h written out, and a tensor that one cluster of
+  // the single-launch form holds (T <= 16 at K = 14336): h first, by the
+  // elementwise pass spread over many CTAs, then the prep of h alone -- each
+  // CTA of the single-launch form would otherwise evaluate its rows' SiLUs on
+  // one SM.
+  if (T > 0 && rs.kind == kEpiSiluMul && !Gb && rs.H && fused_runs_per_thread(K) != 0) {
+    const int tpr = (((K >> 3) / fused_runs_per_thread(K)) + 31) & ~31;
+    const int rpc = 512 / tpr > 0 ? 512 / tpr : 1;
+    if ((T + rpc - 1) / rpc <= kMaxClusterCtas) {
+      const size_t n_vec = (size_t)T * (size_t)(K >> 3);
+      const unsigned grid = (unsigned)((n_vec + kEwThreads - 1) / kEwThreads);
+      prep_swiglu_h_kernel<<<grid, kEwThreads, 0, stream>>>(Xb, rs.B, rs.H, n_vec, T, inv_rms, gmax_bits, 0);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      return launch_prep(rs.H, nullptr, eps, nullptr, T, Tp, K, kind, false, inv_rms, s_g, gmax_bits, sp_codes, meta,
+                         sp_sf, r_codes, r_sf, r_meta, kEpiNone, nullptr, nullptr, stream);
+    }
+  }
+
   if (T > 0) {
     bool launched = false;
     switch (kind) {
@@ -790,7 +861,14 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const bool g = Gb != nullptr;
   const int exact = eps < 0x1p-60f ? 1 : 0;
-  if (T > 0) {
+  if (T > 0 && rs.kind == kEpiSiluMul && !g && rs.H) {
+    // SwiGLU without RMSNorm, h written out: the elementwise first pass
+    const size_t n_vec = (size_t)T * (size_t)(K >> 3);
+    const int per_sm = resident_ctas(prep_swiglu_h_kernel, kEwThreads, dev);
+    long long grid = (long long)((n_vec + kEwThreads - 1) / kEwThreads);
+    if (grid > (long long)sms * per_sm) grid = (long long)sms * per_sm;
+    prep_swiglu_h_kernel<<<(unsigned)grid, kEwThreads, 0, stream>>>(Xb, rs.B, rs.H, n_vec, T, inv_rms, gmax_bits, 1);
+  } else if (T > 0) {
     auto rowstats_fn = g ? (rs.kind ? prep_rowstats_kernel<true, true> : prep_rowstats_kernel<true, false>)
                          : (rs.kind ? prep_rowstats_kernel<false, true> : prep_rowstats_kernel<false, false>);
     const int per_sm = resident_ctas(rowstats_fn, kRowThreads, dev);

@@ -96,6 +96,24 @@ def test_silu_prep_matches_oracle(T, K, out):
         assert bad.size == 0, f"{f}: {len(bad)} mismatches, first {bad[:4].tolist()}"
 
 
+@pytest.mark.parametrize("T,K", [(700, 14336), (16, 14336)])
+def test_silu_prep_h_may_alias_up(T, K):
+    """h written over up itself (the wide form's elementwise first pass and
+    the single-launch form): h is still the SwiGLU product, and the prepared
+    operands equal those of sharq_prep on it."""
+    g, u = _inputs(T, K, 3150 + T)
+    act = _act(T, K, sq.SHARQ_MODE_SHARQ)
+    ud = H.bf16_dev(u)
+    act.prep_silu_mul(H.bf16_dev(g), ud, ud, None, 1e-5)
+    ref = _act(T, K, sq.SHARQ_MODE_SHARQ)
+    hh = O.silu_mul(g, u)
+    ref.prep(H.bf16_dev(hh), None, 1e-5)
+    torch.cuda.synchronize()
+    assert np.array_equal(ud.float().cpu().numpy().view(np.uint32), hh.view(np.uint32))
+    n = ref.view.gmax_bits - 16 - ref.buf.data_ptr()   # operands and scales, not the per-row 1/rms scratch
+    assert torch.equal(act.buf[:n], ref.buf[:n])
+
+
 @pytest.mark.parametrize("T,K", [(16, 4096), (700, 8192)])
 def test_silu_dense_dense_mode_equals_prep_of_h(T, K):
     g, u = _inputs(T, K, 3200 + T)
