@@ -26,6 +26,7 @@ cudaError_t launch_linear(const uint8_t* a_sp, const uint8_t* a_meta, const uint
                           int* err, const int* act_err, cudaStream_t stream, const void* X_fused,
                           const void* gamma_fused, float eps_fused, bool per_token);
 int noalloc_max_rows();
+int split_max_clusters(int splits, bool fused);
 bool prep_per_token_supported(int K);
 cudaError_t launch_prep_noalloc(const void* X, const void* gamma, float eps, const int* row_index, int T, int Tp,
                                 int K, int kind, bool per_token, float* s_g, uint8_t* sp_codes, uint8_t* meta,
@@ -139,7 +140,7 @@ WeightLayout weight_layout(int K, int D, int E, int fmt = SHARQ_FMT_NVFP4) {
 struct GemmShape {
   int bn, splits, m_tiles, n_tiles;
 };
-GemmShape gemm_shape(int T, int K, int D, int E) {
+GemmShape gemm_shape(int T, int K, int D, int E, bool fused = false) {
   GemmShape g{};
   const int Tp = (int)round_up((size_t)T, 128);
   g.m_tiles = Tp / 128;
@@ -157,6 +158,13 @@ GemmShape gemm_shape(int T, int K, int D, int E) {
     int s = (int)(kTargetCtas / mn);
     s = s < 4 ? s : 4;
     s = s < KS ? s : KS;
+    // no second wave: as many clusters as the GPCs hold at once (36 clusters
+    // of 4 do not fit; 36 of 3 do)
+    while (s > 1) {
+      const int mc = sharq::split_max_clusters(s, fused);
+      if (mc == 0 || mn <= mc) break;
+      --s;
+    }
     g.splits = s > 1 ? s : 1;
   }
   return g;
@@ -431,7 +439,7 @@ int sharq_prep_linear(const void* d_X, const void* d_gamma, float eps, int T, co
   if (!d_ws || ws_bytes < sharq_workspace_bytes(T, w->K, w->D, 1) || !aligned(d_ws, 16)) return SHARQ_ERR_WORKSPACE;
   if ((st = check_device())) return st;
   if (T == 0) return SHARQ_OK;
-  const GemmShape g = gemm_shape(T, w->K, w->D, 1);
+  const GemmShape g = gemm_shape(T, w->K, w->D, 1, true);
   cudaError_t e = sharq::launch_linear(
       nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, T, (int)round_up((size_t)T, 128), w->K,
       0 /* SharQ operands */,

@@ -1854,6 +1854,42 @@ cudaError_t launch_cfg(const GemmArgs& a, int m_tiles, cudaStream_t stream) {
 
 }  // namespace
 
+// Clusters of the split-K decode kernel (1 x 1 x splits CTAs) that can be
+// resident at once on this device: clusters must fit within one GPC, so
+// clusters of 4 leave SMs of each GPC idle, and a grid with more clusters
+// than this runs in two waves.  Cached per device, form and split count;
+// 0 if the query fails.
+int split_max_clusters(int splits, bool fused) {
+  static int cache[64][2][5] = {};
+  int dev = 0;
+  if (splits < 2 || splits > 4 || cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 0;
+  int& c = cache[dev][fused ? 1 : 0][splits];
+  if (c == 0) {
+    auto fn = fused ? sharq_gemm_kernel<128, true, true> : sharq_gemm_kernel<128, true, false>;
+    const int smem = fused ? Cfg<128, true, true>::kSmemBytes : Cfg<128, true, false>::kSmemBytes;
+    const int threads = fused ? Cfg<128, true, true>::kThreadsT : Cfg<128, true, false>::kThreadsT;
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, splits);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = -1;
+    }
+    c = n;
+  }
+  return c > 0 ? c : 0;
+}
+
 // The CTA-pair prefill form is on unless the environment sets
 // SHARQ_GEMM_PAIR=0 (read once per process), which runs those shapes on the
 // one-CTA persistent kernel instead -- the same result, for comparing the two.
