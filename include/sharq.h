@@ -284,9 +284,9 @@ int sharq_prep_silu_mul(const void *d_gate, const void *d_up, void *d_h, const v
 
 /*
  * sharq_prep_noalloc - sharq_prep for callers that cannot allocate device
- * memory at run time: code inside a region being captured into a CUDA graph
- * (where cudaMalloc is not allowed), or a host framework whose memory
- * planner owns all device memory and hands out only the tensors it planned.
+ * memory: a host framework whose memory planner owns all device memory and
+ * hands out only the tensors it planned, or a serving loop that must not
+ * call cudaMalloc (it can synchronise the device and stall every stream).
  * The paper has no counterpart; this is a deployment variant of the same
  * computation, with results identical to sharq_prep's.
  * Differences from sharq_prep:
@@ -301,9 +301,9 @@ int sharq_prep_silu_mul(const void *d_gate, const void *d_up, void *d_h, const v
  *  - a->T > 16384 returns SHARQ_ERR_UNSUPPORTED_SHAPE.
  *  - The first call on each device looks the array's address up
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
- *  - Each call clears the array's counters with a 16-byte cudaMemsetAsync
- *    (no allocation).  All calls share the array: calls whose work overlaps
- *    on the GPU (different streams without ordering) race on it.
+ *  - Each call clears the array's counters and error words with a 32-byte
+ *    cudaMemsetAsync (no allocation).  All calls share the array: calls whose
+ *    work overlaps on the GPU (different streams without ordering) race on it.
  * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  */
 int sharq_prep_noalloc(const void *d_X, const void *d_gamma, float eps, const int *d_row_index,

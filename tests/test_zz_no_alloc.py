@@ -1,8 +1,9 @@
 """sharq_prep_noalloc: the allocation-free prep entry point (GPU).
 
-For callers that cannot allocate device memory at run time (graph-capture
-regions, runtimes whose memory planner owns the GPU), sharq_prep_noalloc keeps
-the prep's working memory in a fixed array inside the library.  Called through
+For callers that cannot allocate device memory (runtimes whose memory
+planner owns the GPU, serving loops that must not call cudaMalloc),
+sharq_prep_noalloc keeps the prep's working memory in a fixed array inside
+the library.  Called through
 the C ABI, it must give exactly sharq_prep's outputs -- and the oracle's, bit
 for bit on every row -- and keep doing so on the next call (the array keeps
 the previous call's contents).  The cases cover the single-launch form and the
