@@ -186,3 +186,29 @@ def test_pack_weight_bit_exact(K, D, E):
         _assert_equal("w sf32", sf32, q["sf32"])
         _assert_equal("w sf16", sf16, q["sf16"])
         assert pw.s_w()[e].item() == float(q["s_w"])
+
+
+@pytest.mark.parametrize("case", ["plain", "huge_gamma_on_zero_column", "mixed"])
+def test_wide_rowstats_edge_rows(case):
+    """The wide form (statistics launch, then the strip quantizer) against the
+    oracle on every row and on the stored 1/rms: ordinary rows; a gamma with
+    one huge entry (2^31) on a column that is zero in every row, which
+    changes no Xn; and zero rows and constant rows mixed in."""
+    T, K = 2048, 4096          # 2048 one-row CTAs do not fit at once: the wide form
+    x = synthetic.activations(811, T, K)
+    gamma = synthetic.gamma(812, K)
+    if case == "huge_gamma_on_zero_column":
+        x[:, 17] = 0.0
+        gamma[17] = np.float32(2.0 ** 31)
+    elif case == "mixed":
+        x[::7] = 0.0                                  # zero rows: P = 0
+        x[3::7] = np.float32(0.75)                    # constant rows: every product equal up to gamma
+        gamma[::2] = np.float32(1.0)
+    act = _gpu_prep(x, gamma, 1e-5)
+    got = _read(act, T, K, sq.SHARQ_MODE_SHARQ)
+    p = O.prep(x, gamma, 1e-5)
+    assert got["s_g"] == float(p["s_g"])
+    for f in ("meta", "sp_codes", "sp_sf", "r_codes", "r_sf"):
+        _assert_equal(f, got[f][:T], p[f])
+    inv = act.region("inv_rms", 4 * T).view(torch.float32).cpu().numpy()
+    assert np.array_equal(inv.view(np.uint32), p["inv"].view(np.uint32))
