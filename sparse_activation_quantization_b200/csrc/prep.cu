@@ -129,6 +129,9 @@ __global__ void __launch_bounds__(kRowThreads) prep_rowstats_kernel(
     unsigned int* __restrict__ gmax_bits, Epi rs) {
   constexpr int kC = kEpi ? kRowChunk / 2 : kRowChunk;  // vectors of the row in flight per lane
   __shared__ uint32_t wmax[kRowThreads / 32];
+  // the strip quantizer, launched as this grid's programmatic dependent, may
+  // start its set-up now; it waits for this grid before reading its results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = gridDim.x * (kRowThreads / 32);
   const int nv = K >> 3;  // 16-byte vectors per row
@@ -334,6 +337,9 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
   __shared__ float2 tab[128];
   __shared__ uint32_t msel[16];
   allow_dependents();
+  // launched as a programmatic dependent of the statistics grid: the max,
+  // 1/rms and (with an epilogue) h are read only once it has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float gmax = __uint_as_float(*(volatile const unsigned int*)gmax_bits);
   const float s = gmax > 0.0f ? __fdiv_rn(gmax, kGlobalDiv) : 1.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) *s_g_out = s;  // published even when there are no rows
@@ -904,8 +910,16 @@ cudaError_t launch_prep(const void* X, const void* gamma, float eps, const int* 
   if (rows > T) rows = T;
   const int nw = (int)(rows * G);  // 0 when T == 0: one CTA still publishes s_g
   const int grid = nw > 0 ? (nw + kStripThreads / 32 - 1) / (kStripThreads / 32) : 1;
-  strip_fn<<<grid, kStripThreads, 0, stream>>>(Xq, Gb, row_index, T, K, nw, inv_rms, gmax_bits, s_g, p, rq);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kStripThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = T > 0 ? 1 : 0;  // T == 0: no statistics launch precedes it
+  return cudaLaunchKernelEx(&cfg, strip_fn, Xq, Gb, row_index, T, K, nw, (const float*)inv_rms, gmax_bits, s_g, p, rq);
 }
 
 // ---------------------------------------------------------------------------

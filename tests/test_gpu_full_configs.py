@@ -4,7 +4,7 @@
   config 3  Llama-3.1-8B MLP prefill, T = 2048 and 8192: gate and up
             (4096 -> 14336 each, one shared RMSNorm prep), down 14336 -> 4096
             (Student-t input)
-  config 5  Qwen2.5-7B decoder-layer linears, T = 1, 1024 and 8192: qkv
+  config 5  Qwen2.5-7B decoder-layer linears, T = 1, 64, 1024 and 8192: qkv
             3584 -> 4608 and gate+up 3584 -> 37888 (RMSNorm), o 3584 -> 3584,
             down 18944 -> 3584 (Student-t input)
   config 4  Qwen3-30B-A3B experts: every expert with a non-empty group, every
@@ -130,7 +130,7 @@ QWEN = {"qkv": (3584, 4608, True), "o_proj": (3584, 3584, False), "gate_up": (35
         "down": (18944, 3584, False)}
 
 
-@pytest.mark.parametrize("T", [1, 1024, 8192])
+@pytest.mark.parametrize("T", [1, 64, 1024, 8192])
 @pytest.mark.parametrize("name", list(QWEN))
 def test_config5_qwen_layer_full(name, T):
     K, D, norm = QWEN[name]
