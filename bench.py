@@ -385,11 +385,13 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
 
     def prep(L, i):
-        acts[L.name].prep(xs[L.name][i], gammas[L.name], EPS, stream=stream)
+        x = xs[L.name]
+        acts[L.name].prep(x[i % len(x)], gammas[L.name], EPS, stream=stream)
 
     def gemm(L, i):
         src = L.shares or L.name
-        sq.linear(acts[src], weights[L.name][i], out=outs[L.name], ws=wss[L.name], stream=stream)
+        w = weights[L.name]
+        sq.linear(acts[src], w[i % len(w)], out=outs[L.name], ws=wss[L.name], stream=stream)
 
     FUSED_MAX_T = 32   # include/sharq.h SHARQ_FUSED_MAX_T: one-kernel prep+GEMM
 
@@ -401,7 +403,8 @@ def run_gpu(args, world, rank, local):
         """one whole layer through the public API: sharq_prep_linear where the
         prepared activation is not shared, else sharq_prep + sharq_linear"""
         if fused(L):
-            sq.prep_linear(xs[L.name][i], gammas[L.name], EPS, weights[L.name][i], out=outs[L.name],
+            x, w = xs[L.name], weights[L.name]
+            sq.prep_linear(x[i % len(x)], gammas[L.name], EPS, w[i % len(w)], out=outs[L.name],
                            ws=wss[L.name], stream=stream)
         else:
             if not L.shares:
@@ -449,11 +452,18 @@ def run_gpu(args, world, rank, local):
         assert wss[L.name].check(stream) == 0, "device-side error"
 
     # --- per-layer and per-kernel times -------------------------------------
+    # Back-to-back calls on one activation copy would find part of it in L2
+    # from the previous call (the quantizer walks the rows from the last one
+    # back), so the preps and layers alternate between at least two copies.
+    n_act = max(n_rot, 2)
+    for n in xs:
+        while len(xs[n]) < n_act:
+            xs[n].append(xs[n][0].clone())
     per = {}
     for L in layers:
         g_us = kernel_us(lambda i, L=L: gemm(L, i), n_rot, stream)
-        p_us = None if L.shares else kernel_us(lambda i, L=L: prep(L, i), n_rot, stream)
-        lay = kernel_us(lambda i, L=L: layer(L, i), n_rot, stream)
+        p_us = None if L.shares else kernel_us(lambda i, L=L: prep(L, i), n_act, stream)
+        lay = kernel_us(lambda i, L=L: layer(L, i), n_act, stream)
         per[L.name] = {"T": L.T, "K": L.K, "D": L.D, "fused": fused(L), "layer_us": lay, "gemm_us": g_us,
                        "prep_us": p_us,
                        "layer_tflops": L.flops / (lay * 1e-6) / 1e12,

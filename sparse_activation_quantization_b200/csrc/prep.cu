@@ -326,8 +326,9 @@ constexpr int kStripThreads = 256;
 
 // Wide form, second launch: one thread per 32-K strip of a row.  Warp w of
 // the grid owns strip group w % G (32 adjacent strips = 2 KB of a row, G
-// groups per row) and walks the rows w / G, w / G + nw / G, ... (nw, the
-// warps used, is a multiple of G), so its lanes load and unpack gamma once
+// groups per row) and walks the rows T - 1 - w / G, T - 1 - w / G - nw / G,
+// ... (nw, the warps used, is a multiple of G), so its lanes load and unpack
+// gamma once
 // and prefetch the next row's 64 bytes while quantizing the current one.
 template <bool kSharq, bool kGamma>
 __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
@@ -366,15 +367,19 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
       }
     }
     const uint4 z4 = make_uint4(0, 0, 0, 0);
+    // Rows are walked from the last one back: the statistics launch read the
+    // last rows most recently, so when X is larger than L2 the first rows
+    // this launch reads are still there.  t counts walked rows, T - 1 - t is
+    // the row.
     int t = gw / G;  // < T: the host uses at most T warps per strip group
-    int src = row_index ? row_index[t] : t;
+    int src = row_index ? row_index[T - 1 - t] : T - 1 - t;
     uint4 cur[4];
     float inv = 1.0f;
 #pragma unroll
     for (int u = 0; u < 4; ++u)
       cur[u] = (active && src >= 0) ? reinterpret_cast<const uint4*>(X + (size_t)src * K + 32 * (size_t)j)[u] : z4;
     if (rs.kind && active && src >= 0) apply_epi<4>(cur, (size_t)src * K + 32 * (size_t)j, rs);
-    if (kGamma) inv = inv_rms[t];
+    if (kGamma) inv = inv_rms[T - 1 - t];
     while (t < T) {
       // prefetch the next row of this warp
       const int tn = t + rstride;
@@ -382,13 +387,13 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
       uint4 nxt[4] = {z4, z4, z4, z4};
       float invn = 1.0f;
       if (tn < T) {
-        srcn = row_index ? row_index[tn] : tn;
+        srcn = row_index ? row_index[T - 1 - tn] : T - 1 - tn;
         if (active && srcn >= 0) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) nxt[u] = reinterpret_cast<const uint4*>(X + (size_t)srcn * K + 32 * (size_t)j)[u];
           if (rs.kind) apply_epi<4>(nxt, (size_t)srcn * K + 32 * (size_t)j, rs);
         }
-        if (kGamma) invn = inv_rms[tn];
+        if (kGamma) invn = inv_rms[T - 1 - tn];
       }
       if (active) {
         f2_t P[16];
@@ -404,7 +409,7 @@ __global__ void __launch_bounds__(kStripThreads) prep_strip_kernel(
 #pragma unroll
           for (int i = 0; i < 16; ++i) P[i] = f2_norm(P[i], inv2, gm[i]);
         }
-        quant_strip<kSharq>(P, t, j, KS, ctx, out);
+        quant_strip<kSharq>(P, T - 1 - t, j, KS, ctx, out);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
