@@ -479,26 +479,57 @@ def run_gpu(args, world, rank, local):
     h2d = sum(hx[n].numel() * 2 for n in hx)
     d2h = sum(hy[n].numel() * 2 for n in hy)
 
+    # The copies run on two streams of their own, so that the host link (the
+    # bound here: ~1.5 GB per step) carries both directions at once and
+    # overlaps the kernels; events keep each buffer's reuse in order (a step's
+    # input copy waits for the previous step's prep of that input, a GEMM for
+    # the previous step's read-back of its output).
+    cs_in, cs_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = {n: torch.cuda.Event() for n in xs}            # input on the device
+    ev_used = {n: torch.cuda.Event() for n in xs}          # input read by its prep
+    ev_out = {L.name: torch.cuda.Event() for L in layers}  # output written
+    ev_read = {L.name: torch.cuda.Event() for L in layers}  # output copied to the host
+    seen = set()
+
     def e2e_step(i):
         for L in layers:
             if not L.shares:
-                dx[L.name].copy_(hx[L.name], non_blocking=True)
+                with torch.cuda.stream(cs_in):
+                    if L.name in seen:
+                        cs_in.wait_event(ev_used[L.name])
+                    dx[L.name].copy_(hx[L.name], non_blocking=True)
+                    ev_in[L.name].record(cs_in)
+                stream.wait_event(ev_in[L.name])
+            if L.name in seen:
+                stream.wait_event(ev_read[L.name])
             if fused(L):
-                sq.prep_linear(dx[L.name], gammas[L.name], EPS, weights[L.name][i], out=outs[L.name],
+                w = weights[L.name]
+                sq.prep_linear(dx[L.name], gammas[L.name], EPS, w[i % len(w)], out=outs[L.name],
                                ws=wss[L.name], stream=stream)
+                ev_used[L.name].record(stream)
             else:
                 if not L.shares:
                     acts[L.name].prep(dx[L.name], gammas[L.name], EPS, stream=stream)
+                    ev_used[L.name].record(stream)
                 gemm(L, i)
-            hy[L.name].copy_(outs[L.name], non_blocking=True)
+            ev_out[L.name].record(stream)
+            with torch.cuda.stream(cs_out):
+                cs_out.wait_event(ev_out[L.name])
+                hy[L.name].copy_(outs[L.name], non_blocking=True)
+                ev_read[L.name].record(cs_out)
+            seen.add(L.name)
     for i in range(3):
         e2e_step(i % n_rot)
     torch.cuda.synchronize()
     e2e_steps = max(3, min(args.steps, 50))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    cs_in.wait_stream(stream)
+    cs_out.wait_stream(stream)
     for k in range(e2e_steps):
         e2e_step(k % n_rot)
+    stream.wait_stream(cs_in)
+    stream.wait_stream(cs_out)
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
