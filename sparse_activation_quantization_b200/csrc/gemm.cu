@@ -31,6 +31,8 @@
 //               copy's completion takes a good fraction of a microsecond);
 //               each copy warp commits to the slot's mbarrier, which the MMA
 //               thread waits on.
+// Prefill shapes with at least two 128-row tiles run on CTA pairs instead
+// (tcgen05 cta_group::2, 256 x 256 tiles; roles at sharq_gemm_pair_kernel).
 // Split-K (decode shapes, where output tiles alone cannot fill 148 SMs):
 // the S CTAs that share an output tile form one thread-block cluster
 // (1 x 1 x S); each takes a contiguous range of K stages.  CTA r of the
