@@ -300,7 +300,7 @@ int sharq_prep_silu_mul(const void *d_gate, const void *d_up, void *d_h, const v
  *    on that view has no prep error word to forward.
  *  - a->T > 16384 returns SHARQ_ERR_UNSUPPORTED_SHAPE.
  *  - The first call on each device looks the array's address up
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    (cudaGetSymbolAddress, a host-side query that allocates nothing).
  *  - Each call clears the array's counters and error words with a 32-byte
  *    cudaMemsetAsync (no allocation).  All calls share the array: calls whose
  *    work overlaps on the GPU (different streams without ordering) race on it.
