@@ -53,9 +53,9 @@ def gemm_alg_bytes(T, K, D):
 
 
 def prep_alg_bytes(T, K):
-    """bf16 read (2 B) + outputs (0.90625 B) per element."""
-    Tp = -(-T // 128) * 128
-    return T * K * 2 + Tp * K * 0.90625
+    """bf16 read (2 B) + outputs (0.90625 B) per activation element; the
+    tile-padding rows T..Tp-1 are neither read nor written."""
+    return T * K * (2 + 0.90625)
 
 
 def gemm_split_k(L):
